@@ -1,0 +1,172 @@
+/*
+ * int8mm.h — C ABI of libint8mm.so, the B200 (sm_100a) LLM.int8()
+ * mixed-precision decomposed matmul
+ *
+ *     Y = X W,   X fp16 [M,K] (activations),  W fp16 [K,N] (weights)
+ *
+ * computed as in "LLM.int8(): 8-bit Matrix Multiplication for Transformers at
+ * Scale" (Dettmers et al., 2022), following these web pages about it:
+ *   "LLM.int8() — 大模型激活值里藏着几个超大异常通道" (estelledc.github.io),
+ *       方法1 (vector-wise quantisation) and 方法2 (mixed-precision decomposition);
+ *   "AI 十大核心论文解读: LLM.int8()" (developer.aliyun.com), §2.2 and the
+ *       Fig. 2 caption;
+ *   "LLM.int8()" (brain.gartu.xyz), "La solution", "Seuil de détection α",
+ *       "Vector-wise INT8 Quantization".
+ *
+ *  1. O = { j : max_i |X[i,j]| > alpha }   (outlier feature columns; strict >)
+ *  2. c_x[i] = 127 / max_{j not in O} |X[i,j]|,  Xq[i,j] = rne(X[i,j] c_x[i])
+ *     for j not in O and 0 for j in O;  c_w[j] = 127 / max_k |W[k,j]| over all
+ *     K rows,  Wq[k,j] = rne(W[k,j] c_w[j]).  Codes are clamped to [-127, 127],
+ *     rne rounds an fp32 product to the nearest integer, ties to even; an
+ *     all-zero vector gets scale 0 and codes 0.
+ *  3. Acc = Xq Wq  (int8 x int8 -> int32, exact)
+ *  4. Y[i,j] = fp16( Acc[i,j] / (c_x[i] c_w[j]) + sum_{k in O} X[i,k] W[k,j] )
+ *     with the fp16 outlier product accumulated in fp32.
+ *
+ * Every pointer argument named *_dev is a device pointer on the current CUDA
+ * device; `stream` is a cudaStream_t (NULL = the legacy default stream).
+ * All work is enqueued on `stream`; no call below synchronises the host
+ * unless its comment says so.  The library never frees caller memory.
+ * A handle is not safe for concurrent use from several host threads.
+ *
+ * Errors: argument errors are detected on the host before anything is
+ * enqueued; they return a non-zero status and set int8mm_last_error().
+ * A CUDA launch or allocation error returns INT8MM_ERR_CUDA (or
+ * INT8MM_ERR_OOM).  A device-side wait that exceeded its time limit is
+ * reported later through int8mm_get_status().  NaN or Inf in X or W gives an
+ * unspecified Y (the pages assume finite activations); it is not checked.
+ */
+#ifndef INT8MM_H
+#define INT8MM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct int8mm_weight* int8mm_weight_t; /* opaque, owned by the library */
+
+typedef enum {
+  INT8MM_OK = 0,
+  INT8MM_ERR_INVALID_ARG = 1,       /* null pointer, bad size, NaN alpha, freed handle */
+  INT8MM_ERR_UNSUPPORTED_SHAPE = 2, /* K or N not a multiple of 16, K > 65536, ... */
+  INT8MM_ERR_ALIGNMENT = 3,         /* a pointer not 16-byte aligned */
+  INT8MM_ERR_OOM = 4,               /* device allocation failed */
+  INT8MM_ERR_CUDA = 5,              /* a CUDA runtime/driver call failed */
+  INT8MM_ERR_TIMEOUT = 6            /* a device wait ran out of time (see get_status) */
+} int8mm_status;
+
+/* Shape limits: 16 <= K <= 65536 with K % 16 == 0 (K <= 133144 keeps the
+ * int32 accumulator exact; the row kernel holds a row in registers up to
+ * 65536); 16 <= N < 2^31 with N % 16 == 0; 0 <= M < 2^31. */
+#define INT8MM_MAX_K 65536
+
+/*
+ * Prepare a weight (step 2 for W; "LLM.int8() — 大模型激活值里藏着几个超大异常通道",
+ * 方法1: one normalisation constant per column of the weight matrix).
+ *
+ * W_fp16_dev: [K, N] fp16, row-major, 16-byte aligned.  BORROWED for the
+ *   life of the handle: forward calls read its rows W[O,:] for the fp16
+ *   outlier product, so it must stay valid and unchanged until int8mm_free.
+ * On success *out receives a handle that owns the int8 codes Wq^T [N, K]
+ * (K-major), c_w [N], the TMA descriptors and a workspace that grows with M.
+ * Enqueued on `stream`; the handle may be used on any stream ordered after it.
+ */
+int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N, void* stream,
+                                    int8mm_weight_t* out);
+
+/*
+ * Pre-size the per-forward workspace for up to M_max rows, so that later
+ * forward calls with M <= M_max allocate nothing (needed before CUDA graph
+ * capture of a forward).  Stream-ordered allocation on `stream`.
+ */
+int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream);
+
+/*
+ * Forward (steps 1-4; "LLM.int8() — 大模型激活值里藏着几个超大异常通道", 方法2:
+ * Y = X_int8 W_int8 / scales + X_fp16 W_fp16; the Fig. 2 caption of the
+ * AI 十大核心论文解读 article).
+ *
+ * X_fp16_dev: [M, K] fp16 row-major, 16-byte aligned, read-only.
+ * Y_fp16_dev: [M, N] fp16 row-major, 16-byte aligned, written.
+ * alpha: outlier threshold (6.0 in the pages); INFINITY disables the fp16
+ *   path (pure vector-wise int8); any value below every |x| makes every
+ *   column an outlier.  NaN is an argument error.
+ * M == 0 is a no-op.  Three kernels run on `stream` (outlier detection, row
+ * quantisation, fused int8 GEMM); the outlier count never leaves the device,
+ * so the call does not synchronise.  Grows the workspace when M exceeds
+ * every earlier M (stream-ordered allocation).
+ */
+int8mm_status int8mm_forward(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
+                             void* Y_fp16_dev, void* stream);
+
+/*
+ * Same as int8mm_forward for host-resident X and Y: copies X_fp16_host
+ * [M, K] into a handle-owned device buffer, runs the forward, and copies Y
+ * back into Y_fp16_host [M, N], all enqueued on `stream`.  Y_fp16_host is
+ * valid once `stream` has been synchronised.  Use page-locked host memory
+ * for the copies to be asynchronous.
+ */
+int8mm_status int8mm_forward_host(int8mm_weight_t h, const void* X_fp16_host, int64_t M, float alpha,
+                                  void* Y_fp16_host, void* stream);
+
+/*
+ * Same as int8mm_forward, and records four caller-created CUDA events
+ * (cudaEvent_t, passed as void*) on `stream`: before the outlier pass,
+ * between it and the row pass, between the row pass and the GEMM, and after
+ * the GEMM, so that each kernel can be timed on its own stream.
+ */
+int8mm_status int8mm_forward_events(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
+                                    void* Y_fp16_dev, void* stream, void* const events[4]);
+
+/* Intermediate values of one forward, for verification.  Every field is a
+ * device pointer or NULL (not written). */
+typedef struct int8mm_debug_bufs {
+  float* colmax;          /* [K]    max_i |X[i,j]| (fp32, exact) */
+  int32_t* outlier_idx;   /* [K]    ascending outlier columns; first *count valid */
+  int32_t* outlier_count; /* [1]    |O| */
+  int8_t* x_codes;        /* [M, K] int8 codes of X, outlier columns 0 */
+  float* c_x;             /* [M]    row scales */
+  int8_t* w_codes_t;      /* [N, K] int8 codes of W, transposed (K-major) */
+  float* c_w;             /* [N]    column scales */
+  int32_t* acc;           /* [M, N] int32 accumulators Xq Wq */
+} int8mm_debug_bufs;
+
+/* Forward that also copies the intermediates into `dbg` (stream-ordered).
+ * Filling `acc` makes the GEMM epilogue write the raw accumulators too. */
+int8mm_status int8mm_forward_debug(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
+                                   void* Y_fp16_dev, void* stream, const int8mm_debug_bufs* dbg);
+
+/*
+ * Device status word of the handle: INT8MM_OK, or INT8MM_ERR_TIMEOUT if a
+ * kernel of an earlier forward gave up on a wait (the outputs of that
+ * forward are then incomplete).  SYNCHRONISES the device, then clears the
+ * word.  Also returns INT8MM_ERR_CUDA if the device reports an error.
+ */
+int8mm_status int8mm_get_status(int8mm_weight_t h);
+
+/*
+ * Time limit, in nanoseconds, for each device-side wait of later forwards
+ * (default 2e9, i.e. two seconds).  Diagnostic: a tiny limit makes waits
+ * give up early and report INT8MM_ERR_TIMEOUT through int8mm_get_status.
+ */
+int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns);
+
+/* Device bytes held by the handle (codes, scales, workspace). */
+int8mm_status int8mm_weight_bytes(int8mm_weight_t h, size_t* bytes);
+
+/* Release the handle and everything it owns.  SYNCHRONISES the device
+ * first, so no enqueued forward still uses the memory.  NULL or an already
+ * freed handle is a no-op. */
+void int8mm_free(int8mm_weight_t h);
+
+/* Message of the last error returned on this host thread ("" if none). */
+const char* int8mm_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INT8MM_H */

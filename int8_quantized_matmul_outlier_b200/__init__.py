@@ -1,0 +1,224 @@
+"""Python binding of libint8mm.so, the sm_100a LLM.int8() decomposed matmul.
+
+Argument marshalling only: every function below passes device pointers,
+sizes and a CUDA stream to the C ABI declared in ``include/int8mm.h`` and
+raises ``Int8mmError`` on a non-zero status.  All arithmetic runs in the
+library's CUDA kernels; there is no fallback, and importing this package
+fails loudly when the library has not been built.
+
+PyTorch is used only to pass device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+LIB_PATH = _build.LIB
+
+INT8MM_OK = 0
+INT8MM_ERR_INVALID_ARG = 1
+INT8MM_ERR_UNSUPPORTED_SHAPE = 2
+INT8MM_ERR_ALIGNMENT = 3
+INT8MM_ERR_OOM = 4
+INT8MM_ERR_CUDA = 5
+INT8MM_ERR_TIMEOUT = 6
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_SHAPE", 3: "ALIGNMENT", 4: "OOM",
+                5: "CUDA", 6: "TIMEOUT"}
+MAX_K = 65536
+
+# Symbols of include/int8mm.h and their ctypes signatures.
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_ST = ctypes.c_int
+SIGNATURES = {
+    "int8mm_prepare_weight": (_ST, [_P, _I64, _I64, _P, ctypes.POINTER(_P)]),
+    "int8mm_reserve": (_ST, [_P, _I64, _P]),
+    "int8mm_forward": (_ST, [_P, _P, _I64, ctypes.c_float, _P, _P]),
+    "int8mm_forward_host": (_ST, [_P, _P, _I64, ctypes.c_float, _P, _P]),
+    "int8mm_forward_events": (_ST, [_P, _P, _I64, ctypes.c_float, _P, _P, ctypes.POINTER(_P)]),
+    "int8mm_forward_debug": (_ST, [_P, _P, _I64, ctypes.c_float, _P, _P, _P]),
+    "int8mm_get_status": (_ST, [_P]),
+    "int8mm_set_wait_limit": (_ST, [_P, ctypes.c_uint64]),
+    "int8mm_weight_bytes": (_ST, [_P, ctypes.POINTER(ctypes.c_size_t)]),
+    "int8mm_free": (None, [_P]),
+    "int8mm_last_error": (ctypes.c_char_p, []),
+}
+
+
+class DebugBufs(ctypes.Structure):
+    """Mirror of ``int8mm_debug_bufs`` (all device pointers, NULL = skip)."""
+
+    _fields_ = [("colmax", _P), ("outlier_idx", _P), ("outlier_count", _P), ("x_codes", _P),
+                ("c_x", _P), ("w_codes_t", _P), ("c_w", _P), ("acc", _P)]
+
+
+class Int8mmError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"int8mm status {status} ({STATUS_NAMES.get(status, '?')}): {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libint8mm.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -c 'import __graft_entry__ as g; g.build()'`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def int8mm_last_error() -> str:
+    return lib().int8mm_last_error().decode()
+
+
+def _check(status: int) -> None:
+    if status != INT8MM_OK:
+        raise Int8mmError(status, int8mm_last_error())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _dev_f16_2d(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not (t.is_cuda and t.dtype == torch.float16 and t.dim() == 2 and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous 2-D float16 CUDA tensor")
+    return t
+
+
+class Weight:
+    """A prepared weight (the library-owned handle).  Keeps a reference to
+    the borrowed fp16 weight so that it outlives the handle."""
+
+    def __init__(self, handle: int, W: torch.Tensor):
+        self.handle = handle
+        self.W = W
+        self.K, self.N = W.shape
+
+    def __del__(self):
+        h, self.handle = getattr(self, "handle", None), None
+        if h and _lib is not None:
+            _lib.int8mm_free(h)
+
+
+def int8mm_prepare_weight(W: torch.Tensor, stream=None) -> Weight:
+    _dev_f16_2d(W, "W")
+    K, N = W.shape
+    out = _P()
+    _check(lib().int8mm_prepare_weight(W.data_ptr(), K, N, _stream(stream), ctypes.byref(out)))
+    return Weight(out.value, W)
+
+
+def int8mm_reserve(w: Weight, M_max: int, stream=None) -> None:
+    _check(lib().int8mm_reserve(w.handle, int(M_max), _stream(stream)))
+
+
+def int8mm_forward(w: Weight, X: torch.Tensor, alpha: float = 6.0, Y: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    _dev_f16_2d(X, "X")
+    M = X.shape[0]
+    if X.shape[1] != w.K:
+        raise ValueError(f"X has {X.shape[1]} columns, the weight has K={w.K}")
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.float16, device=X.device)
+    _dev_f16_2d(Y, "Y")
+    _check(lib().int8mm_forward(w.handle, X.data_ptr(), M, float(alpha), Y.data_ptr(), _stream(stream)))
+    return Y
+
+
+def int8mm_forward_host(w: Weight, X: torch.Tensor, alpha: float = 6.0, Y: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """X and Y are host (CPU) float16 tensors; pin them for asynchronous copies.
+    Y is valid after the stream is synchronised."""
+    if X.is_cuda or X.dtype != torch.float16 or not X.is_contiguous() or X.dim() != 2:
+        raise ValueError("X must be a contiguous 2-D float16 CPU tensor")
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.float16, pin_memory=X.is_pinned())
+    _check(lib().int8mm_forward_host(w.handle, X.data_ptr(), M, float(alpha), Y.data_ptr(), _stream(stream)))
+    return Y
+
+
+def _event_handle(ev: torch.cuda.Event, stream) -> int:
+    if not ev.cuda_event:
+        ev.record(stream)  # torch creates the CUDA event on its first record
+    return ev.cuda_event
+
+
+def int8mm_forward_events(w: Weight, X: torch.Tensor, alpha: float, Y: torch.Tensor, events, stream=None):
+    """Forward that records the 4 given torch.cuda.Events (timing enabled) around
+    its three kernels on the launch stream."""
+    _dev_f16_2d(X, "X")
+    _dev_f16_2d(Y, "Y")
+    s = stream if stream is not None else torch.cuda.current_stream()
+    arr = (_P * 4)(*[_event_handle(e, s) for e in events])
+    _check(lib().int8mm_forward_events(w.handle, X.data_ptr(), X.shape[0], float(alpha), Y.data_ptr(),
+                                       _stream(s), arr))
+    return Y
+
+
+def int8mm_forward_debug(w: Weight, X: torch.Tensor, alpha: float = 6.0, Y: torch.Tensor | None = None,
+                         stream=None, want_acc: bool = True) -> dict:
+    """Forward plus its intermediates as device tensors: colmax, outlier_idx
+    (trimmed to the count), x_codes, c_x, w_codes_t, c_w and (if asked) acc."""
+    _dev_f16_2d(X, "X")
+    M, K = X.shape
+    N = w.N
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    out = dict(
+        colmax=torch.empty(K, dtype=torch.float32, device=dev),
+        outlier_idx=torch.empty(K, dtype=torch.int32, device=dev),
+        outlier_count=torch.empty(1, dtype=torch.int32, device=dev),
+        x_codes=torch.empty((M, K), dtype=torch.int8, device=dev),
+        c_x=torch.empty(M, dtype=torch.float32, device=dev),
+        w_codes_t=torch.empty((N, K), dtype=torch.int8, device=dev),
+        c_w=torch.empty(N, dtype=torch.float32, device=dev),
+        acc=torch.empty((M, N), dtype=torch.int32, device=dev) if want_acc else None,
+    )
+    d = DebugBufs(*[(t.data_ptr() if t is not None else None) for t in
+                    (out["colmax"], out["outlier_idx"], out["outlier_count"], out["x_codes"],
+                     out["c_x"], out["w_codes_t"], out["c_w"], out["acc"])])
+    _check(lib().int8mm_forward_debug(w.handle, X.data_ptr(), M, float(alpha), Y.data_ptr(),
+                                      _stream(stream), ctypes.byref(d)))
+    out["Y"] = Y
+    return out
+
+
+def int8mm_get_status(w: Weight) -> int:
+    """Synchronises the device; returns the status code (does not raise)."""
+    return int(lib().int8mm_get_status(w.handle))
+
+
+def int8mm_set_wait_limit(w: Weight, timeout_ns: int) -> None:
+    _check(lib().int8mm_set_wait_limit(w.handle, int(timeout_ns)))
+
+
+def int8mm_weight_bytes(w: Weight) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().int8mm_weight_bytes(w.handle, ctypes.byref(n)))
+    return int(n.value)
+
+
+def int8mm_free(w: Weight) -> None:
+    h, w.handle = w.handle, None
+    if h:
+        lib().int8mm_free(h)
+

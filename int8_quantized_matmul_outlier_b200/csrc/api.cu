@@ -1,0 +1,456 @@
+// C ABI of libint8mm.so (declared in include/int8mm.h): weight handles, the
+// per-forward workspace, TMA descriptors, argument checks and the launch
+// sequence of the decomposed int8 matmul.
+#include "int8mm.h"
+#include "kernels.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_set>
+
+using namespace i8mm;
+
+struct int8mm_weight {
+  int device = 0;
+  int num_sms = 148;
+  int64_t K = 0, N = 0;
+  const __half* W = nullptr;  // borrowed fp16 weight [K, N]
+  int8_t* Wq_t = nullptr;     // [N, K] int8 codes, K-major
+  float* c_w = nullptr;       // [N]
+  float* inv_cw = nullptr;    // [N]
+  uint32_t* colmax_bits = nullptr;  // [N] prep scratch
+  CUtensorMap tmB;
+  // fixed-size scratch of the outlier pass
+  unsigned* stripe_ticket = nullptr;
+  unsigned* all_ticket = nullptr;
+  uint32_t* mask = nullptr;
+  int32_t* idx = nullptr;
+  int32_t* count = nullptr;
+  float* colmax = nullptr;
+  int* status = nullptr;
+  // workspace sized by the largest M seen
+  int64_t ws_rows = 0;
+  int8_t* Xq = nullptr;
+  float* c_x = nullptr;
+  __half* X_OT = nullptr;
+  uint16_t* partial = nullptr;
+  // tensor map of Xq for the current (pointer, M)
+  CUtensorMap tmA;
+  const void* tmA_ptr = nullptr;
+  int64_t tmA_rows = -1;
+  // device copies for host-buffer forwards
+  int64_t io_rows = 0;
+  __half* dX = nullptr;
+  __half* dY = nullptr;
+  unsigned long long timeout_ns = 2000000000ull;
+  size_t bytes = 0;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+std::mutex g_mu;
+std::unordered_set<const int8mm_weight*> g_live;
+
+int8mm_status fail(int8mm_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int8mm_status fail(int8mm_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+int8mm_status cuda_fail(cudaError_t e, const char* what) {
+  const int8mm_status s = (e == cudaErrorMemoryAllocation) ? INT8MM_ERR_OOM : INT8MM_ERR_CUDA;
+  return fail(s, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool live(const int8mm_weight* h) {
+  std::lock_guard<std::mutex> g(g_mu);
+  return h != nullptr && g_live.count(h) != 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D int8 tensor [outer, inner] (inner contiguous), 128-byte swizzled boxes
+// of box_inner x box_outer elements, zero fill outside the tensor.
+int8mm_status make_tmap_i8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                           uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return fail(INT8MM_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(INT8MM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return INT8MM_OK;
+}
+
+template <typename T>
+cudaError_t alloc(T** p, size_t count, cudaStream_t s, size_t* total) {
+  *p = nullptr;
+  if (count == 0) count = 1;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(p), count * sizeof(T), s);
+  if (e == cudaSuccess && total) *total += count * sizeof(T);
+  return e;
+}
+
+template <typename T>
+void release(T** p) {
+  if (*p) cudaFree(*p);
+  *p = nullptr;
+}
+
+void free_workspace(int8mm_weight* h) {
+  release(&h->Xq);
+  release(&h->c_x);
+  release(&h->X_OT);
+  release(&h->partial);
+  h->ws_rows = 0;
+  h->tmA_ptr = nullptr;
+  h->tmA_rows = -1;
+}
+
+void free_all(int8mm_weight* h) {
+  free_workspace(h);
+  release(&h->dX);
+  release(&h->dY);
+  release(&h->Wq_t);
+  release(&h->c_w);
+  release(&h->inv_cw);
+  release(&h->colmax_bits);
+  release(&h->stripe_ticket);
+  release(&h->all_ticket);
+  release(&h->mask);
+  release(&h->idx);
+  release(&h->count);
+  release(&h->colmax);
+  release(&h->status);
+}
+
+size_t ws_bytes(const int8mm_weight* h, int64_t rows) {
+  const int chunks = outlier_row_chunks_bound(rows, h->K, h->num_sms);
+  return static_cast<size_t>(rows) * h->K                  // Xq
+         + static_cast<size_t>(rows) * 4                   // c_x
+         + static_cast<size_t>(rows) * h->K * 2            // X_OT
+         + static_cast<size_t>(chunks) * h->K * 2;         // partial
+}
+
+int8mm_status ensure_workspace(int8mm_weight* h, int64_t M, cudaStream_t s) {
+  if (M <= h->ws_rows) return INT8MM_OK;
+  int64_t rows = std::max<int64_t>(M, 2 * h->ws_rows);
+  rows = std::max<int64_t>(rows, 128);
+  // The old buffers may still be read by kernels enqueued earlier: free in
+  // stream order on the same stream.
+  if (h->ws_rows) {
+    cudaFreeAsync(h->Xq, s);
+    cudaFreeAsync(h->c_x, s);
+    cudaFreeAsync(h->X_OT, s);
+    cudaFreeAsync(h->partial, s);
+    h->bytes -= ws_bytes(h, h->ws_rows);
+    h->Xq = nullptr;
+    h->c_x = nullptr;
+    h->X_OT = nullptr;
+    h->partial = nullptr;
+    h->ws_rows = 0;
+  }
+  const int chunks = outlier_row_chunks_bound(rows, h->K, h->num_sms);
+  cudaError_t e;
+  if ((e = alloc(&h->Xq, static_cast<size_t>(rows) * h->K, s, nullptr)) != cudaSuccess ||
+      (e = alloc(&h->c_x, static_cast<size_t>(rows), s, nullptr)) != cudaSuccess ||
+      (e = alloc(&h->X_OT, static_cast<size_t>(rows) * h->K, s, nullptr)) != cudaSuccess ||
+      (e = alloc(&h->partial, static_cast<size_t>(chunks) * h->K, s, nullptr)) != cudaSuccess) {
+    cudaStreamSynchronize(s);
+    free_workspace(h);
+    return cuda_fail(e, "workspace allocation");
+  }
+  h->ws_rows = rows;
+  h->bytes += ws_bytes(h, rows);
+  h->tmA_ptr = nullptr;
+  h->tmA_rows = -1;
+  return INT8MM_OK;
+}
+
+int8mm_status check_forward_args(const int8mm_weight* h, const void* X, int64_t M, float alpha, const void* Y) {
+  if (!live(h)) return fail(INT8MM_ERR_INVALID_ARG, "invalid or freed weight handle");
+  if (M < 0 || M >= (int64_t(1) << 31)) return fail(INT8MM_ERR_INVALID_ARG, "M=%lld out of range", (long long)M);
+  if (std::isnan(alpha)) return fail(INT8MM_ERR_INVALID_ARG, "alpha is NaN");
+  if (M == 0) return INT8MM_OK;
+  if (X == nullptr || Y == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "X or Y is NULL");
+  const int64_t tiles = ((M + kGemmBM - 1) / kGemmBM) * ((h->N + kGemmBN - 1) / kGemmBN);
+  if (tiles >= (int64_t(1) << 31) || M * h->N >= (int64_t(1) << 62))
+    return fail(INT8MM_ERR_UNSUPPORTED_SHAPE, "M=%lld x N=%lld is too large", (long long)M, (long long)h->N);
+  if (!aligned16(X) || !aligned16(Y)) return fail(INT8MM_ERR_ALIGNMENT, "X and Y must be 16-byte aligned");
+  return INT8MM_OK;
+}
+
+int8mm_status set_device(const int8mm_weight* h) {
+  int cur = -1;
+  cudaGetDevice(&cur);
+  if (cur != h->device) {
+    cudaError_t e = cudaSetDevice(h->device);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  }
+  return INT8MM_OK;
+}
+
+int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alpha, void* Y, cudaStream_t s,
+                           void* const* events, const int8mm_debug_bufs* dbg) {
+  int8mm_status st = check_forward_args(h, X, M, alpha, Y);
+  if (st != INT8MM_OK) return st;
+  if (M == 0) return INT8MM_OK;
+  if ((st = set_device(h)) != INT8MM_OK) return st;
+  if ((st = ensure_workspace(h, M, s)) != INT8MM_OK) return st;
+  if (h->tmA_ptr != h->Xq || h->tmA_rows != M) {
+    if ((st = make_tmap_i8(&h->tmA, h->Xq, h->K, M, kGemmBK, kGemmBM)) != INT8MM_OK) return st;
+    h->tmA_ptr = h->Xq;
+    h->tmA_rows = M;
+  }
+  OutlierScratch sc{h->partial, h->stripe_ticket, h->all_ticket, h->mask, h->idx, h->count, h->colmax};
+  const __half* Xh = static_cast<const __half*>(X);
+  cudaError_t e;
+  auto rec = [&](int i) {
+    if (events && events[i]) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
+  };
+  rec(0);
+  if ((e = launch_outlier_detect(Xh, M, h->K, alpha, sc, h->num_sms, s)) != cudaSuccess)
+    return cuda_fail(e, "outlier detection launch");
+  rec(1);
+  if ((e = launch_row_quant(Xh, M, h->K, sc, h->Xq, h->c_x, h->X_OT, s)) != cudaSuccess)
+    return cuda_fail(e, "row quantisation launch");
+  rec(2);
+  GemmArgs a;
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(h->N);
+  a.K = static_cast<int>(h->K);
+  a.c_x = h->c_x;
+  a.inv_cw = h->inv_cw;
+  a.W = h->W;
+  a.X_OT = h->X_OT;
+  a.idx = h->idx;
+  a.count = h->count;
+  a.Y = static_cast<__half*>(Y);
+  a.acc_dump = dbg ? dbg->acc : nullptr;
+  a.status = h->status;
+  a.timeout_ns = h->timeout_ns;
+  if ((e = launch_gemm_decomp(h->tmA, h->tmB, a, h->num_sms, s)) != cudaSuccess)
+    return cuda_fail(e, "int8 GEMM launch");
+  rec(3);
+  if (dbg) {
+    const size_t K = static_cast<size_t>(h->K), N = static_cast<size_t>(h->N), Mz = static_cast<size_t>(M);
+    struct C {
+      void* dst;
+      const void* src;
+      size_t n;
+    } cps[] = {
+        {dbg->colmax, h->colmax, K * 4},  {dbg->outlier_idx, h->idx, K * 4}, {dbg->outlier_count, h->count, 4},
+        {dbg->x_codes, h->Xq, Mz * K},    {dbg->c_x, h->c_x, Mz * 4},        {dbg->w_codes_t, h->Wq_t, N * K},
+        {dbg->c_w, h->c_w, N * 4},
+    };
+    for (const C& c : cps)
+      if (c.dst && (e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+        return cuda_fail(e, "debug copy");
+  }
+  return INT8MM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N, void* stream,
+                                    int8mm_weight_t* out) {
+  if (out == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (W_fp16_dev == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "W is NULL");
+  if (K < 16 || N < 16 || K % 16 != 0 || N % 16 != 0 || K > INT8MM_MAX_K || N >= (int64_t(1) << 31))
+    return fail(INT8MM_ERR_UNSUPPORTED_SHAPE,
+                "K=%lld, N=%lld: need 16 <= K <= %d and N >= 16, both multiples of 16", (long long)K,
+                (long long)N, INT8MM_MAX_K);
+  if (!aligned16(W_fp16_dev)) return fail(INT8MM_ERR_ALIGNMENT, "W must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int8mm_weight* h = new int8mm_weight();
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+  if (e != cudaSuccess) {
+    delete h;
+    return cuda_fail(e, "device query");
+  }
+  h->K = K;
+  h->N = N;
+  h->W = static_cast<const __half*>(W_fp16_dev);
+  const size_t Kz = static_cast<size_t>(K), Nz = static_cast<size_t>(N);
+  const size_t stripes = (Kz + 255) / 256, words = (Kz + 31) / 32;
+  size_t* tot = &h->bytes;
+  if ((e = alloc(&h->Wq_t, Nz * Kz, s, tot)) != cudaSuccess || (e = alloc(&h->c_w, Nz, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->inv_cw, Nz, s, tot)) != cudaSuccess || (e = alloc(&h->colmax_bits, Nz, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->stripe_ticket, stripes, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->all_ticket, 1, s, tot)) != cudaSuccess || (e = alloc(&h->mask, words, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->idx, Kz, s, tot)) != cudaSuccess || (e = alloc(&h->count, 1, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->colmax, Kz, s, tot)) != cudaSuccess || (e = alloc(&h->status, 1, s, tot)) != cudaSuccess) {
+    cudaStreamSynchronize(s);
+    free_all(h);
+    delete h;
+    return cuda_fail(e, "weight allocation");
+  }
+  if ((e = cudaMemsetAsync(h->stripe_ticket, 0, stripes * 4, s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(h->all_ticket, 0, 4, s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(h->mask, 0, words * 4, s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(h->count, 0, 4, s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(h->status, 0, 4, s)) != cudaSuccess ||
+      (e = launch_weight_prep(h->W, K, N, h->colmax_bits, h->Wq_t, h->c_w, h->inv_cw, h->num_sms, s)) !=
+          cudaSuccess) {
+    cudaStreamSynchronize(s);
+    free_all(h);
+    delete h;
+    return cuda_fail(e, "weight preparation");
+  }
+  int8mm_status st = make_tmap_i8(&h->tmB, h->Wq_t, Kz, Nz, kGemmBK, kGemmBN);
+  if (st != INT8MM_OK) {
+    cudaStreamSynchronize(s);
+    free_all(h);
+    delete h;
+    return st;
+  }
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    g_live.insert(h);
+  }
+  *out = h;
+  return INT8MM_OK;
+}
+
+int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream) {
+  if (!live(h)) return fail(INT8MM_ERR_INVALID_ARG, "invalid or freed weight handle");
+  if (M_max < 0 || M_max >= (int64_t(1) << 31)) return fail(INT8MM_ERR_INVALID_ARG, "M_max out of range");
+  int8mm_status st = set_device(h);
+  if (st != INT8MM_OK) return st;
+  return ensure_workspace(h, M_max, static_cast<cudaStream_t>(stream));
+}
+
+int8mm_status int8mm_forward(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha, void* Y_fp16_dev,
+                             void* stream) {
+  return forward_impl(h, X_fp16_dev, M, alpha, Y_fp16_dev, static_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+int8mm_status int8mm_forward_events(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
+                                    void* Y_fp16_dev, void* stream, void* const events[4]) {
+  return forward_impl(h, X_fp16_dev, M, alpha, Y_fp16_dev, static_cast<cudaStream_t>(stream), events, nullptr);
+}
+
+int8mm_status int8mm_forward_debug(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
+                                   void* Y_fp16_dev, void* stream, const int8mm_debug_bufs* dbg) {
+  if (dbg && dbg->acc && !aligned16(dbg->acc)) return fail(INT8MM_ERR_ALIGNMENT, "dbg->acc must be 16-byte aligned");
+  return forward_impl(h, X_fp16_dev, M, alpha, Y_fp16_dev, static_cast<cudaStream_t>(stream), nullptr, dbg);
+}
+
+int8mm_status int8mm_forward_host(int8mm_weight_t h, const void* X_fp16_host, int64_t M, float alpha,
+                                  void* Y_fp16_host, void* stream) {
+  int8mm_status st = check_forward_args(h, X_fp16_host, M, 0.0f, Y_fp16_host);
+  if (st != INT8MM_OK) return st;
+  if (std::isnan(alpha)) return fail(INT8MM_ERR_INVALID_ARG, "alpha is NaN");
+  if (M == 0) return INT8MM_OK;
+  if ((st = set_device(h)) != INT8MM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (M > h->io_rows) {
+    if (h->io_rows) {
+      cudaFreeAsync(h->dX, s);
+      cudaFreeAsync(h->dY, s);
+      h->bytes -= static_cast<size_t>(h->io_rows) * (h->K + h->N) * 2;
+      h->dX = h->dY = nullptr;
+      h->io_rows = 0;
+    }
+    if ((e = alloc(&h->dX, static_cast<size_t>(M) * h->K, s, nullptr)) != cudaSuccess ||
+        (e = alloc(&h->dY, static_cast<size_t>(M) * h->N, s, nullptr)) != cudaSuccess) {
+      cudaStreamSynchronize(s);
+      release(&h->dX);
+      release(&h->dY);
+      return cuda_fail(e, "host-forward buffers");
+    }
+    h->io_rows = M;
+    h->bytes += static_cast<size_t>(M) * (h->K + h->N) * 2;
+  }
+  if ((e = cudaMemcpyAsync(h->dX, X_fp16_host, static_cast<size_t>(M) * h->K * 2, cudaMemcpyHostToDevice, s)) !=
+      cudaSuccess)
+    return cuda_fail(e, "copy of X to the device");
+  if ((st = forward_impl(h, h->dX, M, alpha, h->dY, s, nullptr, nullptr)) != INT8MM_OK) return st;
+  if ((e = cudaMemcpyAsync(Y_fp16_host, h->dY, static_cast<size_t>(M) * h->N * 2, cudaMemcpyDeviceToHost, s)) !=
+      cudaSuccess)
+    return cuda_fail(e, "copy of Y to the host");
+  return INT8MM_OK;
+}
+
+int8mm_status int8mm_get_status(int8mm_weight_t h) {
+  if (!live(h)) return fail(INT8MM_ERR_INVALID_ARG, "invalid or freed weight handle");
+  int8mm_status st = set_device(h);
+  if (st != INT8MM_OK) return st;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "device synchronise");
+  int word = 0;
+  if ((e = cudaMemcpy(&word, h->status, 4, cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "status read");
+  if ((e = cudaMemset(h->status, 0, 4)) != cudaSuccess) return cuda_fail(e, "status reset");
+  if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "device synchronise");
+  if (word & kStatusTimeout) return fail(INT8MM_ERR_TIMEOUT, "a device wait ran out of time");
+  return INT8MM_OK;
+}
+
+int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns) {
+  if (!live(h)) return fail(INT8MM_ERR_INVALID_ARG, "invalid or freed weight handle");
+  if (timeout_ns == 0) return fail(INT8MM_ERR_INVALID_ARG, "timeout must be positive");
+  h->timeout_ns = timeout_ns;
+  return INT8MM_OK;
+}
+
+int8mm_status int8mm_weight_bytes(int8mm_weight_t h, size_t* bytes) {
+  if (!live(h) || bytes == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "invalid handle or NULL output");
+  *bytes = h->bytes;
+  return INT8MM_OK;
+}
+
+void int8mm_free(int8mm_weight_t h) {
+  if (h == nullptr) return;
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    if (g_live.erase(h) == 0) return;
+  }
+  int cur = -1;
+  cudaGetDevice(&cur);
+  cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  free_all(h);
+  if (cur >= 0) cudaSetDevice(cur);
+  delete h;
+}
+
+const char* int8mm_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,297 @@
+// Fused int8 GEMM of the LLM.int8() decomposed matmul for sm_100a.
+//
+//   Y[i,j] = fp16( Acc[i,j] / (c_x[i] c_w[j]) + sum_{k in O} X[i,k] W[k,j] )
+//   Acc    = Xq Wq^T, int8 x int8 -> int32 on the 5th-generation tensor cores
+//
+// Method: "LLM.int8() — 大模型激活值里藏着几个超大异常通道", 方法1 (the int8
+// product is dequantised by the outer product of the row and column scales)
+// and 方法2 (the fp16 product of the outlier columns is added back); the Fig. 2
+// caption of the AI 十大核心论文解读 article (Out_i32 dequantised by C_x ⊗ C_w,
+// then summed with the fp16 outlier output).  The pages describe this as an
+// int8 cuBLAS GEMM followed by a separate fp16 GEMM; here both, and the
+// dequantisation, run in one persistent kernel.
+//
+// Structure (one CTA per SM, 6 warps):
+//   warp 0      TMA producer: 128x128 A tiles (Xq) and 256x128 B tiles (Wq^T),
+//               128-byte swizzled, into a STAGES-deep shared-memory ring;
+//   warp 1      allocates 512 TMEM columns; one thread issues
+//               tcgen05.mma.kind::i8 (128x256x32) into a double-buffered
+//               int32 accumulator (2 x 256 columns);
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32*(w%4)..+31, one output row per thread), scale by
+//               1/c_x and 1/c_w, add the |O| outlier FMAs, write fp16.
+// The epilogue of tile t overlaps the main loop of tile t+1.  Every wait is
+// bounded; a timeout sets the status word and the CTA drains and exits.
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+#include <algorithm>
+
+namespace i8mm {
+namespace {
+
+constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK;  // 16 KB
+constexpr int B_BYTES = BN * BK;  // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
+constexpr int NUM_BARS = 2 * STAGES + 5;  // full, empty, tmem_full[2], tmem_empty[2], drain
+constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
+constexpr int SMEM_BYTES = MISC_OFFSET + 16 + 1024;  // + slack to align the base to 1024
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t IDESC = idesc_i8(BM, BN);
+static_assert(TMEM_COLS == 512, "two 128x256 int32 accumulators fill TMEM");
+
+__device__ __forceinline__ void fail(const GemmArgs& a, volatile int* abort_flag) {
+  *abort_flag = 1;
+  atomicOr(a.status, kStatusTimeout);
+}
+
+__device__ __forceinline__ float dequant(uint32_t acc, float rx, float rw) {
+  return __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(acc)), rx), rw);
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_i8_decomp_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFFSET);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFFSET);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + MISC_OFFSET + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = a.M, N = a.N, K = a.K;
+  const int num_m = (M + BM - 1) / BM;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const unsigned long long tmo = a.timeout_ns;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m_blk = tile % num_m, n_blk = tile / num_m;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_2d(sa, &tmA, &full[stage], kb * BK, m_blk * BM);
+          tma_load_2d(sa + A_BYTES, &tmB, &full[stage], kb * BK, n_blk * BN);
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        fail(a, abort_flag);
+        // Let every load already issued land before the CTA can exit.
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, tmo, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // -------------------------------------------------------- MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int lt = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++lt) {
+        const int buf = lt & 1;
+        const uint32_t use = static_cast<uint32_t>(lt >> 1);
+        if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, tmo, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, tmo, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint64_t adesc = smem_desc_k_sw128(sa);
+          const uint64_t bdesc = smem_desc_k_sw128(sa + A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            // advance 32 bytes along K inside the 128-byte swizzled row
+            mma_i8(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), IDESC,
+                   (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) mma_commit(&tfull[buf]);
+      }
+      if (!ok) {
+        fail(a, abort_flag);
+        mma_commit(drain);
+        mbar_wait(drain, 0, tmo, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    const int row_t = q * 32 + lane;
+    const int cnt = *a.count;
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
+      const int m_blk = tile % num_m, n_blk = tile / num_m;
+      const int buf = lt & 1;
+      const uint32_t use = static_cast<uint32_t>(lt >> 1);
+      // all lanes wait; the vote keeps the warp converged for tcgen05.ld
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], use & 1u, tmo, abort_flag));
+      if (!ok) {
+        if (lane == 0) fail(a, abort_flag);
+        break;
+      }
+      tc_fence_after();
+      const int m = m_blk * BM + row_t;
+      const bool row_ok = m < M;
+      float rx = 0.0f;
+      if (row_ok) {
+        const float c = a.c_x[m];
+        rx = c == 0.0f ? 0.0f : __frcp_rn(c);
+      }
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), r);
+        tmem_wait_ld();
+        const int n = n_blk * BN + ch * 32;
+        if (n >= N) continue;  // warp-uniform
+        const bool full32 = n + 32 <= N;
+        float v[32];
+        const float4* rw4 = reinterpret_cast<const float4*>(a.inv_cw + n);
+#pragma unroll
+        for (int t4 = 0; t4 < 8; ++t4) {
+          const float4 w = (full32 || t4 < 4) ? __ldg(rw4 + t4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[4 * t4 + 0] = dequant(r[4 * t4 + 0], rx, w.x);
+          v[4 * t4 + 1] = dequant(r[4 * t4 + 1], rx, w.y);
+          v[4 * t4 + 2] = dequant(r[4 * t4 + 2], rx, w.z);
+          v[4 * t4 + 3] = dequant(r[4 * t4 + 3], rx, w.w);
+        }
+        // fp16 outlier product: X[m, O] . W[O, n..n+31], fp32 accumulation
+        for (int o = 0; o < cnt; ++o) {
+          const int j = __ldg(a.idx + o);
+          const float xo = row_ok ? __half2float(a.X_OT[static_cast<size_t>(o) * M + m]) : 0.0f;
+          const uint4* wr = reinterpret_cast<const uint4*>(a.W + static_cast<size_t>(j) * N + n);
+          uint4 wv[4];
+          wv[0] = __ldg(wr);
+          wv[1] = __ldg(wr + 1);
+          wv[2] = full32 ? __ldg(wr + 2) : make_uint4(0, 0, 0, 0);
+          wv[3] = full32 ? __ldg(wr + 3) : make_uint4(0, 0, 0, 0);
+          const __half2* wh = reinterpret_cast<const __half2*>(wv);
+#pragma unroll
+          for (int p = 0; p < 16; ++p) {
+            const float2 f = __half22float2(wh[p]);
+            v[2 * p] = __fmaf_rn(xo, f.x, v[2 * p]);
+            v[2 * p + 1] = __fmaf_rn(xo, f.y, v[2 * p + 1]);
+          }
+        }
+        if (row_ok) {
+          uint4* yp = reinterpret_cast<uint4*>(a.Y + static_cast<size_t>(m) * N + n);
+          uint4 out[4];
+          uint32_t* ou = reinterpret_cast<uint32_t*>(out);
+#pragma unroll
+          for (int p = 0; p < 16; ++p) {
+            const __half2 h = __floats2half2_rn(v[2 * p], v[2 * p + 1]);
+            ou[p] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          yp[0] = out[0];
+          yp[1] = out[1];
+          if (full32) {
+            yp[2] = out[2];
+            yp[3] = out[3];
+          }
+          if (a.acc_dump != nullptr) {
+            uint4* ap = reinterpret_cast<uint4*>(a.acc_dump + static_cast<size_t>(m) * N + n);
+#pragma unroll
+            for (int t4 = 0; t4 < 8; ++t4)
+              if (full32 || t4 < 4) ap[t4] = make_uint4(r[4 * t4], r[4 * t4 + 1], r[4 * t4 + 2], r[4 * t4 + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
+                               cudaStream_t stream) {
+  static unsigned long long attr_set = 0;  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_i8_decomp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set |= bit;
+  }
+  const int num_tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
+  const int grid = std::max(1, std::min(num_tiles, num_sms));
+  gemm_i8_decomp_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, a);
+  return cudaGetLastError();
+}
+
+}  // namespace i8mm

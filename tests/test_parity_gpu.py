@@ -1,0 +1,247 @@
+"""GPU path against the CPU oracle, through the C ABI.
+
+Bit-exact: the outlier set, colmax, the int8 codes of X and W, the fp32
+scales c_x and c_w, and the int32 accumulators.  Within tolerance: fp16 Y,
+per element max(2 fp16 ulp, 1e-3 * sum_{k in O} |x_ik w_kj|).
+At full sizes the accumulators and Y are compared on seeded sampled rows
+(always including the first and the last row); codes and scales on all.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import int8_quantized_matmul_outlier_b200 as m
+import oracle
+import workloads
+from tests._parity import assert_y_close, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def dev():
+    return torch.device("cuda", torch.cuda.current_device())
+
+
+def check(p: workloads.Problem, rows=None, w=None, wq=None, check_w_codes=True):
+    """Run the debug forward of problem p on the GPU and compare with the oracle."""
+    X = torch.from_numpy(p.X).to(dev())
+    if w is None:
+        W = torch.from_numpy(p.W).to(dev())
+        w = m.int8mm_prepare_weight(W)
+    d = m.int8mm_forward_debug(w, X, p.alpha)
+    torch.cuda.synchronize()
+    assert m.int8mm_get_status(w) == m.INT8MM_OK
+
+    colmax, idx = oracle.outlier_columns(p.X, p.alpha)
+    cnt = int(d["outlier_count"].item())
+    assert cnt == idx.size
+    assert d["outlier_idx"][:cnt].cpu().numpy().tolist() == idx.tolist()
+    assert (d["colmax"].cpu().numpy() == colmax).all()
+
+    qx, c_x = oracle.quantize_rows(p.X, idx)
+    assert (d["c_x"].cpu().numpy() == c_x).all()
+    assert (d["x_codes"].cpu().numpy() == qx).all()
+
+    qw, c_w = oracle.quantize_cols(p.W) if wq is None else wq
+    assert (d["c_w"].cpu().numpy() == c_w).all()
+    if check_w_codes:
+        assert (d["w_codes_t"].cpu().numpy() == qw.T).all()
+
+    r = np.arange(p.X.shape[0]) if rows is None else np.asarray(rows)
+    acc_o = oracle.int8_matmul(np.ascontiguousarray(qx[r]), qw)
+    rt = torch.from_numpy(r).to(dev())
+    acc_g = d["acc"].index_select(0, rt).cpu().numpy()
+    assert (acc_g == acc_o).all()
+    Xr = np.ascontiguousarray(p.X[r])
+    y_o, _ = oracle.dequant_add_outliers(acc_o, c_x[r], c_w, Xr, p.W, idx)
+    y_g = d["Y"].index_select(0, rt).cpu().numpy()
+    err = assert_y_close(y_g, y_o, p.X, p.W, idx, rows=r)
+    return dict(w=w, cnt=cnt, err=err, d=d)
+
+
+# ---------------------------------------------------------------- small cases
+
+def test_tiny():
+    out = check(workloads.tiny())
+    assert out["cnt"] == 2
+
+
+SHAPES = [
+    # M, K, N, planted outliers, alpha
+    (1, 16, 16, 0, 6.0),
+    (3, 48, 48, 1, 6.0),
+    (17, 256, 272, 2, 6.0),
+    (128, 128, 256, 3, 6.0),
+    (129, 272, 528, 4, 6.0),
+    (300, 1040, 784, 5, 6.0),
+    (257, 384, 512, 7, math.inf),   # pure vector-wise int8
+    (64, 512, 256, 6, 0.0),         # every non-zero column is an outlier
+    (33, 4096, 1024, 7, 6.0),
+    (130, 2064, 2320, 9, 6.0),
+    (513, 640, 4112, 3, 6.0),       # many N tiles, ragged N tail
+]
+
+
+@pytest.mark.parametrize("M,K,N,n_out,alpha", SHAPES)
+def test_ragged_shapes(M, K, N, n_out, alpha):
+    p = workloads.small(M, K, N, n_out, seed=M * 7 + K + N + n_out, alpha=alpha)
+    out = check(p)
+    if alpha == 6.0:
+        assert out["cnt"] == n_out
+    elif math.isinf(alpha):
+        assert out["cnt"] == 0
+
+
+def test_threshold_ties_on_gpu():
+    # entries exactly at alpha are not outliers; the next fp16 value is
+    p = workloads.small(40, 64, 32, 0, seed=3)
+    p.X[5, 3] = 6.0
+    p.X[9, 10] = -6.0
+    p.X[11, 20] = np.float16(6.00390625)
+    p.X[0, 63] = -100
+    out = check(p)
+    assert out["cnt"] == 2
+
+
+def test_zero_rows_and_columns():
+    p = workloads.small(20, 128, 64, 2, seed=5)
+    p.X[4, :] = 0
+    p.W[:, 7] = 0
+    out = check(p)
+    d = out["d"]
+    assert float(d["c_x"][4]) == 0.0 and float(d["c_w"][7]) == 0.0
+    assert (d["Y"][:, 7].float() == 0).all()
+
+
+def test_repeat_and_stale_state():
+    # outlier state must not leak from one forward into the next
+    p1 = workloads.small(200, 512, 384, 6, seed=11)
+    p0 = workloads.small(200, 512, 384, 0, seed=12)
+    p0.W = p1.W
+    W = torch.from_numpy(p1.W).to(dev())
+    w = m.int8mm_prepare_weight(W)
+    wq = oracle.quantize_cols(p1.W)
+    a = check(p1, w=w, wq=wq)
+    b = check(p0, w=w, wq=wq)
+    c = check(p1, w=w, wq=wq)
+    assert (a["cnt"], b["cnt"], c["cnt"]) == (6, 0, 6)
+    assert torch.equal(a["d"]["Y"], c["d"]["Y"])
+
+
+def test_forward_matches_debug_forward_and_host_forward():
+    p = workloads.small(77, 640, 272, 4, seed=21)
+    X = torch.from_numpy(p.X).to(dev())
+    W = torch.from_numpy(p.W).to(dev())
+    w = m.int8mm_prepare_weight(W)
+    y1 = m.int8mm_forward(w, X, p.alpha)
+    y2 = m.int8mm_forward_debug(w, X, p.alpha)["Y"]
+    Xh = torch.from_numpy(p.X).pin_memory()
+    y3 = m.int8mm_forward_host(w, Xh, p.alpha)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert torch.equal(y1.cpu(), y3)
+
+
+def test_events_time_each_kernel():
+    p = workloads.small(256, 1024, 1024, 3, seed=31)
+    X = torch.from_numpy(p.X).to(dev())
+    W = torch.from_numpy(p.W).to(dev())
+    w = m.int8mm_prepare_weight(W)
+    Y = torch.empty((256, 1024), dtype=torch.float16, device=dev())
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    m.int8mm_forward_events(w, X, p.alpha, Y, ev)
+    torch.cuda.synchronize()
+    t = [ev[i].elapsed_time(ev[i + 1]) for i in range(3)]
+    assert all(x >= 0 for x in t) and sum(t) > 0
+    assert torch.equal(Y, m.int8mm_forward(w, X, p.alpha))
+
+
+def test_argument_errors_and_empty_input():
+    p = workloads.small(8, 64, 32, 1, seed=41)
+    X = torch.from_numpy(p.X).to(dev())
+    W = torch.from_numpy(p.W).to(dev())
+    w = m.int8mm_prepare_weight(W)
+    Y0 = torch.empty((0, 32), dtype=torch.float16, device=dev())
+    m.int8mm_forward(w, X[:0], 6.0, Y0)            # M == 0 is a no-op
+    with pytest.raises(m.Int8mmError) as e:
+        m.int8mm_forward(w, X, float("nan"))
+    assert e.value.status == m.INT8MM_ERR_INVALID_ARG
+    buf = torch.empty(8 * 64 + 1, dtype=torch.float16, device=dev())
+    Xmis = buf[1:].view(8, 64)                     # 2-byte offset: not 16-byte aligned
+    with pytest.raises(m.Int8mmError) as e:
+        m.int8mm_forward(w, Xmis, 6.0)
+    assert e.value.status == m.INT8MM_ERR_ALIGNMENT
+    Wbad = torch.empty((64, 40), dtype=torch.float16, device=dev())
+    with pytest.raises(m.Int8mmError) as e:
+        m.int8mm_prepare_weight(Wbad)
+    assert e.value.status == m.INT8MM_ERR_UNSUPPORTED_SHAPE
+    assert m.int8mm_weight_bytes(w) > 0
+    m.int8mm_free(w)
+    assert m.lib().int8mm_get_status(None) == m.INT8MM_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------- full-size configs
+
+@pytest.fixture(scope="module")
+def w175():
+    """The 175B-scale FFN expansion weight (K=12288, N=49152), shared by the
+    175B prefill and decode checks."""
+    p = workloads.gpt175b_prefill()
+    W = torch.from_numpy(p.W).to(dev())
+    w = m.int8mm_prepare_weight(W)
+    wq = oracle.quantize_cols(p.W)
+    yield p, w, wq
+    m.int8mm_free(w)
+
+
+def test_opt13b_prefill_full_size():
+    p = workloads.opt13b_prefill()
+    out = check(p, rows=sample_rows(p.X.shape[0], 16, seed=1))
+    assert out["cnt"] == 7
+    m.int8mm_free(out["w"])
+
+
+def test_175b_prefill_full_size(w175):
+    p, w, wq = w175
+    out = check(p, rows=sample_rows(p.X.shape[0], 8, seed=2), w=w, wq=wq)
+    assert out["cnt"] == 7
+
+
+@pytest.mark.parametrize("M", [1, 8, 32])
+def test_decode_full_size(M, w175):
+    p175, w, wq = w175
+    p = workloads.decode(M, with_weight=False)
+    p.W = p175.W
+    out = check(p, w=w, wq=wq, check_w_codes=False)
+    assert out["cnt"] == 7
+
+
+@pytest.fixture(scope="module")
+def w8192():
+    W = workloads.weight(8192, 8192, 4 * 1000 + 500_000)
+    Wd = torch.from_numpy(W).to(dev())
+    w = m.int8mm_prepare_weight(Wd)
+    wq = oracle.quantize_cols(W)
+    yield W, w, wq
+    m.int8mm_free(w)
+
+
+@pytest.mark.parametrize("M", [16, 128, 1024, 8192])
+@pytest.mark.parametrize("n_out", [0, 1, 7, 32, 128])
+def test_sweep_k8192(M, n_out, w8192):
+    W, w, wq = w8192
+    p = workloads.sweep(M, n_out, with_weight=False)
+    p.W = W
+    out = check(p, rows=sample_rows(M, 12, seed=M + n_out), w=w, wq=wq, check_w_codes=(M == 16 and n_out == 0))
+    assert out["cnt"] == n_out
+
+
+@pytest.mark.parametrize("M", [128, 1024])
+def test_sweep_alpha_inf_pure_vectorwise(M, w8192):
+    W, w, wq = w8192
+    p = workloads.sweep(M, 7, alpha=math.inf, with_weight=False)
+    p.W = W
+    out = check(p, rows=sample_rows(M, 12, seed=M), w=w, wq=wq, check_w_codes=False)
+    assert out["cnt"] == 0
