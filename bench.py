@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 LLM.int8() decomposed matmul.
+
+One step = one forward of the whole path (outlier detection, row
+quantisation, fused int8 GEMM with dequantisation and the fp16 outlier
+product) over one batch of synthetic activations, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config opt13b|175b]
+                    [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs an independent replica of the problem
+on its own GPU (weak scaling: the path has no exchange step); the reported
+time is the maximum over ranks.  Rank 0 prints one JSON line.
+
+Metric: effective TOPS = 2*M*N*K / time per step (the int8 contraction over
+the full K), inputs resident in HBM, L2 scrubbed (256 MB write) between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "int8-decomp matmul effective TOPS & % INT8 tensor peak; decode-shape HBM GB/s"
+# Dense tensor-core throughput ratio int8 : bf16 on B200 (4.5 POPS : 2.25 PFLOP/s).
+INT8_PER_BF16 = 2.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_SCRUB_BYTES = 256 << 20
+GEMM_SOURCES = ["int8_quantized_matmul_outlier_b200/csrc/gemm_i8.cu",
+                "int8_quantized_matmul_outlier_b200/csrc/ptx.cuh",
+                "int8_quantized_matmul_outlier_b200/csrc/kernels.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", choices=["opt13b", "175b"], default="opt13b")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="rows of the oracle CPU sample (0: sized to about 10 s)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return a
+
+
+def make_problem(config: str, rank: int) -> workloads.Problem:
+    if config == "opt13b":
+        return workloads.opt13b_prefill(repeat=rank)
+    return workloads.gpt175b_prefill(repeat=rank)
+
+
+def workload_config(p: workloads.Problem) -> dict:
+    M, K, N = p.shape
+    return {"workload": p.name, "M": M, "K": K, "N": N, "alpha": p.alpha,
+            "planted_outlier_columns": int(p.planted.size),
+            "inputs": "seeded synthetic fp16 (FFN-input statistics of the pages' OPT-13B example)",
+            "l2": "scrubbed between steps (256 MB write), outside the timed events"}
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on the current GEMM source (else None)."""
+    path = os.path.join(ROOT, "profiles", "gemm_i8_decomp_traffic.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path, encoding="utf-8").read()
+    src = re.search(r"gemm_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not src or src.group(1) != gemm_source_hash():
+        return None
+    m = re.search(rf"traffic_bytes_per_launch\[{re.escape(workload)}\]:\s*([0-9.eE+]+)", text)
+    return float(m.group(1)) if m else None
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML while running."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device, period_s: float = 0.01):
+        self.samples = []
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = self._handle(pynvml, device)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report no clocks
+            self.err = str(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    @staticmethod
+    def _handle(nv, device):
+        """NVML handle of the torch device, matched by PCI bus id (CUDA and
+        NVML number devices differently under CUDA_VISIBLE_DEVICES)."""
+        import torch
+        pr = torch.cuda.get_device_properties(device)
+        try:
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId_v2(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(device.index)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                try:
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                self.samples.append((mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        active = set()
+        for _, r in self.samples:
+            for name, bit in self.REASONS.items():
+                if r & bit:
+                    active.add(name)
+        return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(active), "samples": len(mhz), "source": "nvml"}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline and the reference arm)
+
+def oracle_rows_sample(p: workloads.Problem, rows: int, wq=None):
+    """Time the oracle's forward on a batch made of the first `rows` rows of
+    X (a bounded sample of the workload: same K, N, alpha and value
+    distributions): outlier detection, row quantisation, the int8
+    contraction, dequantisation and the fp16 outlier product.  The weight
+    codes, prepared once per weight, are made outside the timed region."""
+    import oracle
+    if wq is None:
+        wq = oracle.quantize_cols(p.W)
+    qw, c_w = wq
+    Xr = np.ascontiguousarray(p.X[:rows])
+    t0 = time.perf_counter()
+    _, idx = oracle.outlier_columns(Xr, p.alpha)
+    qx, c_x = oracle.quantize_rows(Xr, idx)
+    acc = oracle.int8_matmul(qx, qw)
+    oracle.dequant_add_outliers(acc, c_x, c_w, Xr, p.W, idx)
+    return time.perf_counter() - t0, wq
+
+
+def cpu_rows_for(p, target_s: float, wq):
+    t, _ = oracle_rows_sample(p, 16, wq)
+    M = p.shape[0]
+    return int(max(1, min(M, 16 * target_s / max(t, 1e-4))))
+
+
+def cpu_baseline(p: workloads.Problem, rows: int) -> dict:
+    import oracle
+    wq = oracle.quantize_cols(p.W)
+    if rows <= 0:
+        rows = cpu_rows_for(p, 10.0, wq)
+    t, _ = oracle_rows_sample(p, rows, wq)
+    M, K, N = p.shape
+    return {"value": 2.0 * rows * N * K / t / 1e12, "unit": "TOPS", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"batch of the first {rows} of {M} rows, whole forward on it; "
+                      f"weight codes prepared outside the timed region",
+            "seconds": t}
+
+
+# --------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    p = make_problem(args.config, 0)
+    M, K, N = p.shape
+    wq = oracle.quantize_cols(p.W)
+    # each step is a bounded sample sized so that the whole run stays within minutes
+    budget_s = 120.0 / max(1, args.steps + args.warmup)
+    rows = min(M, max(1, cpu_rows_for(p, min(budget_s, 5.0), wq)))
+    for _ in range(args.warmup):
+        oracle_rows_sample(p, rows, wq)
+    ts = [oracle_rows_sample(p, rows, wq)[0] for _ in range(args.steps)]
+    t = sum(ts)
+    value = 2.0 * rows * N * K * args.steps / t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": workload_config(p),
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"each step: whole forward on a batch of the first {rows} of {M} rows; "
+                                   f"weight codes prepared once, untimed"},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+
+    import int8_quantized_matmul_outlier_b200 as m
+
+    world, rank, local = dist_env()
+    distributed = world > 1
+    if distributed:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    def barrier():
+        if distributed:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if not distributed:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    p = make_problem(args.config, rank)
+    M, K, N = p.shape
+    X = torch.from_numpy(p.X).to(dev)
+    W = torch.from_numpy(p.W).to(dev)
+    w = m.int8mm_prepare_weight(W)
+    m.int8mm_reserve(w, M)
+    Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    scrub = torch.empty(L2_SCRUB_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        m.int8mm_forward(w, X, p.alpha, Y)
+        scrub.zero_()
+    torch.cuda.synchronize()
+    if m.int8mm_get_status(w) != m.INT8MM_OK:
+        raise RuntimeError("device wait timed out during warm-up")
+
+    steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clocks:
+        t0 = time.perf_counter()
+        for s in range(steps):
+            m.int8mm_forward_events(w, X, p.alpha, Y, ev[s], stream=stream)
+            scrub.zero_()
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+    barrier()
+    if m.int8mm_get_status(w) != m.INT8MM_OK:
+        raise RuntimeError("device wait timed out in the timed region")
+    seg = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in ev])  # ms
+    step_ms = seg.sum(axis=1)
+    total_ms = max_over_ranks(float(step_ms.sum()))
+    ms_per_step = total_ms / steps
+    flops = 2.0 * M * N * K
+    value = flops * steps * world / (total_ms * 1e-3) / 1e12
+    gemm_ms = max_over_ranks(float(seg[:, 2].mean()))
+    detect_ms = max_over_ranks(float(seg[:, 0].mean()))
+    quant_ms = max_over_ranks(float(seg[:, 1].mean()))
+
+    # end to end through the host-buffer entry point: pinned X in, pinned Y out
+    Xh = torch.from_numpy(p.X).pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.float16).pin_memory()
+    e2e_steps = max(1, min(args.e2e_steps, steps))
+    for _ in range(3):
+        m.int8mm_forward_host(w, Xh, p.alpha, Yh)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        m.int8mm_forward_host(w, Xh, p.alpha, Yh)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+
+    peaks = measured_peaks()
+    peak_tops = peaks["bf16_tflops"] * INT8_PER_BF16
+    achieved = flops / (gemm_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": workload_config(p),
+        "roofline": {
+            "bound": "tensor", "achieved": achieved, "peak": peak_tops, "unit": "TFLOP/s",
+            "frac": achieved / peak_tops, "traffic": recorded_traffic(p.name),
+            "kernel": "gemm_i8_decomp_kernel",
+            "peak_note": (f"dense int8 = {INT8_PER_BF16:g} x {peaks['source']} bf16 burst "
+                          f"{peaks['bf16_tflops']:g} TFLOP/s; int8 ops counted as 2*M*N*K"),
+        },
+        "kernels_ms": {"outlier_detect": detect_ms, "row_quant": quant_ms, "gemm_i8_decomp": gemm_ms},
+        "pct_int8_peak_whole_step": 100.0 * value / world / peak_tops,
+        "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": M * K * 2,
+                "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms,
+                "entry_point": "int8mm_forward_host (pinned host buffers)"},
+        "gpu_launches": 3 * steps,
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(p, args.cpu_rows)
+    m.int8mm_free(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if distributed:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
