@@ -157,6 +157,36 @@ int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns);
 /* Device bytes held by the handle (codes, scales, workspace). */
 int8mm_status int8mm_weight_bytes(int8mm_weight_t h, size_t* bytes);
 
+/*
+ * Outlier-column detection (step 1 above) that allocates no device memory.
+ * The paper has no counterpart of this entry point; it exists for callers
+ * that cannot allocate when they need the outlier set: an engine plugin whose
+ * enqueue step may not allocate, a serving loop that forbids allocation after
+ * warm-up, or a process whose caching allocator already holds nearly all of
+ * the device memory.
+ *
+ * X_fp16_dev: [M, K] fp16 row-major, 16-byte aligned (M >= 0).
+ * idx_dev:    [K] int32, written with the ascending outlier columns; the
+ *             first *count_dev entries are valid.
+ * count_dev:  [1] int32, written with |O|.
+ * colmax_dev: [K] fp32 max_i |X[i,j]|, or NULL to skip it.
+ * All three outputs are device memory owned by the caller.  Same results as
+ * the outlier_idx / outlier_count / colmax of int8mm_forward_debug.
+ *
+ * Scratch lives in one static device array of INT8MM_NOALLOC_SCRATCH_BYTES
+ * (1 MiB), which every GPU that loads the library holds until the process
+ * exits; the call itself makes no cudaMalloc, cudaFree or other allocation.
+ * Limit: 16 <= K <= INT8MM_MAX_K, K % 16 == 0 (larger K is rejected with
+ * INT8MM_ERR_UNSUPPORTED_SHAPE).  The first call on a device looks up the
+ * array's device address; make that first call before any CUDA stream
+ * capture.  All calls share the array and each call clears what must start
+ * at zero; calls whose kernels overlap on the GPU (unordered streams) race.
+ */
+#define INT8MM_NOALLOC_SCRATCH_BYTES (1u << 20)
+int8mm_status int8mm_outlier_columns_noalloc(const void* X_fp16_dev, int64_t M, int64_t K, float alpha,
+                                             int32_t* idx_dev, int32_t* count_dev, float* colmax_dev,
+                                             void* stream);
+
 /* Release the handle and everything it owns.  SYNCHRONISES the device
  * first, so no enqueued forward still uses the memory.  NULL or an already
  * freed handle is a no-op. */

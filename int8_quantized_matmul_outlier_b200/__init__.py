@@ -46,6 +46,7 @@ SIGNATURES = {
     "int8mm_weight_bytes": (_ST, [_P, ctypes.POINTER(ctypes.c_size_t)]),
     "int8mm_free": (None, [_P]),
     "int8mm_last_error": (ctypes.c_char_p, []),
+    "int8mm_outlier_columns_noalloc": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P]),
 }
 
 
@@ -200,6 +201,23 @@ def int8mm_forward_debug(w: Weight, X: torch.Tensor, alpha: float = 6.0, Y: torc
                                       _stream(stream), ctypes.byref(d)))
     out["Y"] = Y
     return out
+
+
+def int8mm_outlier_columns_noalloc(X: torch.Tensor, alpha: float = 6.0, stream=None,
+                                   want_colmax: bool = True):
+    """Outlier columns of X with no device allocation inside the library:
+    returns (idx [K] int32, count [1] int32, colmax [K] fp32 or None) as
+    device tensors, allocated here by the caller side (PyTorch)."""
+    _dev_f16_2d(X, "X")
+    M, K = X.shape
+    idx = torch.empty(K, dtype=torch.int32, device=X.device)
+    count = torch.empty(1, dtype=torch.int32, device=X.device)
+    colmax = torch.empty(K, dtype=torch.float32, device=X.device) if want_colmax else None
+    _check(lib().int8mm_outlier_columns_noalloc(X.data_ptr(), M, K, float(alpha), idx.data_ptr(),
+                                                count.data_ptr(),
+                                                colmax.data_ptr() if colmax is not None else None,
+                                                _stream(stream)))
+    return idx, count, colmax
 
 
 def int8mm_get_status(w: Weight) -> int:

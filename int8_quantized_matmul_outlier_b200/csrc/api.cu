@@ -283,6 +283,8 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
 
 }  // namespace
 
+void i8mm::set_last_error(const std::string& message) { g_last_error = message; }
+
 extern "C" {
 
 int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N, void* stream,

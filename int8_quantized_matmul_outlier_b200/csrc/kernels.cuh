@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstdint>
+#include <string>
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -11,6 +12,9 @@ namespace i8mm {
 
 // Status bits in the device status word.
 constexpr int kStatusTimeout = 1;
+
+// Sets the message returned by int8mm_last_error() on this host thread.
+void set_last_error(const std::string& message);
 
 // ---- weight preparation (once per weight) --------------------------------
 // Per output column j of W[K,N] (fp16, row-major): absmax over all K rows,

@@ -1,0 +1,127 @@
+// Outlier-column detection that allocates no device memory.
+//
+// Some callers cannot allocate device memory at the point where they need
+// the outlier set of an activation matrix: an inference engine's plugin whose
+// enqueue step is forbidden to allocate, a serving loop that must not
+// allocate after warm-up, or a process whose caching allocator has already
+// reserved nearly all of the device memory, so that a fresh cudaMalloc (or a
+// stream-ordered allocation) fails or fragments the pool.  For them this file
+// runs the outlier-detection kernel with its scratch (per-chunk column
+// maxima, completion tickets and the column bitmask) in a fixed static
+// device array instead of a handle-owned workspace.
+//
+// The array is kNoAllocScratchBytes (1 MiB) per device.  It is part of the
+// library's device image, so every GPU that loads the library holds it until
+// the process exits.  All calls share it: two calls whose kernels overlap on
+// the GPU (for example on two streams without ordering between them) race
+// on it and give wrong results.
+#include "int8mm.h"
+#include "kernels.cuh"
+
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = INT8MM_NOALLOC_SCRATCH_BYTES;
+constexpr size_t kTicketBytes = 2048;     // stripe tickets (<= 256) + 1 grid ticket
+constexpr size_t kMaskBytes = 8192;       // ceil(65536 / 32) words
+constexpr size_t kColmaxBytes = 262144;   // 65536 fp32, used when the caller passes none
+constexpr size_t kPartialOffset = kTicketBytes + kMaskBytes + kColmaxBytes;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
+
+int8mm_status setup_error(int8mm_status s, const std::string& msg) {
+  i8mm::set_last_error(msg);  // reported by int8mm_last_error()
+  return s;
+}
+
+// Once per device, with that device current: the device address of the
+// static scratch array (its host-side name is only a stand-in).
+int8mm_status device_scratch(int dev, void** ptr, int* num_sms) {
+  std::lock_guard<std::mutex> g(g_setup_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess)
+      return setup_error(INT8MM_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess)
+      return setup_error(INT8MM_ERR_CUDA, std::string("device query: ") + cudaGetErrorString(e));
+    g_num_sms[dev] = sms;
+    g_scratch_ptr[dev] = p;
+  }
+  *ptr = g_scratch_ptr[dev];
+  *num_sms = g_num_sms[dev];
+  return INT8MM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int8mm_status int8mm_outlier_columns_noalloc(const void* X_fp16_dev, int64_t M, int64_t K, float alpha,
+                                             int32_t* idx_dev, int32_t* count_dev, float* colmax_dev,
+                                             void* stream) {
+  if (X_fp16_dev == nullptr || idx_dev == nullptr || count_dev == nullptr)
+    return setup_error(INT8MM_ERR_INVALID_ARG, "X, idx and count must not be NULL");
+  if (std::isnan(alpha)) return setup_error(INT8MM_ERR_INVALID_ARG, "alpha is NaN");
+  if (M < 0 || M >= (int64_t(1) << 31))
+    return setup_error(INT8MM_ERR_INVALID_ARG, "M must be in [0, 2^31)");
+  if (K < 16 || K % 16 != 0 || K > INT8MM_MAX_K)
+    return setup_error(INT8MM_ERR_UNSUPPORTED_SHAPE,
+                       "K=" + std::to_string(K) + ": the no-allocation detection needs 16 <= K <= " +
+                           std::to_string(INT8MM_MAX_K) + ", a multiple of 16");
+  if ((reinterpret_cast<uintptr_t>(X_fp16_dev) & 15u) != 0)
+    return setup_error(INT8MM_ERR_ALIGNMENT, "X must be 16-byte aligned");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return setup_error(INT8MM_ERR_CUDA, "no usable current CUDA device");
+  void* base = nullptr;
+  int sms = 0;
+  int8mm_status st = device_scratch(dev, &base, &sms);
+  if (st != INT8MM_OK) return st;
+
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (M == 0) {  // no rows: no outlier columns
+    if ((e = cudaMemsetAsync(count_dev, 0, sizeof(int32_t), cs)) != cudaSuccess)
+      return setup_error(INT8MM_ERR_CUDA, std::string("count reset: ") + cudaGetErrorString(e));
+    return INT8MM_OK;
+  }
+  const int chunks = i8mm::outlier_row_chunks(M, K, sms);
+  const size_t partial_bytes = static_cast<size_t>(chunks) * static_cast<size_t>(K) * sizeof(uint16_t);
+  if (kPartialOffset + partial_bytes > kNoAllocScratchBytes)
+    return setup_error(INT8MM_ERR_UNSUPPORTED_SHAPE,
+                       "scratch of " + std::to_string(kPartialOffset + partial_bytes) +
+                           " bytes exceeds the static " + std::to_string(kNoAllocScratchBytes) + " bytes");
+
+  unsigned char* s = static_cast<unsigned char*>(base);
+  // The array keeps the previous call's contents: the tickets must start at 0.
+  if ((e = cudaMemsetAsync(s, 0, kTicketBytes, cs)) != cudaSuccess)
+    return setup_error(INT8MM_ERR_CUDA, std::string("ticket reset: ") + cudaGetErrorString(e));
+  i8mm::OutlierScratch sc;
+  sc.stripe_ticket = reinterpret_cast<unsigned*>(s);
+  sc.all_ticket = reinterpret_cast<unsigned*>(s) + 256;
+  sc.mask = reinterpret_cast<uint32_t*>(s + kTicketBytes);
+  sc.colmax = colmax_dev ? colmax_dev : reinterpret_cast<float*>(s + kTicketBytes + kMaskBytes);
+  sc.partial = reinterpret_cast<uint16_t*>(s + kPartialOffset);
+  sc.idx = idx_dev;
+  sc.count = count_dev;
+  if ((e = i8mm::launch_outlier_detect(static_cast<const __half*>(X_fp16_dev), M, K, alpha, sc, sms, cs)) !=
+      cudaSuccess)
+    return setup_error(INT8MM_ERR_CUDA, std::string("outlier detection launch: ") + cudaGetErrorString(e));
+  return INT8MM_OK;
+}
+
+}  // extern "C"
