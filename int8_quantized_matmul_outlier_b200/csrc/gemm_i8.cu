@@ -17,9 +17,13 @@
 //   warp 1      allocates 512 TMEM columns; one thread issues
 //               tcgen05.mma.kind::i8 (128x256x32) into a double-buffered
 //               int32 accumulator (2 x 256 columns);
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32*(w%4)..+31, one output row per thread), scale by
-//               1/c_x and 1/c_w, add the |O| outlier FMAs, write fp16.
+//   warps 2-9   epilogue, two warps per TMEM lane quarter (warp w reads lanes
+//               32*(w%4)..+31, one output row per thread), each covering one
+//               128-column half of the tile: tcgen05.ld of the accumulator,
+//               scale by 1/c_x and 1/c_w, add the |O| outlier FMAs, write fp16.
+//               While the tile still accumulates, the four warps of a half
+//               stage 1/c_w and the outlier weight rows W[O, half] in shared
+//               memory and load their rows' outlier activations.
 // The epilogue of tile t overlaps the main loop of tile t+1.  Every wait is
 // bounded; a timeout sets the status word and the CTA drains and exits.
 #include "kernels.cuh"
@@ -38,15 +42,29 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
 constexpr int NUM_BARS = 2 * STAGES + 5;  // full, empty, tmem_full[2], tmem_empty[2], drain
 constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
-constexpr int SMEM_BYTES = MISC_OFFSET + 16 + 1024;  // + slack to align the base to 1024
+// Epilogue staging: per 128-column half of the tile, the first OUT_CAP
+// outlier rows W[idx[o], cols] and 1/c_w[cols] as fp32.
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int HALF_N = BN / 2;
+constexpr int OUT_CAP = 16;
+constexpr int WO_OFFSET = (MISC_OFFSET + 16 + 15) & ~15;
+constexpr int WO_BYTES = 2 * OUT_CAP * HALF_N * 4;
+constexpr int RW_OFFSET = WO_OFFSET + WO_BYTES;
+constexpr int RW_BYTES = 2 * HALF_N * 4;
+constexpr int SMEM_BYTES = RW_OFFSET + RW_BYTES + 1024;  // + slack to align the base to 1024
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+static_assert(SMEM_BYTES <= 232448, "fits the 227 KB of shared memory per block");
 constexpr uint32_t IDESC = idesc_i8(BM, BN);
 static_assert(TMEM_COLS == 512, "two 128x256 int32 accumulators fill TMEM");
 
 __device__ __forceinline__ void fail(const GemmArgs& a, volatile int* abort_flag) {
   *abort_flag = 1;
   atomicOr(a.status, kStatusTimeout);
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ float dequant(uint32_t acc, float rx, float rw) {
@@ -80,7 +98,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], NUM_EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -178,51 +196,111 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    const int ew = warp - 2;                  // 0..7
+    const int q = warp & 3;                   // TMEM lane quarter this warp may read
+    const int h = ew >> 2;                    // 128-column half of the tile
+    const int tl = (ew & 3) * 32 + lane;      // thread index among the half's 4 warps
     const int row_t = q * 32 + lane;
     const int cnt = *a.count;
+    const int cs = min(cnt, OUT_CAP);         // outliers staged in shared memory
+    float* wo = reinterpret_cast<float*>(smem + WO_OFFSET) + h * OUT_CAP * HALF_N;  // [OUT_CAP][HALF_N]
+    float* rws = reinterpret_cast<float*>(smem + RW_OFFSET) + h * HALF_N;           // [HALF_N]
+    const uint32_t bar_id = 1 + h;
+    bool alive = true;
     int lt = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
       const int m_blk = tile % num_m, n_blk = tile / num_m;
       const int buf = lt & 1;
       const uint32_t use = static_cast<uint32_t>(lt >> 1);
-      // all lanes wait; the vote keeps the warp converged for tcgen05.ld
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], use & 1u, tmo, abort_flag));
-      if (!ok) {
-        if (lane == 0) fail(a, abort_flag);
-        break;
-      }
-      tc_fence_after();
+      const int nh = n_blk * BN + h * HALF_N;  // first column of this half
       const int m = m_blk * BM + row_t;
       const bool row_ok = m < M;
+
+      // (1) stage this tile's scales and outlier weight rows; this runs
+      //     while the tensor cores still accumulate the tile.
+      named_bar_sync(bar_id, 128);  // readers of the previous tile are done
+      if (tl < HALF_N / 4) {
+        const int n = nh + tl * 4;
+        const float4 f = n < N ? __ldg(reinterpret_cast<const float4*>(a.inv_cw + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4*>(rws)[tl] = f;
+      }
+      for (int e = tl; e < cs * (HALF_N / 8); e += 128) {
+        const int o = e / (HALF_N / 8), part = e % (HALF_N / 8);
+        const int n = nh + part * 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (n < N) v = __ldg(reinterpret_cast<const uint4*>(a.W + static_cast<size_t>(__ldg(a.idx + o)) * N + n));
+        const __half2* hv = reinterpret_cast<const __half2*>(&v);
+        const float2 f0 = __half22float2(hv[0]), f1 = __half22float2(hv[1]);
+        const float2 f2 = __half22float2(hv[2]), f3 = __half22float2(hv[3]);
+        float4* dst = reinterpret_cast<float4*>(wo + o * HALF_N + part * 8);
+        dst[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+        dst[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
+      }
+      float xo[OUT_CAP];
+#pragma unroll
+      for (int o = 0; o < OUT_CAP; ++o)
+        xo[o] = (o < cs && row_ok) ? __half2float(a.X_OT[static_cast<size_t>(o) * M + m]) : 0.0f;
       float rx = 0.0f;
       if (row_ok) {
         const float c = a.c_x[m];
         rx = c == 0.0f ? 0.0f : __frcp_rn(c);
       }
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
+      named_bar_sync(bar_id, 128);  // staging visible to the half's 4 warps
+
+      // (2) wait for the accumulator (all lanes; the vote keeps the warp
+      //     converged for tcgen05.ld).  After a timeout the warp keeps taking
+      //     part in the named barriers but does no more work.
+      if (alive) {
+        alive = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], use & 1u, tmo, abort_flag));
+        if (!alive && lane == 0) fail(a, abort_flag);
+      }
+      if (!alive) continue;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(buf * BN + h * HALF_N);
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
+      for (int ch = 0; ch < HALF_N / 32; ++ch) {
+        const int cl = ch * 32;
         uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(ch * 32), r);
+        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(cl), r);
         tmem_wait_ld();
-        const int n = n_blk * BN + ch * 32;
+        if (ch == HALF_N / 32 - 1) {  // accumulator buffer no longer read: release it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+        }
+        const int n = nh + cl;
         if (n >= N) continue;  // warp-uniform
         const bool full32 = n + 32 <= N;
         float v[32];
-        const float4* rw4 = reinterpret_cast<const float4*>(a.inv_cw + n);
+        const float4* rw4 = reinterpret_cast<const float4*>(rws + cl);
 #pragma unroll
         for (int t4 = 0; t4 < 8; ++t4) {
-          const float4 w = (full32 || t4 < 4) ? __ldg(rw4 + t4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 w = rw4[t4];
           v[4 * t4 + 0] = dequant(r[4 * t4 + 0], rx, w.x);
           v[4 * t4 + 1] = dequant(r[4 * t4 + 1], rx, w.y);
           v[4 * t4 + 2] = dequant(r[4 * t4 + 2], rx, w.z);
           v[4 * t4 + 3] = dequant(r[4 * t4 + 3], rx, w.w);
         }
-        // fp16 outlier product: X[m, O] . W[O, n..n+31], fp32 accumulation
-        for (int o = 0; o < cnt; ++o) {
+        // fp16 outlier product X[m, O] . W[O, n..n+31] with fp32 accumulation,
+        // in ascending order of O: staged rows first, then any beyond OUT_CAP.
+#pragma unroll
+        for (int o = 0; o < OUT_CAP; ++o) {
+          if (o < cs) {
+            const float4* w4 = reinterpret_cast<const float4*>(wo + o * HALF_N + cl);
+#pragma unroll
+            for (int t4 = 0; t4 < 8; ++t4) {
+              const float4 w = w4[t4];
+              v[4 * t4 + 0] = __fmaf_rn(xo[o], w.x, v[4 * t4 + 0]);
+              v[4 * t4 + 1] = __fmaf_rn(xo[o], w.y, v[4 * t4 + 1]);
+              v[4 * t4 + 2] = __fmaf_rn(xo[o], w.z, v[4 * t4 + 2]);
+              v[4 * t4 + 3] = __fmaf_rn(xo[o], w.w, v[4 * t4 + 3]);
+            }
+          }
+        }
+        for (int o = OUT_CAP; o < cnt; ++o) {
           const int j = __ldg(a.idx + o);
-          const float xo = row_ok ? __half2float(a.X_OT[static_cast<size_t>(o) * M + m]) : 0.0f;
+          const float x1 = row_ok ? __half2float(a.X_OT[static_cast<size_t>(o) * M + m]) : 0.0f;
           const uint4* wr = reinterpret_cast<const uint4*>(a.W + static_cast<size_t>(j) * N + n);
           uint4 wv[4];
           wv[0] = __ldg(wr);
@@ -233,8 +311,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int p = 0; p < 16; ++p) {
             const float2 f = __half22float2(wh[p]);
-            v[2 * p] = __fmaf_rn(xo, f.x, v[2 * p]);
-            v[2 * p + 1] = __fmaf_rn(xo, f.y, v[2 * p + 1]);
+            v[2 * p] = __fmaf_rn(x1, f.x, v[2 * p]);
+            v[2 * p + 1] = __fmaf_rn(x1, f.y, v[2 * p + 1]);
           }
         }
         if (row_ok) {
@@ -243,8 +321,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t* ou = reinterpret_cast<uint32_t*>(out);
 #pragma unroll
           for (int p = 0; p < 16; ++p) {
-            const __half2 h = __floats2half2_rn(v[2 * p], v[2 * p + 1]);
-            ou[p] = *reinterpret_cast<const uint32_t*>(&h);
+            const __half2 hh = __floats2half2_rn(v[2 * p], v[2 * p + 1]);
+            ou[p] = *reinterpret_cast<const uint32_t*>(&hh);
           }
           yp[0] = out[0];
           yp[1] = out[1];
@@ -260,9 +338,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
     }
   }
 
