@@ -95,8 +95,9 @@ int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream);
  *   path (pure vector-wise int8); any value below every |x| makes every
  *   column an outlier.  NaN is an argument error.
  * M == 0 is a no-op.  Three kernels run on `stream` (outlier detection, row
- * quantisation, fused int8 GEMM); the outlier count never leaves the device,
- * so the call does not synchronise.  Grows the workspace when M exceeds
+ * quantisation, fused int8 GEMM), the last two as programmatic dependent
+ * launches that start while their predecessor finishes; the outlier count
+ * never leaves the device, so the call does not synchronise.  Grows the workspace when M exceeds
  * every earlier M (stream-ordered allocation).
  */
 int8mm_status int8mm_forward(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
@@ -113,13 +114,15 @@ int8mm_status int8mm_forward_host(int8mm_weight_t h, const void* X_fp16_host, in
                                   void* Y_fp16_host, void* stream);
 
 /*
- * Same as int8mm_forward, and records four caller-created CUDA events
- * (cudaEvent_t, passed as void*) on `stream`: before the outlier pass,
- * between it and the row pass, between the row pass and the GEMM, and after
- * the GEMM, so that each kernel can be timed on its own stream.
+ * Same as int8mm_forward, and records three caller-created CUDA events
+ * (cudaEvent_t, passed as void*; NULL entries are skipped) on `stream`:
+ * before the activation passes, between them and the GEMM, and after the
+ * GEMM, so that the GEMM can be timed on the stream it runs on.  A middle
+ * event makes the GEMM an ordinary launch instead of a programmatic
+ * dependent of the row pass (its prologue then no longer overlaps that pass).
  */
 int8mm_status int8mm_forward_events(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
-                                    void* Y_fp16_dev, void* stream, void* const events[4]);
+                                    void* Y_fp16_dev, void* stream, void* const events[3]);
 
 /* Intermediate values of one forward, for verification.  Every field is a
  * device pointer or NULL (not written). */

@@ -30,9 +30,11 @@ struct int8mm_weight {
   uint32_t* colmax_bits = nullptr;  // [N] prep scratch
   CUtensorMap tmB;
   // fixed-size scratch of the outlier pass
-  unsigned* stripe_ticket = nullptr;
-  unsigned* all_ticket = nullptr;
+  unsigned long long* colkey = nullptr;  // [K]
+  unsigned long long* epoch = nullptr;   // [1]
+  unsigned* ticket = nullptr;            // [1]
   uint32_t* mask = nullptr;
+  int32_t* pre = nullptr;
   int32_t* idx = nullptr;
   int32_t* count = nullptr;
   float* colmax = nullptr;
@@ -42,7 +44,6 @@ struct int8mm_weight {
   int8_t* Xq = nullptr;
   float* c_x = nullptr;
   __half* X_OT = nullptr;
-  uint16_t* partial = nullptr;
   // tensor map of Xq for the current (pointer, M)
   CUtensorMap tmA;
   const void* tmA_ptr = nullptr;
@@ -132,7 +133,6 @@ void free_workspace(int8mm_weight* h) {
   release(&h->Xq);
   release(&h->c_x);
   release(&h->X_OT);
-  release(&h->partial);
   h->ws_rows = 0;
   h->tmA_ptr = nullptr;
   h->tmA_rows = -1;
@@ -146,9 +146,11 @@ void free_all(int8mm_weight* h) {
   release(&h->c_w);
   release(&h->inv_cw);
   release(&h->colmax_bits);
-  release(&h->stripe_ticket);
-  release(&h->all_ticket);
+  release(&h->colkey);
+  release(&h->epoch);
+  release(&h->ticket);
   release(&h->mask);
+  release(&h->pre);
   release(&h->idx);
   release(&h->count);
   release(&h->colmax);
@@ -156,11 +158,9 @@ void free_all(int8mm_weight* h) {
 }
 
 size_t ws_bytes(const int8mm_weight* h, int64_t rows) {
-  const int chunks = outlier_row_chunks_bound(rows, h->K, h->num_sms);
   return static_cast<size_t>(rows) * h->K                  // Xq
          + static_cast<size_t>(rows) * 4                   // c_x
-         + static_cast<size_t>(rows) * h->K * 2            // X_OT
-         + static_cast<size_t>(chunks) * h->K * 2;         // partial
+         + static_cast<size_t>(rows) * h->K * 2;           // X_OT
 }
 
 int8mm_status ensure_workspace(int8mm_weight* h, int64_t M, cudaStream_t s) {
@@ -173,20 +173,16 @@ int8mm_status ensure_workspace(int8mm_weight* h, int64_t M, cudaStream_t s) {
     cudaFreeAsync(h->Xq, s);
     cudaFreeAsync(h->c_x, s);
     cudaFreeAsync(h->X_OT, s);
-    cudaFreeAsync(h->partial, s);
     h->bytes -= ws_bytes(h, h->ws_rows);
     h->Xq = nullptr;
     h->c_x = nullptr;
     h->X_OT = nullptr;
-    h->partial = nullptr;
     h->ws_rows = 0;
   }
-  const int chunks = outlier_row_chunks_bound(rows, h->K, h->num_sms);
   cudaError_t e;
   if ((e = alloc(&h->Xq, static_cast<size_t>(rows) * h->K, s, nullptr)) != cudaSuccess ||
       (e = alloc(&h->c_x, static_cast<size_t>(rows), s, nullptr)) != cudaSuccess ||
-      (e = alloc(&h->X_OT, static_cast<size_t>(rows) * h->K, s, nullptr)) != cudaSuccess ||
-      (e = alloc(&h->partial, static_cast<size_t>(chunks) * h->K, s, nullptr)) != cudaSuccess) {
+      (e = alloc(&h->X_OT, static_cast<size_t>(rows) * h->K, s, nullptr)) != cudaSuccess) {
     cudaStreamSynchronize(s);
     free_workspace(h);
     return cuda_fail(e, "workspace allocation");
@@ -205,7 +201,8 @@ int8mm_status check_forward_args(const int8mm_weight* h, const void* X, int64_t 
   if (M == 0) return INT8MM_OK;
   if (X == nullptr || Y == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "X or Y is NULL");
   const int64_t tiles = ((M + kGemmBM - 1) / kGemmBM) * ((h->N + kGemmBN - 1) / kGemmBN);
-  if (tiles >= (int64_t(1) << 31) || M * h->N >= (int64_t(1) << 62))
+  const int64_t detect_blocks = ((h->K + 255) / 256) * ((M + 63) / 64);
+  if (tiles >= (int64_t(1) << 31) || detect_blocks >= (int64_t(1) << 31) || M * h->N >= (int64_t(1) << 62))
     return fail(INT8MM_ERR_UNSUPPORTED_SHAPE, "M=%lld x N=%lld is too large", (long long)M, (long long)h->N);
   if (!aligned16(X) || !aligned16(Y)) return fail(INT8MM_ERR_ALIGNMENT, "X and Y must be 16-byte aligned");
   return INT8MM_OK;
@@ -233,19 +230,18 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     h->tmA_ptr = h->Xq;
     h->tmA_rows = M;
   }
-  OutlierScratch sc{h->partial, h->stripe_ticket, h->all_ticket, h->mask, h->idx, h->count, h->colmax};
+  OutlierScratch sc{h->colkey, h->epoch, h->ticket, h->mask, h->pre, h->idx, h->count, h->colmax};
   const __half* Xh = static_cast<const __half*>(X);
   cudaError_t e;
   auto rec = [&](int i) {
     if (events && events[i]) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
   };
   rec(0);
-  if ((e = launch_outlier_detect(Xh, M, h->K, alpha, sc, h->num_sms, s)) != cudaSuccess)
+  if ((e = launch_outlier_detect(Xh, M, h->K, alpha, sc, s)) != cudaSuccess)
     return cuda_fail(e, "outlier detection launch");
-  rec(1);
-  if ((e = launch_row_quant(Xh, M, h->K, sc, h->Xq, h->c_x, h->X_OT, s)) != cudaSuccess)
+  if ((e = launch_row_quant(Xh, M, h->K, sc, h->Xq, h->c_x, h->X_OT, /*pdl=*/true, s)) != cudaSuccess)
     return cuda_fail(e, "row quantisation launch");
-  rec(2);
+  rec(1);
   GemmArgs a;
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(h->N);
@@ -260,9 +256,12 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
   a.acc_dump = dbg ? dbg->acc : nullptr;
   a.status = h->status;
   a.timeout_ns = h->timeout_ns;
-  if ((e = launch_gemm_decomp(h->tmA, h->tmB, a, h->num_sms, s)) != cudaSuccess)
+  // Without events between them, the GEMM is a programmatic dependent of the
+  // row pass; an event record in between makes it an ordinary launch.
+  const bool pdl = !(events && events[1]);
+  if ((e = launch_gemm_decomp(h->tmA, h->tmB, a, h->num_sms, pdl, s)) != cudaSuccess)
     return cuda_fail(e, "int8 GEMM launch");
-  rec(3);
+  rec(2);
   if (dbg) {
     const size_t K = static_cast<size_t>(h->K), N = static_cast<size_t>(h->N), Mz = static_cast<size_t>(M);
     struct C {
@@ -309,21 +308,23 @@ int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N
   h->N = N;
   h->W = static_cast<const __half*>(W_fp16_dev);
   const size_t Kz = static_cast<size_t>(K), Nz = static_cast<size_t>(N);
-  const size_t stripes = (Kz + 255) / 256, words = (Kz + 31) / 32;
+  const size_t words = (Kz + 31) / 32;
   size_t* tot = &h->bytes;
   if ((e = alloc(&h->Wq_t, Nz * Kz, s, tot)) != cudaSuccess || (e = alloc(&h->c_w, Nz, s, tot)) != cudaSuccess ||
       (e = alloc(&h->inv_cw, Nz, s, tot)) != cudaSuccess || (e = alloc(&h->colmax_bits, Nz, s, tot)) != cudaSuccess ||
-      (e = alloc(&h->stripe_ticket, stripes, s, tot)) != cudaSuccess ||
-      (e = alloc(&h->all_ticket, 1, s, tot)) != cudaSuccess || (e = alloc(&h->mask, words, s, tot)) != cudaSuccess ||
-      (e = alloc(&h->idx, Kz, s, tot)) != cudaSuccess || (e = alloc(&h->count, 1, s, tot)) != cudaSuccess ||
-      (e = alloc(&h->colmax, Kz, s, tot)) != cudaSuccess || (e = alloc(&h->status, 1, s, tot)) != cudaSuccess) {
+      (e = alloc(&h->colkey, Kz, s, tot)) != cudaSuccess || (e = alloc(&h->epoch, 1, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->ticket, 1, s, tot)) != cudaSuccess || (e = alloc(&h->mask, words, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->pre, words, s, tot)) != cudaSuccess || (e = alloc(&h->idx, Kz, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->count, 1, s, tot)) != cudaSuccess || (e = alloc(&h->colmax, Kz, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->status, 1, s, tot)) != cudaSuccess) {
     cudaStreamSynchronize(s);
     free_all(h);
     delete h;
     return cuda_fail(e, "weight allocation");
   }
-  if ((e = cudaMemsetAsync(h->stripe_ticket, 0, stripes * 4, s)) != cudaSuccess ||
-      (e = cudaMemsetAsync(h->all_ticket, 0, 4, s)) != cudaSuccess ||
+  if ((e = cudaMemsetAsync(h->colkey, 0, Kz * 8, s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(h->epoch, 0, 8, s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(h->ticket, 0, 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->mask, 0, words * 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->count, 0, 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->status, 0, 4, s)) != cudaSuccess ||
@@ -363,7 +364,7 @@ int8mm_status int8mm_forward(int8mm_weight_t h, const void* X_fp16_dev, int64_t 
 }
 
 int8mm_status int8mm_forward_events(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
-                                    void* Y_fp16_dev, void* stream, void* const events[4]) {
+                                    void* Y_fp16_dev, void* stream, void* const events[3]) {
   return forward_impl(h, X_fp16_dev, M, alpha, Y_fp16_dev, static_cast<cudaStream_t>(stream), events, nullptr);
 }
 

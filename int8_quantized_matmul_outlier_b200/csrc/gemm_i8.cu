@@ -63,6 +63,10 @@ __device__ __forceinline__ void fail(const GemmArgs& a, volatile int* abort_flag
   atomicOr(a.status, kStatusTimeout);
 }
 
+// Wait until the kernel this one depends on (programmatic dependent launch)
+// has finished and its memory is visible; a no-op without that launch mode.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -123,9 +127,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
       bool ok = true;
+      // The weight tiles of the first k-blocks do not depend on the
+      // activation pass: issue them before waiting for it, then the
+      // matching activation tiles (all stages start empty).
+      const int first = blockIdx.x;
+      const int pre = first < num_tiles ? min(STAGES, num_kb) : 0;
+      for (int kb = 0; kb < pre; ++kb) {
+        mbar_arrive_expect_tx(&full[kb], STAGE_BYTES);
+        tma_load_2d(smem + kb * STAGE_BYTES + A_BYTES, &tmB, &full[kb], kb * BK, (first / num_m) * BN);
+      }
+      pdl_wait();
+      for (int kb = 0; kb < pre; ++kb) {
+        tma_load_2d(smem + kb * STAGE_BYTES, &tmA, &full[kb], kb * BK, (first % num_m) * BM);
+        issued_mask |= 1u << kb;
+      }
+      stage = pre % STAGES;
+      phase = pre == STAGES ? 1u : 0u;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int m_blk = tile % num_m, n_blk = tile / num_m;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = tile == first ? pre : 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
             ok = false;
             break;
@@ -201,6 +221,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int h = ew >> 2;                    // 128-column half of the tile
     const int tl = (ew & 3) * 32 + lane;      // thread index among the half's 4 warps
     const int row_t = q * 32 + lane;
+    pdl_wait();  // count, idx, X_OT and c_x come from the activation pass
     const int cnt = *a.count;
     const int cs = min(cnt, OUT_CAP);         // outliers staged in shared memory
     float* wo = reinterpret_cast<float*>(smem + WO_OFFSET) + h * OUT_CAP * HALF_N;  // [OUT_CAP][HALF_N]
@@ -352,7 +373,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }  // namespace
 
 cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
-                               cudaStream_t stream) {
+                               bool pdl, cudaStream_t stream) {
   static unsigned long long attr_set = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -365,8 +386,17 @@ cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, c
   }
   const int num_tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
   const int grid = std::max(1, std::min(num_tiles, num_sms));
-  gemm_i8_decomp_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemm_i8_decomp_kernel, tmA, tmB, a);
 }
 
 }  // namespace i8mm

@@ -27,29 +27,30 @@ cudaError_t launch_weight_prep(const __half* W, int64_t K, int64_t N, uint32_t* 
 
 // ---- activation passes (every forward) -----------------------------------
 struct OutlierScratch {
-  uint16_t* partial;          // [rows_chunks][K] per-chunk column maxima (|x| bits)
-  unsigned* stripe_ticket;    // [ceil(K/256)], zero between launches
-  unsigned* all_ticket;       // [1], zero between launches
-  uint32_t* mask;             // [ceil(K/32)] outlier column bitmask
-  int32_t* idx;               // [K] ascending outlier columns
-  int32_t* count;             // [1] |O|
-  float* colmax;              // [K] max_i |X[i,j]|
+  unsigned long long* colkey;  // [K] (epoch << 16) | max |x| bits; never cleared
+  unsigned long long* epoch;   // [1] epoch of the next launch (the last block advances it)
+  unsigned* ticket;            // [1] zero between launches
+  uint32_t* mask;              // [ceil(K/32)] outlier column bitmask
+  int32_t* pre;                // [ceil(K/32)] exclusive prefix of popc over the mask words
+  int32_t* idx;                // [K] ascending outlier columns
+  int32_t* count;              // [1] |O|
+  float* colmax;               // [K] max_i |X[i,j]|
 };
 
-// Number of row chunks the outlier pass splits M rows into, and an upper
-// bound on it for every M' <= M (sizes `partial`).
-int outlier_row_chunks(int64_t M, int64_t K, int num_sms);
-int outlier_row_chunks_bound(int64_t M, int64_t K, int num_sms);
-
 // Pass 1: column maxima of X and the outlier set O = {j : colmax_j > alpha}.
+// Blocks fold their chunk maxima into colkey with 64-bit atomicMax; keys of
+// earlier launches carry a smaller epoch, so colkey needs no clearing.  The
+// last block (ticket) writes colmax, mask, pre, idx and count.
 cudaError_t launch_outlier_detect(const __half* X, int64_t M, int64_t K, float alpha,
-                                  const OutlierScratch& s, int num_sms, cudaStream_t stream);
+                                  const OutlierScratch& s, cudaStream_t stream);
 
 // Pass 2: per row, absmax over non-outlier columns, c_x = 127/absmax, int8
-// codes (outlier columns 0), and the fp16 outlier values gathered as
-// X_OT[o][i] = X[i, idx[o]] (o-major, M entries per o).
+// codes (outlier columns 0), and the fp16 outlier values scattered as
+// X_OT[o][i] = X[i, idx[o]] (o-major, M entries per o).  With `pdl`,
+// launched as a programmatic dependent of pass 1: it loads its row of X
+// while that pass finishes.
 cudaError_t launch_row_quant(const __half* X, int64_t M, int64_t K, const OutlierScratch& s,
-                             int8_t* Xq, float* c_x, __half* X_OT, cudaStream_t stream);
+                             int8_t* Xq, float* c_x, __half* X_OT, bool pdl, cudaStream_t stream);
 
 // ---- fused tcgen05 GEMM ---------------------------------------------------
 struct GemmArgs {
@@ -72,7 +73,9 @@ struct GemmArgs {
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 128;
+// With `pdl`, launched as a programmatic dependent of the row pass: its
+// prologue and the first weight-tile loads overlap that pass.
 cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
-                               int num_sms, cudaStream_t stream);
+                               int num_sms, bool pdl, cudaStream_t stream);
 
 }  // namespace i8mm

@@ -6,9 +6,9 @@
 // allocate after warm-up, or a process whose caching allocator has already
 // reserved nearly all of the device memory, so that a fresh cudaMalloc (or a
 // stream-ordered allocation) fails or fragments the pool.  For them this file
-// runs the outlier-detection kernel with its scratch (per-chunk column
-// maxima, completion tickets and the column bitmask) in a fixed static
-// device array instead of a handle-owned workspace.
+// runs the outlier-detection kernel with its scratch (epoch-tagged column
+// maxima, the completion ticket, the column bitmask and its word prefix) in a
+// fixed static device array instead of a handle-owned workspace.
 //
 // The array is kNoAllocScratchBytes (1 MiB) per device.  It is part of the
 // library's device image, so every GPU that loads the library holds it until
@@ -28,17 +28,22 @@
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = INT8MM_NOALLOC_SCRATCH_BYTES;
-constexpr size_t kTicketBytes = 2048;     // stripe tickets (<= 256) + 1 grid ticket
-constexpr size_t kMaskBytes = 8192;       // ceil(65536 / 32) words
-constexpr size_t kColmaxBytes = 262144;   // 65536 fp32, used when the caller passes none
-constexpr size_t kPartialOffset = kTicketBytes + kMaskBytes + kColmaxBytes;
+// Layout of the array (byte offsets): ticket and epoch, then the column keys,
+// the bitmask, its word prefix, and column maxima for callers that pass none.
+constexpr size_t kTicketOffset = 0;                       // u32, cleared by every call
+constexpr size_t kEpochOffset = 8;                        // u64, grows from call to call
+constexpr size_t kColkeyOffset = 256;                     // 65536 u64
+constexpr size_t kMaskOffset = kColkeyOffset + 65536 * 8; // 2048 u32
+constexpr size_t kPreOffset = kMaskOffset + 2048 * 4;     // 2048 i32
+constexpr size_t kColmaxOffset = kPreOffset + 2048 * 4;   // 65536 fp32
+constexpr size_t kScratchUsed = kColmaxOffset + 65536 * 4;
+static_assert(kScratchUsed <= kNoAllocScratchBytes, "layout fits the static array");
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
-int g_num_sms[kMaxDevices] = {};
 
 int8mm_status setup_error(int8mm_status s, const std::string& msg) {
   i8mm::set_last_error(msg);  // reported by int8mm_last_error()
@@ -47,22 +52,16 @@ int8mm_status setup_error(int8mm_status s, const std::string& msg) {
 
 // Once per device, with that device current: the device address of the
 // static scratch array (its host-side name is only a stand-in).
-int8mm_status device_scratch(int dev, void** ptr, int* num_sms) {
+int8mm_status device_scratch(int dev, void** ptr) {
   std::lock_guard<std::mutex> g(g_setup_mu);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess)
       return setup_error(INT8MM_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
-    int sms = 0;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess)
-      return setup_error(INT8MM_ERR_CUDA, std::string("device query: ") + cudaGetErrorString(e));
-    g_num_sms[dev] = sms;
     g_scratch_ptr[dev] = p;
   }
   *ptr = g_scratch_ptr[dev];
-  *num_sms = g_num_sms[dev];
   return INT8MM_OK;
 }
 
@@ -82,6 +81,8 @@ int8mm_status int8mm_outlier_columns_noalloc(const void* X_fp16_dev, int64_t M, 
     return setup_error(INT8MM_ERR_UNSUPPORTED_SHAPE,
                        "K=" + std::to_string(K) + ": the no-allocation detection needs 16 <= K <= " +
                            std::to_string(INT8MM_MAX_K) + ", a multiple of 16");
+  if (((K + 255) / 256) * ((M + 63) / 64) >= (int64_t(1) << 31))
+    return setup_error(INT8MM_ERR_UNSUPPORTED_SHAPE, "M is too large for one detection launch");
   if ((reinterpret_cast<uintptr_t>(X_fp16_dev) & 15u) != 0)
     return setup_error(INT8MM_ERR_ALIGNMENT, "X must be 16-byte aligned");
   int dev = 0;
@@ -89,8 +90,7 @@ int8mm_status int8mm_outlier_columns_noalloc(const void* X_fp16_dev, int64_t M, 
   if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return setup_error(INT8MM_ERR_CUDA, "no usable current CUDA device");
   void* base = nullptr;
-  int sms = 0;
-  int8mm_status st = device_scratch(dev, &base, &sms);
+  int8mm_status st = device_scratch(dev, &base);
   if (st != INT8MM_OK) return st;
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -99,26 +99,22 @@ int8mm_status int8mm_outlier_columns_noalloc(const void* X_fp16_dev, int64_t M, 
       return setup_error(INT8MM_ERR_CUDA, std::string("count reset: ") + cudaGetErrorString(e));
     return INT8MM_OK;
   }
-  const int chunks = i8mm::outlier_row_chunks(M, K, sms);
-  const size_t partial_bytes = static_cast<size_t>(chunks) * static_cast<size_t>(K) * sizeof(uint16_t);
-  if (kPartialOffset + partial_bytes > kNoAllocScratchBytes)
-    return setup_error(INT8MM_ERR_UNSUPPORTED_SHAPE,
-                       "scratch of " + std::to_string(kPartialOffset + partial_bytes) +
-                           " bytes exceeds the static " + std::to_string(kNoAllocScratchBytes) + " bytes");
-
   unsigned char* s = static_cast<unsigned char*>(base);
-  // The array keeps the previous call's contents: the tickets must start at 0.
-  if ((e = cudaMemsetAsync(s, 0, kTicketBytes, cs)) != cudaSuccess)
+  // The array keeps the previous call's contents.  The ticket must start at
+  // zero; the column keys need no clearing (each call raises the epoch that
+  // its keys carry).
+  if ((e = cudaMemsetAsync(s + kTicketOffset, 0, sizeof(unsigned), cs)) != cudaSuccess)
     return setup_error(INT8MM_ERR_CUDA, std::string("ticket reset: ") + cudaGetErrorString(e));
   i8mm::OutlierScratch sc;
-  sc.stripe_ticket = reinterpret_cast<unsigned*>(s);
-  sc.all_ticket = reinterpret_cast<unsigned*>(s) + 256;
-  sc.mask = reinterpret_cast<uint32_t*>(s + kTicketBytes);
-  sc.colmax = colmax_dev ? colmax_dev : reinterpret_cast<float*>(s + kTicketBytes + kMaskBytes);
-  sc.partial = reinterpret_cast<uint16_t*>(s + kPartialOffset);
+  sc.ticket = reinterpret_cast<unsigned*>(s + kTicketOffset);
+  sc.epoch = reinterpret_cast<unsigned long long*>(s + kEpochOffset);
+  sc.colkey = reinterpret_cast<unsigned long long*>(s + kColkeyOffset);
+  sc.mask = reinterpret_cast<uint32_t*>(s + kMaskOffset);
+  sc.pre = reinterpret_cast<int32_t*>(s + kPreOffset);
+  sc.colmax = colmax_dev ? colmax_dev : reinterpret_cast<float*>(s + kColmaxOffset);
   sc.idx = idx_dev;
   sc.count = count_dev;
-  if ((e = i8mm::launch_outlier_detect(static_cast<const __half*>(X_fp16_dev), M, K, alpha, sc, sms, cs)) !=
+  if ((e = i8mm::launch_outlier_detect(static_cast<const __half*>(X_fp16_dev), M, K, alpha, sc, cs)) !=
       cudaSuccess)
     return setup_error(INT8MM_ERR_CUDA, std::string("outlier detection launch: ") + cudaGetErrorString(e));
   return INT8MM_OK;

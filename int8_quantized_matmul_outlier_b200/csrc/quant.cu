@@ -36,6 +36,57 @@ __device__ __forceinline__ float scale_from_absmax_bits(uint32_t bits) {
 
 __device__ __forceinline__ uint32_t max_pair(uint32_t m) { return max(m & 0xffffu, m >> 16); }
 
+// rne(x * c) as int8 in the low byte.  |x| <= absmax and c = 127/absmax
+// bound |x * c| by 127 (1 + 2^-24), which rounds to at most 127, so the
+// saturating conversion equals the clamp to [-127, 127] exactly.
+__device__ __forceinline__ uint32_t q8(float x, float c) {
+  int32_t q;
+  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(q) : "f"(__fmul_rn(x, c)));
+  return static_cast<uint32_t>(q);
+}
+
+// Eight halves -> eight int8 codes, as two little-endian words.
+__device__ __forceinline__ uint2 quant8(const uint4& v, float c) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+  const float2 f0 = __half22float2(h[0]), f1 = __half22float2(h[1]);
+  const float2 f2 = __half22float2(h[2]), f3 = __half22float2(h[3]);
+  const uint32_t a01 = __byte_perm(q8(f0.x, c), q8(f0.y, c), 0x0040);
+  const uint32_t a23 = __byte_perm(q8(f1.x, c), q8(f1.y, c), 0x0040);
+  const uint32_t b01 = __byte_perm(q8(f2.x, c), q8(f2.y, c), 0x0040);
+  const uint32_t b23 = __byte_perm(q8(f3.x, c), q8(f3.y, c), 0x0040);
+  return make_uint2(__byte_perm(a01, a23, 0x5410), __byte_perm(b01, b23, 0x5410));
+}
+
+// Bits 0..3 of n -> 0xff in bytes 0..3 of the result.
+__device__ __forceinline__ uint32_t expand_nibble(uint32_t n) {
+  return ((n * 0x00204081u) & 0x01010101u) * 0xffu;
+}
+
+// Max of the magnitudes of the halves of v whose flag bit is clear.
+__device__ __forceinline__ uint32_t masked_absmax2(uint32_t m, const uint4& v, uint32_t fl) {
+  if (fl == 0) {
+    m = __vmaxu2(m, v.x & 0x7fff7fffu);
+    m = __vmaxu2(m, v.y & 0x7fff7fffu);
+    m = __vmaxu2(m, v.z & 0x7fff7fffu);
+    return __vmaxu2(m, v.w & 0x7fff7fffu);
+  }
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const uint32_t keep = (((fl >> (2 * p)) & 1u) ? 0u : 0x0000ffffu) | (((fl >> (2 * p + 1)) & 1u) ? 0u : 0xffff0000u);
+    m = __vmaxu2(m, w[p] & 0x7fff7fffu & keep);
+  }
+  return m;
+}
+
+// Programmatic dependent launch: let the next kernel of the stream start its
+// prologue, and wait until the previous kernel's results are visible.  Both
+// are no-ops for a kernel launched without the programmatic attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------------
 // Weight prep, step 1: column absmax of W[K,N] into colmax_bits[N] (atomicMax
 // on the magnitude bits).  Block (32, 8): 32 threads x 8 columns = 256
@@ -131,97 +182,98 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(const __half* __restr
 }
 
 // ------------------------------------------------------------------------
-// Outlier detection.  Grid (ceil(K/256), chunks), block (32, 8).  Each block
-// reduces a 256-column stripe over one chunk of rows into `partial`.  The
-// last block to finish a stripe (ticket) reduces the chunks, writes colmax
-// and the stripe's 8 mask words; the last stripe to finish (second ticket)
-// compacts the mask into the ascending index list and the count.  Tickets
-// are returned to zero by the block that consumed them, so no per-launch
-// clearing is needed.
+// Outlier detection.  ceil(K/256) * ceil(M/64) blocks of (32, 8) threads: a
+// block covers a 256-column stripe of a 64-row chunk; thread (tx, ty) reads the
+// 8 columns tx*8.. of rows ty, ty+8, .., ty+56 with all 8 loads in flight.
+// Column maxima of the chunk are folded into colkey with one 64-bit
+// atomicMax per column; the key's high bits hold the launch epoch, so values
+// left by earlier launches always lose.  The last block to finish (ticket)
+// reads colkey and writes colmax, the outlier bitmask, the per-word prefix
+// of its popcounts, the ascending index list and the count, then advances
+// the epoch and returns the ticket to zero.
+constexpr int kDetectRowsPerThread = 8;
+constexpr int kDetectRowsPerBlock = 8 * kDetectRowsPerThread;
+
 __global__ void __launch_bounds__(256) outlier_detect_kernel(const __half* __restrict__ X, int M, int K,
-                                                             float alpha, int rows_per_chunk,
-                                                             OutlierScratch s) {
+                                                             float alpha, OutlierScratch s) {
   const int tx = threadIdx.x, ty = threadIdx.y, tid = ty * 32 + tx;
-  const int stripe = blockIdx.x;
-  const int col = stripe * 256 + tx * 8;
-  const int r0 = blockIdx.y * rows_per_chunk;
-  const int r1 = min(M, r0 + rows_per_chunk);
+  const int stripes = (K + 255) / 256;
+  const int col = (static_cast<int>(blockIdx.x) % stripes) * 256 + tx * 8;
+  const int r0 = (static_cast<int>(blockIdx.x) / stripes) * kDetectRowsPerBlock;
+  const unsigned long long epoch = __ldcg(s.epoch);
   uint32_t m[4] = {0, 0, 0, 0};
   if (col < K) {
-    const __half* base = X + col;
-    int r = r0 + ty;
-    for (; r + 24 < r1; r += 32) {
-      uint4 v[4];
+    uint4 v[kDetectRowsPerThread];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        v[u] = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(r + 8 * u) * K));
+    for (int u = 0; u < kDetectRowsPerThread; ++u) {
+      const int r = r0 + ty + 8 * u;
+      v[u] = r < M ? __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K + col))
+                   : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        m[0] = __vmaxu2(m[0], v[u].x & 0x7fff7fffu);
-        m[1] = __vmaxu2(m[1], v[u].y & 0x7fff7fffu);
-        m[2] = __vmaxu2(m[2], v[u].z & 0x7fff7fffu);
-        m[3] = __vmaxu2(m[3], v[u].w & 0x7fff7fffu);
+    for (int u = 0; u < kDetectRowsPerThread; ++u) {
+      m[0] = __vmaxu2(m[0], v[u].x & 0x7fff7fffu);
+      m[1] = __vmaxu2(m[1], v[u].y & 0x7fff7fffu);
+      m[2] = __vmaxu2(m[2], v[u].z & 0x7fff7fffu);
+      m[3] = __vmaxu2(m[3], v[u].w & 0x7fff7fffu);
+    }
+  }
+  __shared__ uint16_t red[8][256];  // [row lane][column of the stripe]
+  __shared__ unsigned s_last;
+  __shared__ int s_words[2048];       // popcount per mask word, then its prefix
+  __shared__ int s_scan[8];
+  {
+    uint4 mv = make_uint4(m[0], m[1], m[2], m[3]);
+    *reinterpret_cast<uint4*>(&red[ty][tx * 8]) = mv;
+  }
+  __syncthreads();
+  {
+    // thread tid owns column tid of the stripe: one atomic per column
+    const int c = (static_cast<int>(blockIdx.x) % stripes) * 256 + tid;
+    if (c < K) {
+      uint32_t v = red[0][tid];
+#pragma unroll
+      for (int y = 1; y < 8; ++y) v = max(v, static_cast<uint32_t>(red[y][tid]));
+      atomicMax(s.colkey + c, (epoch << 16) | v);
+      __threadfence();  // the atomic is ordered before the ticket below
+    }
+  }
+  pdl_launch_dependents();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(s.ticket, 1u) == gridDim.x - 1) ? 1u : 0u;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  // Last block: column maxima, bitmask and word popcounts, 256 columns per
+  // sweep with 16 sweeps' loads in flight.
+  const int nwords = (K + 31) / 32;
+  for (int base = 0; base < K; base += 16 * 256) {
+    unsigned long long key[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int c = base + u * 256 + tid;
+      key[u] = c < K ? __ldcg(s.colkey + c) : 0ull;
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int c = base + u * 256 + tid;
+      const float cm = __half2float(__ushort_as_half(static_cast<unsigned short>(key[u] & 0xffffu)));
+      if (c < K) s.colmax[c] = cm;
+      const unsigned word = __ballot_sync(0xffffffffu, c < K && cm > alpha);
+      const int w = (base + u * 256) / 32 + ty;
+      if (tx == 0 && w < nwords) {
+        s.mask[w] = word;
+        s_words[w] = __popc(word);
       }
     }
-    for (; r < r1; r += 8) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + static_cast<size_t>(r) * K));
-      m[0] = __vmaxu2(m[0], v.x & 0x7fff7fffu);
-      m[1] = __vmaxu2(m[1], v.y & 0x7fff7fffu);
-      m[2] = __vmaxu2(m[2], v.z & 0x7fff7fffu);
-      m[3] = __vmaxu2(m[3], v.w & 0x7fff7fffu);
-    }
   }
-  __shared__ uint32_t red[8][32][4];
-  __shared__ unsigned s_last;
-  __shared__ int s_scan[8];
-#pragma unroll
-  for (int p = 0; p < 4; ++p) red[ty][tx][p] = m[p];
   __syncthreads();
-  if (ty == 0 && col < K) {
-    uint4 out;
-    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      uint32_t v = red[0][tx][p];
-      for (int y = 1; y < 8; ++y) v = __vmaxu2(v, red[y][tx][p]);
-      o[p] = v;
-    }
-    *reinterpret_cast<uint4*>(s.partial + static_cast<size_t>(blockIdx.y) * K + col) = out;
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(s.stripe_ticket + stripe, 1u) == gridDim.y - 1) ? 1u : 0u;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  // Last block of this stripe: reduce the chunks, one column per thread.
-  {
-    const int c = stripe * 256 + tid;
-    uint32_t mx = 0;
-    if (c < K) {
-      for (int ch = 0; ch < static_cast<int>(gridDim.y); ++ch)
-        mx = max(mx, static_cast<uint32_t>(__ldcg(s.partial + static_cast<size_t>(ch) * K + c)));
-    }
-    const float cm = __half2float(__ushort_as_half(static_cast<unsigned short>(mx)));
-    if (c < K) s.colmax[c] = cm;
-    const unsigned word = __ballot_sync(0xffffffffu, (c < K) && (cm > alpha));
-    if (tx == 0 && c < K) s.mask[c >> 5] = word;
-    if (tid == 0) s.stripe_ticket[stripe] = 0;
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(s.all_ticket, 1u) == gridDim.x - 1) ? 1u : 0u;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  // Last stripe overall: compact the bitmask into ascending indices.
-  const int nwords = (K + 31) / 32;
+  // exclusive prefix over the words: thread t takes a run of words
   const int wpt = (nwords + 255) / 256;
   const int w0 = min(nwords, tid * wpt), w1 = min(nwords, w0 + wpt);
   int cnt = 0;
-  for (int w = w0; w < w1; ++w) cnt += __popc(__ldcg(s.mask + w));
+  for (int w = w0; w < w1; ++w) cnt += s_words[w];
   int incl = cnt;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -239,6 +291,7 @@ __global__ void __launch_bounds__(256) outlier_detect_kernel(const __half* __res
   }
   int pos = before + incl - cnt;
   for (int w = w0; w < w1; ++w) {
+    s.pre[w] = pos;
     uint32_t bits = __ldcg(s.mask + w);
     while (bits) {
       const int b = __ffs(bits) - 1;
@@ -248,18 +301,19 @@ __global__ void __launch_bounds__(256) outlier_detect_kernel(const __half* __res
   }
   if (tid == 0) {
     *s.count = total;
-    *s.all_ticket = 0;
+    *s.epoch = epoch + 1;
+    *s.ticket = 0;
   }
 }
 
 // ------------------------------------------------------------------------
 // Row quantisation: one block per row of X; each thread holds VPT vectors
-// of 8 halves in registers between the absmax and the quantise steps.
+// of 8 halves in registers between the absmax and the quantise steps.  The
+// slot of an outlier entry is pre[word] + (set bits below it in its word).
 template <int VPT, int NT>
 __global__ void __launch_bounds__(NT) row_quant_kernel(const __half* __restrict__ X, int M, int K,
                                                        const uint32_t* __restrict__ mask,
-                                                       const int32_t* __restrict__ idx,
-                                                       const int32_t* __restrict__ count,
+                                                       const int32_t* __restrict__ pre,
                                                        int8_t* __restrict__ Xq, float* __restrict__ c_x,
                                                        __half* __restrict__ X_OT) {
   const int row = blockIdx.x, tid = threadIdx.x;
@@ -267,23 +321,20 @@ __global__ void __launch_bounds__(NT) row_quant_kernel(const __half* __restrict_
   const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(row) * K);
   uint4 v[VPT];
   uint32_t fl[VPT];
+  // X is an input of the forward, not a result of the detection pass: load
+  // the row before waiting for that pass to finish.
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int c8 = tid + i * NT;
+    v[i] = c8 < nvec ? __ldg(xr + c8) : make_uint4(0, 0, 0, 0);
+  }
+  pdl_wait();
   uint32_t m = 0;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int c8 = tid + i * NT;
-    fl[i] = 0xffu;
-    v[i] = make_uint4(0, 0, 0, 0);
-    if (c8 < nvec) {
-      v[i] = __ldg(xr + c8);
-      fl[i] = (__ldg(mask + (c8 >> 2)) >> ((c8 & 3) * 8)) & 0xffu;
-    }
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(&v[i]);
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const uint32_t keep = (((fl[i] >> (2 * p)) & 1u) ? 0u : 0x0000ffffu) |
-                            (((fl[i] >> (2 * p + 1)) & 1u) ? 0u : 0xffff0000u);
-      m = __vmaxu2(m, w[p] & 0x7fff7fffu & keep);
-    }
+    fl[i] = c8 < nvec ? (__ldcg(mask + (c8 >> 2)) >> ((c8 & 3) * 8)) & 0xffu : 0xffu;
+    m = masked_absmax2(m, v[i], fl[i]);
   }
   m = max_pair(m);
   m = __reduce_max_sync(0xffffffffu, m);
@@ -307,31 +358,41 @@ __global__ void __launch_bounds__(NT) row_quant_kernel(const __half* __restrict_
   for (int i = 0; i < VPT; ++i) {
     const int c8 = tid + i * NT;
     if (c8 < nvec) {
-      const __half2* h = reinterpret_cast<const __half2*>(&v[i]);
-      uint32_t lo = 0, hi = 0;
+      uint2 q = quant8(v[i], c);
+      if (fl[i]) {  // outlier columns: code 0, and the fp16 value goes to its slot
+        q.x &= ~expand_nibble(fl[i] & 0xfu);
+        q.y &= ~expand_nibble(fl[i] >> 4);
+        const int w = c8 >> 2, sh = (c8 & 3) * 8;
+        int o = __ldcg(pre + w) + __popc(__ldcg(mask + w) & ((1u << sh) - 1u));
+        const unsigned short* hs = reinterpret_cast<const unsigned short*>(&v[i]);
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const float2 f = __half22float2(h[p]);
-        const uint32_t a = ((fl[i] >> (2 * p)) & 1u) ? 0u : static_cast<uint8_t>(quant_rne(f.x, c));
-        const uint32_t b = ((fl[i] >> (2 * p + 1)) & 1u) ? 0u : static_cast<uint8_t>(quant_rne(f.y, c));
-        const uint32_t pair = a | (b << 8);
-        if (p < 2) lo |= pair << (16 * p);
-        else hi |= pair << (16 * (p - 2));
+        for (int e = 0; e < 8; ++e)
+          if ((fl[i] >> e) & 1u) {
+            X_OT[static_cast<size_t>(o) * M + row] = __ushort_as_half(hs[e]);
+            ++o;
+          }
       }
-      *reinterpret_cast<uint2*>(qr + c8 * 8) = make_uint2(lo, hi);
+      *reinterpret_cast<uint2*>(qr + c8 * 8) = q;
     }
   }
-  const int cnt = *count;
-  for (int o = tid; o < cnt; o += NT)
-    X_OT[static_cast<size_t>(o) * M + row] = X[static_cast<size_t>(row) * K + idx[o]];
+  pdl_launch_dependents();
 }
 
 template <int VPT, int NT>
 cudaError_t launch_row_quant_t(const __half* X, int64_t M, int64_t K, const OutlierScratch& s, int8_t* Xq,
-                               float* c_x, __half* X_OT, cudaStream_t stream) {
-  row_quant_kernel<VPT, NT><<<static_cast<unsigned>(M), NT, 0, stream>>>(
-      X, static_cast<int>(M), static_cast<int>(K), s.mask, s.idx, s.count, Xq, c_x, X_OT);
-  return cudaGetLastError();
+                               float* c_x, __half* X_OT, bool pdl, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(M));
+  cfg.blockDim = dim3(NT);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, row_quant_kernel<VPT, NT>, X, static_cast<int>(M), static_cast<int>(K),
+                            static_cast<const uint32_t*>(s.mask), static_cast<const int32_t*>(s.pre), Xq, c_x,
+                            X_OT);
 }
 
 }  // namespace
@@ -355,44 +416,33 @@ cudaError_t launch_weight_prep(const __half* W, int64_t K, int64_t N, uint32_t* 
   return cudaGetLastError();
 }
 
-namespace {
-int64_t chunk_target(int64_t M, int64_t K, int num_sms) {
-  const int64_t stripes = (K + 255) / 256;
-  const int64_t chunks = std::max<int64_t>(1, (4 * num_sms + stripes - 1) / stripes);
-  return std::max<int64_t>(1, std::min<int64_t>(chunks, (M + 7) / 8));
-}
-}  // namespace
-
-int outlier_row_chunks(int64_t M, int64_t K, int num_sms) {
-  const int64_t chunks = chunk_target(M, K, num_sms);
-  const int64_t rows_per_chunk = (M + chunks - 1) / chunks;
-  return static_cast<int>((M + rows_per_chunk - 1) / rows_per_chunk);
-}
-
-int outlier_row_chunks_bound(int64_t M, int64_t K, int num_sms) {
-  // non-decreasing in M and >= outlier_row_chunks(M', K) for every M' <= M
-  return static_cast<int>(chunk_target(M, K, num_sms));
-}
-
 cudaError_t launch_outlier_detect(const __half* X, int64_t M, int64_t K, float alpha, const OutlierScratch& s,
-                                  int num_sms, cudaStream_t stream) {
-  const int stripes = static_cast<int>((K + 255) / 256);
-  const int chunks = outlier_row_chunks(M, K, num_sms);
-  const int rows_per_chunk = static_cast<int>((M + chunks - 1) / chunks);
-  outlier_detect_kernel<<<dim3(stripes, chunks), dim3(32, 8), 0, stream>>>(
-      X, static_cast<int>(M), static_cast<int>(K), alpha, rows_per_chunk, s);
+                                  cudaStream_t stream) {
+  const int64_t stripes = (K + 255) / 256;
+  const int64_t chunks = (M + kDetectRowsPerBlock - 1) / kDetectRowsPerBlock;
+  outlier_detect_kernel<<<static_cast<unsigned>(stripes * chunks), dim3(32, 8), 0, stream>>>(
+      X, static_cast<int>(M), static_cast<int>(K), alpha, s);
   return cudaGetLastError();
 }
 
 cudaError_t launch_row_quant(const __half* X, int64_t M, int64_t K, const OutlierScratch& s, int8_t* Xq,
-                             float* c_x, __half* X_OT, cudaStream_t stream) {
+                             float* c_x, __half* X_OT, bool pdl, cudaStream_t stream) {
+  // 128 threads per row up to K = 16384, then 256 and 512; each thread
+  // keeps VPT vectors of 8 halves of its row in registers.
   const int64_t nvec = K / 8;
-  if (nvec <= 256 * 1) return launch_row_quant_t<1, 256>(X, M, K, s, Xq, c_x, X_OT, stream);
-  if (nvec <= 256 * 2) return launch_row_quant_t<2, 256>(X, M, K, s, Xq, c_x, X_OT, stream);
-  if (nvec <= 256 * 4) return launch_row_quant_t<4, 256>(X, M, K, s, Xq, c_x, X_OT, stream);
-  if (nvec <= 256 * 8) return launch_row_quant_t<8, 256>(X, M, K, s, Xq, c_x, X_OT, stream);
-  if (nvec <= 256 * 16) return launch_row_quant_t<16, 256>(X, M, K, s, Xq, c_x, X_OT, stream);
-  if (nvec <= 512 * 16) return launch_row_quant_t<16, 512>(X, M, K, s, Xq, c_x, X_OT, stream);
+#define I8MM_ROWQ(V, T) \
+  if (nvec <= int64_t(V) * (T)) return launch_row_quant_t<V, T>(X, M, K, s, Xq, c_x, X_OT, pdl, stream)
+  I8MM_ROWQ(1, 128);
+  I8MM_ROWQ(2, 128);
+  I8MM_ROWQ(3, 128);
+  I8MM_ROWQ(4, 128);
+  I8MM_ROWQ(6, 128);
+  I8MM_ROWQ(8, 128);
+  I8MM_ROWQ(12, 128);
+  I8MM_ROWQ(16, 128);
+  I8MM_ROWQ(16, 256);
+  I8MM_ROWQ(16, 512);
+#undef I8MM_ROWQ
   return cudaErrorInvalidValue;
 }
 

@@ -150,10 +150,10 @@ def test_events_time_each_kernel():
     W = torch.from_numpy(p.W).to(dev())
     w = m.int8mm_prepare_weight(W)
     Y = torch.empty((256, 1024), dtype=torch.float16, device=dev())
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     m.int8mm_forward_events(w, X, p.alpha, Y, ev)
     torch.cuda.synchronize()
-    t = [ev[i].elapsed_time(ev[i + 1]) for i in range(3)]
+    t = [ev[i].elapsed_time(ev[i + 1]) for i in range(2)]
     assert all(x >= 0 for x in t) and sum(t) > 0
     assert torch.equal(Y, m.int8mm_forward(w, X, p.alpha))
 
