@@ -98,17 +98,17 @@ def gemm_source_hash() -> str:
 
 
 def recorded_traffic(workload: str):
-    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
-    taken on the current GEMM source (else None)."""
-    path = os.path.join(ROOT, "profiles", "gemm_i8_decomp_traffic.md")
-    if not os.path.exists(path):
-        return None
-    text = open(path, encoding="utf-8").read()
-    src = re.search(r"gemm_source_sha256_16:\s*([0-9a-f]+)", text)
-    if not src or src.group(1) != gemm_source_hash():
-        return None
-    m = re.search(rf"traffic_bytes_per_launch\[{re.escape(workload)}\]:\s*([0-9.eE+]+)", text)
-    return float(m.group(1)) if m else None
+    """DRAM bytes per GEMM launch from a committed ncu summary
+    (profiles/gemm_i8_decomp_*.md), if it was taken on the current GEMM
+    source (else None)."""
+    import glob
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "gemm_i8_decomp_*.md"))):
+        text = open(path, encoding="utf-8").read()
+        src = re.search(r"gemm_source_sha256_16:\s*([0-9a-f]+)", text)
+        m = re.search(rf"traffic_bytes_per_launch\[{re.escape(workload)}\]:\s*([0-9.eE+]+)", text)
+        if src and m and src.group(1) == gemm_source_hash():
+            return float(m.group(1))
+    return None
 
 
 class ClockSampler:
@@ -227,6 +227,24 @@ def cpu_baseline(p: workloads.Problem, rows: int) -> dict:
 
 # --------------------------------------------------------------------------
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Maximum of x over all ranks of the default process group (x itself
+    when no group is initialised).  NCCL needs a CUDA device tensor; gloo
+    (CPU tests) a CPU one."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(ops_per_step: float, steps: int, world: int, max_total_ms: float) -> float:
+    """Whole-job TOPS: the operations of all ranks over the slowest rank's time."""
+    return ops_per_step * steps * world / (max_total_ms * 1e-3) / 1e12
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -284,13 +302,6 @@ def run_ours(args):
         if distributed:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if not distributed:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     p = make_problem(args.config, rank)
     M, K, N = p.shape
     X = torch.from_numpy(p.X).to(dev)
@@ -325,12 +336,12 @@ def run_ours(args):
         raise RuntimeError("device wait timed out in the timed region")
     seg = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(2)] for e in ev])  # ms
     step_ms = seg.sum(axis=1)
-    total_ms = max_over_ranks(float(step_ms.sum()))
+    total_ms = max_over_ranks(float(step_ms.sum()), dev)
     ms_per_step = total_ms / steps
     flops = 2.0 * M * N * K
-    value = flops * steps * world / (total_ms * 1e-3) / 1e12
-    gemm_ms = max_over_ranks(float(seg[:, 1].mean()))
-    xprep_ms = max_over_ranks(float(seg[:, 0].mean()))
+    value = job_throughput(flops, steps, world, total_ms)
+    gemm_ms = max_over_ranks(float(seg[:, 1].mean()), dev)
+    xprep_ms = max_over_ranks(float(seg[:, 0].mean()), dev)
 
     # end to end through the host-buffer entry point: pinned X in, pinned Y out
     Xh = torch.from_numpy(p.X).pin_memory()
@@ -348,8 +359,8 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
-    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+    e2e_value = job_throughput(flops, 1, world, e2e_ms)
 
     peaks = measured_peaks()
     peak_tops = peaks["bf16_tflops"] * INT8_PER_BF16
@@ -366,7 +377,7 @@ def run_ours(args):
             "peak_note": (f"dense int8 = {INT8_PER_BF16:g} x {peaks['source']} bf16 burst "
                           f"{peaks['bf16_tflops']:g} TFLOP/s; int8 ops counted as 2*M*N*K"),
         },
-        "kernels_ms": {"xprep (outlier detection + row quantisation)": xprep_ms, "gemm_i8_decomp": gemm_ms},
+        "kernels_ms": {"activation (outlier_detect + row_quant)": xprep_ms, "gemm_i8_decomp": gemm_ms},
         "pct_int8_peak_whole_step": 100.0 * value / world / peak_tops,
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": M * K * 2,
                 "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms,

@@ -298,3 +298,30 @@ def test_outlier_row_of_W_is_multiplied_by_zero_codes():
     # change in Y is close to X[:, j] * (W2[j,3] - W[j,3]) plus int8 requantisation
     d = p.X[:, j].astype(np.float64) * (float(W2[j, 3]) - float(p.W[j, 3]))
     assert np.abs(ex - d).max() < 0.05 * np.abs(d).max() + 0.02
+
+
+# --------------------------------------------------------------------------
+# the two comparators the harness reports errors against
+
+def test_matmul_f64_matches_numpy():
+    rng = np.random.default_rng(8)
+    X = (rng.integers(-512, 512, (7, 33)) / 128.0).astype(np.float16)
+    W = (rng.integers(-512, 512, (33, 5)) / 128.0).astype(np.float16)
+    ref = X.astype(np.float64) @ W.astype(np.float64)   # exact: small dyadic values
+    assert (oracle.matmul_f64(X, W) == ref).all()
+
+
+def test_tensorwise_absmax_hand_example():
+    # one scale for all of X (127/8) and one for all of W (127/2), no split:
+    # X = [[8, 1], [-4, 0.5]] -> codes [[127, 15.875->16], [-63.5->-64, 7.9375->8]]
+    # W = [[2, -1], [0.5, 1]]  -> codes [[127, -63.5->-64], [31.75->32, 63.5->64]]
+    X = np.array([[8, 1], [-4, 0.5]], np.float16)
+    W = np.array([[2, -1], [0.5, 1]], np.float16)
+    r = oracle.tensorwise_absmax(X, W)
+    assert r["c_x"] == np.float32(127 / 8) and r["c_w"] == np.float32(63.5)
+    assert r["qx"].tolist() == [[127, 16], [-64, 8]]
+    assert r["qw"].tolist() == [[127, -64], [32, 64]]
+    # acc row 0: [127*127 + 16*32, 127*-64 + 16*64] = [16641, -7104]
+    # y = acc / (15.875 * 63.5) = acc / 1008.0625 -> [16.5078.., -7.0472..]
+    acc = np.array([[16641, -7104], [-64 * 127 + 8 * 32, -64 * -64 + 8 * 64]], np.float64)
+    assert (r["Y"].astype(np.float64) == (acc / (15.875 * 63.5)).astype(np.float16)).all()
