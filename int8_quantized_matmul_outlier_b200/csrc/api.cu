@@ -24,11 +24,16 @@ struct int8mm_weight {
   int num_sms = 148;
   int64_t K = 0, N = 0;
   const __half* W = nullptr;  // borrowed fp16 weight [K, N]
-  int8_t* Wq_t = nullptr;     // [N, K] int8 codes, K-major
+  int64_t N_pad = 0;          // N rounded up to kWeightRowPad
+  int8_t* Wb = nullptr;       // [K/128][N_pad][128] int8 codes, K-blocked
   float* c_w = nullptr;       // [N]
   float* inv_cw = nullptr;    // [N]
   uint32_t* colmax_bits = nullptr;  // [N] prep scratch
-  CUtensorMap tmB;
+  CUtensorMap tmB;     // Wb, 256-row boxes (prefill GEMM operand B)
+  CUtensorMap tmW128;  // Wb, 128-row boxes (decode GEMM operand A)
+  // decode (M <= 64) scratch: int32 partial sums and per-n-block tickets
+  int32_t* part = nullptr;
+  unsigned* dticket = nullptr;
   // fixed-size scratch of the outlier pass
   unsigned long long* colkey = nullptr;  // [K]
   unsigned long long* epoch = nullptr;   // [1]
@@ -44,10 +49,11 @@ struct int8mm_weight {
   int8_t* Xq = nullptr;
   float* c_x = nullptr;
   __half* X_OT = nullptr;
-  // tensor map of Xq for the current (pointer, M)
+  // tensor map of Xq for the current (pointer, M, box rows)
   CUtensorMap tmA;
   const void* tmA_ptr = nullptr;
   int64_t tmA_rows = -1;
+  int tmA_box = 0;
   // device copies for host-buffer forwards
   int64_t io_rows = 0;
   __half* dX = nullptr;
@@ -142,7 +148,9 @@ void free_all(int8mm_weight* h) {
   free_workspace(h);
   release(&h->dX);
   release(&h->dY);
-  release(&h->Wq_t);
+  release(&h->part);
+  release(&h->dticket);
+  release(&h->Wb);
   release(&h->c_w);
   release(&h->inv_cw);
   release(&h->colmax_bits);
@@ -225,10 +233,26 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
   if (M == 0) return INT8MM_OK;
   if ((st = set_device(h)) != INT8MM_OK) return st;
   if ((st = ensure_workspace(h, M, s)) != INT8MM_OK) return st;
-  if (h->tmA_ptr != h->Xq || h->tmA_rows != M) {
-    if ((st = make_tmap_i8(&h->tmA, h->Xq, h->K, M, kGemmBK, kGemmBM)) != INT8MM_OK) return st;
+  const bool decode = M <= kDecodeMaxM;
+  const int box_rows = decode ? decode_padded_tokens(M) : kGemmBM;
+  if (h->tmA_ptr != h->Xq || h->tmA_rows != M || h->tmA_box != box_rows) {
+    if ((st = make_tmap_i8(&h->tmA, h->Xq, h->K, M, kGemmBK, box_rows)) != INT8MM_OK) return st;
     h->tmA_ptr = h->Xq;
     h->tmA_rows = M;
+    h->tmA_box = box_rows;
+  }
+  if (decode && h->part == nullptr) {
+    const size_t nb = static_cast<size_t>((h->N + 127) / 128);
+    cudaError_t ea;
+    if ((ea = alloc(&h->part, static_cast<size_t>(kDecodeMaxM) * h->N, s, &h->bytes)) != cudaSuccess ||
+        (ea = alloc(&h->dticket, nb, s, &h->bytes)) != cudaSuccess ||
+        (ea = cudaMemsetAsync(h->part, 0, static_cast<size_t>(kDecodeMaxM) * h->N * 4, s)) != cudaSuccess ||
+        (ea = cudaMemsetAsync(h->dticket, 0, nb * 4, s)) != cudaSuccess) {
+      cudaStreamSynchronize(s);
+      release(&h->part);
+      release(&h->dticket);
+      return cuda_fail(ea, "decode scratch allocation");
+    }
   }
   OutlierScratch sc{h->colkey, h->epoch, h->ticket, h->mask, h->pre, h->idx, h->count, h->colmax};
   const __half* Xh = static_cast<const __half*>(X);
@@ -237,30 +261,59 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     if (events && events[i]) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
   };
   rec(0);
-  if ((e = launch_outlier_detect(Xh, M, h->K, alpha, sc, s)) != cudaSuccess)
-    return cuda_fail(e, "outlier detection launch");
-  if ((e = launch_row_quant(Xh, M, h->K, sc, h->Xq, h->c_x, h->X_OT, /*pdl=*/true, s)) != cudaSuccess)
-    return cuda_fail(e, "row quantisation launch");
+  if (decode && small_act_fits(M, h->K)) {
+    SmallActArgs sa{Xh, static_cast<int>(M), static_cast<int>(h->K), alpha, h->Xq, h->c_x, h->X_OT,
+                    h->colmax, h->idx, h->count};
+    if ((e = launch_small_act(sa, s)) != cudaSuccess) return cuda_fail(e, "activation pass launch");
+  } else {
+    if ((e = launch_outlier_detect(Xh, M, h->K, alpha, sc, s)) != cudaSuccess)
+      return cuda_fail(e, "outlier detection launch");
+    if ((e = launch_row_quant(Xh, M, h->K, sc, h->Xq, h->c_x, h->X_OT, /*pdl=*/true, s)) != cudaSuccess)
+      return cuda_fail(e, "row quantisation launch");
+  }
   rec(1);
-  GemmArgs a;
-  a.M = static_cast<int>(M);
-  a.N = static_cast<int>(h->N);
-  a.K = static_cast<int>(h->K);
-  a.c_x = h->c_x;
-  a.inv_cw = h->inv_cw;
-  a.W = h->W;
-  a.X_OT = h->X_OT;
-  a.idx = h->idx;
-  a.count = h->count;
-  a.Y = static_cast<__half*>(Y);
-  a.acc_dump = dbg ? dbg->acc : nullptr;
-  a.status = h->status;
-  a.timeout_ns = h->timeout_ns;
   // Without events between them, the GEMM is a programmatic dependent of the
   // row pass; an event record in between makes it an ordinary launch.
   const bool pdl = !(events && events[1]);
-  if ((e = launch_gemm_decomp(h->tmA, h->tmB, a, h->num_sms, pdl, s)) != cudaSuccess)
-    return cuda_fail(e, "int8 GEMM launch");
+  if (decode) {
+    DecodeArgs d;
+    d.M = static_cast<int>(M);
+    d.N = static_cast<int>(h->N);
+    d.K = static_cast<int>(h->K);
+    d.N_pad = static_cast<int>(h->N_pad);
+    d.c_x = h->c_x;
+    d.inv_cw = h->inv_cw;
+    d.W = h->W;
+    d.X_OT = h->X_OT;
+    d.idx = h->idx;
+    d.count = h->count;
+    d.Y = static_cast<__half*>(Y);
+    d.acc_dump = dbg ? dbg->acc : nullptr;
+    d.part = h->part;
+    d.ticket = h->dticket;
+    d.status = h->status;
+    d.timeout_ns = h->timeout_ns;
+    if ((e = launch_gemm_decode(h->tmW128, h->tmA, d, h->num_sms, pdl, s)) != cudaSuccess)
+      return cuda_fail(e, "int8 decode GEMM launch");
+  } else {
+    GemmArgs a;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(h->N);
+    a.K = static_cast<int>(h->K);
+    a.N_pad = static_cast<int>(h->N_pad);
+    a.c_x = h->c_x;
+    a.inv_cw = h->inv_cw;
+    a.W = h->W;
+    a.X_OT = h->X_OT;
+    a.idx = h->idx;
+    a.count = h->count;
+    a.Y = static_cast<__half*>(Y);
+    a.acc_dump = dbg ? dbg->acc : nullptr;
+    a.status = h->status;
+    a.timeout_ns = h->timeout_ns;
+    if ((e = launch_gemm_decomp(h->tmA, h->tmB, a, h->num_sms, pdl, s)) != cudaSuccess)
+      return cuda_fail(e, "int8 GEMM launch");
+  }
   rec(2);
   if (dbg) {
     const size_t K = static_cast<size_t>(h->K), N = static_cast<size_t>(h->N), Mz = static_cast<size_t>(M);
@@ -270,12 +323,21 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
       size_t n;
     } cps[] = {
         {dbg->colmax, h->colmax, K * 4},  {dbg->outlier_idx, h->idx, K * 4}, {dbg->outlier_count, h->count, 4},
-        {dbg->x_codes, h->Xq, Mz * K},    {dbg->c_x, h->c_x, Mz * 4},        {dbg->w_codes_t, h->Wq_t, N * K},
+        {dbg->x_codes, h->Xq, Mz * K},    {dbg->c_x, h->c_x, Mz * 4},
         {dbg->c_w, h->c_w, N * 4},
     };
     for (const C& c : cps)
       if (c.dst && (e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
         return cuda_fail(e, "debug copy");
+    if (dbg->w_codes_t) {  // K-blocked [K/128][N_pad][128] -> [N, K]
+      for (size_t kb = 0; kb * 128 < K; ++kb) {
+        const size_t width = std::min<size_t>(128, K - kb * 128);
+        if ((e = cudaMemcpy2DAsync(static_cast<int8_t*>(dbg->w_codes_t) + kb * 128, K,
+                                   h->Wb + kb * static_cast<size_t>(h->N_pad) * 128, 128, width, N,
+                                   cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+          return cuda_fail(e, "debug copy of the weight codes");
+      }
+    }
   }
   return INT8MM_OK;
 }
@@ -296,6 +358,9 @@ int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N
                 "K=%lld, N=%lld: need 16 <= K <= %d and N >= 16, both multiples of 16", (long long)K,
                 (long long)N, INT8MM_MAX_K);
   if (!aligned16(W_fp16_dev)) return fail(INT8MM_ERR_ALIGNMENT, "W must be 16-byte aligned");
+  if ((K + 127) / 128 * ((N + kWeightRowPad - 1) / kWeightRowPad * kWeightRowPad) >= (int64_t(1) << 31))
+    return fail(INT8MM_ERR_UNSUPPORTED_SHAPE, "K=%lld x N=%lld exceeds the weight layout's 2^31 rows of 128 bytes",
+                (long long)K, (long long)N);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int8mm_weight* h = new int8mm_weight();
   cudaError_t e = cudaGetDevice(&h->device);
@@ -310,7 +375,10 @@ int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N
   const size_t Kz = static_cast<size_t>(K), Nz = static_cast<size_t>(N);
   const size_t words = (Kz + 31) / 32;
   size_t* tot = &h->bytes;
-  if ((e = alloc(&h->Wq_t, Nz * Kz, s, tot)) != cudaSuccess || (e = alloc(&h->c_w, Nz, s, tot)) != cudaSuccess ||
+  h->N_pad = (N + kWeightRowPad - 1) / kWeightRowPad * kWeightRowPad;
+  const size_t kblocks = (Kz + 127) / 128;
+  const size_t wb_bytes = kblocks * static_cast<size_t>(h->N_pad) * 128;
+  if ((e = alloc(&h->Wb, wb_bytes, s, tot)) != cudaSuccess || (e = alloc(&h->c_w, Nz, s, tot)) != cudaSuccess ||
       (e = alloc(&h->inv_cw, Nz, s, tot)) != cudaSuccess || (e = alloc(&h->colmax_bits, Nz, s, tot)) != cudaSuccess ||
       (e = alloc(&h->colkey, Kz, s, tot)) != cudaSuccess || (e = alloc(&h->epoch, 1, s, tot)) != cudaSuccess ||
       (e = alloc(&h->ticket, 1, s, tot)) != cudaSuccess || (e = alloc(&h->mask, words, s, tot)) != cudaSuccess ||
@@ -322,20 +390,23 @@ int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N
     delete h;
     return cuda_fail(e, "weight allocation");
   }
-  if ((e = cudaMemsetAsync(h->colkey, 0, Kz * 8, s)) != cudaSuccess ||
+  if ((e = cudaMemsetAsync(h->Wb, 0, wb_bytes, s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(h->colkey, 0, Kz * 8, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->epoch, 0, 8, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->ticket, 0, 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->mask, 0, words * 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->count, 0, 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->status, 0, 4, s)) != cudaSuccess ||
-      (e = launch_weight_prep(h->W, K, N, h->colmax_bits, h->Wq_t, h->c_w, h->inv_cw, h->num_sms, s)) !=
+      (e = launch_weight_prep(h->W, K, N, h->colmax_bits, h->Wb, h->N_pad, h->c_w, h->inv_cw, h->num_sms, s)) !=
           cudaSuccess) {
     cudaStreamSynchronize(s);
     free_all(h);
     delete h;
     return cuda_fail(e, "weight preparation");
   }
-  int8mm_status st = make_tmap_i8(&h->tmB, h->Wq_t, Kz, Nz, kGemmBK, kGemmBN);
+  const uint64_t wb_rows = kblocks * static_cast<uint64_t>(h->N_pad);
+  int8mm_status st = make_tmap_i8(&h->tmB, h->Wb, 128, wb_rows, kGemmBK, kGemmBN);
+  if (st == INT8MM_OK) st = make_tmap_i8(&h->tmW128, h->Wb, 128, wb_rows, kGemmBK, 128);
   if (st != INT8MM_OK) {
     cudaStreamSynchronize(s);
     free_all(h);
@@ -422,7 +493,13 @@ int8mm_status int8mm_get_status(int8mm_weight_t h) {
     return cuda_fail(e, "status read");
   if ((e = cudaMemset(h->status, 0, 4)) != cudaSuccess) return cuda_fail(e, "status reset");
   if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "device synchronise");
-  if (word & kStatusTimeout) return fail(INT8MM_ERR_TIMEOUT, "a device wait ran out of time");
+  if (word & kStatusTimeout) {
+    // an aborted decode GEMM may leave partial sums and tickets behind
+    if (h->part) cudaMemset(h->part, 0, static_cast<size_t>(kDecodeMaxM) * h->N * 4);
+    if (h->dticket) cudaMemset(h->dticket, 0, static_cast<size_t>((h->N + 127) / 128) * 4);
+    cudaDeviceSynchronize();
+    return fail(INT8MM_ERR_TIMEOUT, "a device wait ran out of time");
+  }
   return INT8MM_OK;
 }
 

@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int pre = first < num_tiles ? min(STAGES, num_kb) : 0;
       for (int kb = 0; kb < pre; ++kb) {
         mbar_arrive_expect_tx(&full[kb], STAGE_BYTES);
-        tma_load_2d(smem + kb * STAGE_BYTES + A_BYTES, &tmB, &full[kb], kb * BK, (first / num_m) * BN);
+        tma_load_2d(smem + kb * STAGE_BYTES + A_BYTES, &tmB, &full[kb], 0, kb * a.N_pad + (first / num_m) * BN);
       }
       pdl_wait();
       for (int kb = 0; kb < pre; ++kb) {
@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t* sa = smem + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
           tma_load_2d(sa, &tmA, &full[stage], kb * BK, m_blk * BM);
-          tma_load_2d(sa + A_BYTES, &tmB, &full[stage], kb * BK, n_blk * BN);
+          tma_load_2d(sa + A_BYTES, &tmB, &full[stage], 0, kb * a.N_pad + n_blk * BN);
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {

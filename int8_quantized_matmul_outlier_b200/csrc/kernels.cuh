@@ -18,12 +18,14 @@ void set_last_error(const std::string& message);
 
 // ---- weight preparation (once per weight) --------------------------------
 // Per output column j of W[K,N] (fp16, row-major): absmax over all K rows,
-// c_w[j] = 127/absmax, codes rne(w * c_w) clamped to +-127, written
-// transposed as Wq_t[N,K] (K-major, the tensor-core operand layout).
-// colmax_bits is [N] u32 scratch; it is zeroed here.
-cudaError_t launch_weight_prep(const __half* W, int64_t K, int64_t N, uint32_t* colmax_bits,
-                               int8_t* Wq_t, float* c_w, float* inv_cw, int num_sms,
-                               cudaStream_t stream);
+// c_w[j] = 127/absmax, codes rne(w * c_w) clamped to +-127, written in the
+// K-blocked, K-major layout Wb[kb][n][0..128) (kb = k / 128, n < N_pad, N_pad
+// a multiple of 256; codes past K or N are 0), so that every tensor-core
+// operand tile of 128 or 256 rows is one contiguous block of memory.  Wb
+// must be zeroed before.  colmax_bits is [N] u32 scratch; it is zeroed here.
+constexpr int kWeightRowPad = 256;
+cudaError_t launch_weight_prep(const __half* W, int64_t K, int64_t N, uint32_t* colmax_bits, int8_t* Wb,
+                               int64_t N_pad, float* c_w, float* inv_cw, int num_sms, cudaStream_t stream);
 
 // ---- activation passes (every forward) -----------------------------------
 struct OutlierScratch {
@@ -55,6 +57,7 @@ cudaError_t launch_row_quant(const __half* X, int64_t M, int64_t K, const Outlie
 // ---- fused tcgen05 GEMM ---------------------------------------------------
 struct GemmArgs {
   int M, N, K;
+  int N_pad;               // rows per k block in the weight layout
   const float* c_x;        // [M]
   const float* inv_cw;     // [N] 1/c_w (0 where c_w == 0)
   const __half* W;         // [K,N] fp16, rows of the outlier set are read
@@ -67,15 +70,67 @@ struct GemmArgs {
   unsigned long long timeout_ns;
 };
 
-// Y = (Xq Wq_t^T) / (c_x c_w^T) + X[:,O] W[O,:].  tmA maps Xq [M,K] int8,
-// tmB maps Wq_t [N,K] int8, both with 128x128-byte swizzled boxes
-// (tmB's box is kGemmBN rows).
+// Y = (Xq Wq^T) / (c_x c_w^T) + X[:,O] W[O,:].  tmA maps Xq [M,K] int8 with
+// 128x128-byte swizzled boxes; tmB maps the K-blocked weight Wb as a 2-D
+// array of (K/128 * N_pad) rows of 128 bytes with kGemmBN-row boxes (the box
+// of n block j at k block kb starts at row kb * N_pad + j * kGemmBN).
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 128;
 // With `pdl`, launched as a programmatic dependent of the row pass: its
 // prologue and the first weight-tile loads overlap that pass.
 cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
+                               int num_sms, bool pdl, cudaStream_t stream);
+
+// Largest K any kernel here accepts (the row kernels keep a row in registers).
+constexpr int64_t kMaxK = 65536;
+// Forwards with at most this many rows take the few-token path.
+constexpr int kDecodeMaxM = 64;
+
+// ---- activation pass for few tokens (M <= kDecodeMaxM) ---------------------
+// One thread-block cluster does detection, quantisation and the outlier
+// gather in one launch (csrc/xact_small.cu); it writes colmax, idx, count,
+// Xq, c_x and X_OT (not mask/pre).  It lets a programmatic dependent launch
+// (the decode GEMM) start at once.
+struct SmallActArgs {
+  const __half* X;  // [M, K]
+  int M, K;
+  float alpha;
+  int8_t* Xq;       // [M, K]
+  float* c_x;       // [M]
+  __half* X_OT;     // [|O|][M]
+  float* colmax;    // [K]
+  int32_t* idx;     // [K]
+  int32_t* count;   // [1]
+};
+constexpr size_t kSmallActSmemMax = 200 * 1024;
+// Whether an M x K activation takes the single-cluster kernel.
+bool small_act_fits(int64_t M, int64_t K);
+cudaError_t launch_small_act(const SmallActArgs& a, cudaStream_t stream);
+
+// ---- decode-shape GEMM (M <= 64 tokens) -----------------------------------
+struct DecodeArgs {
+  int M, N, K;
+  int N_pad;               // rows per k block in the weight layout
+  const float* c_x;        // [M]
+  const float* inv_cw;     // [N]
+  const __half* W;         // [K,N] fp16 (outlier rows are read)
+  const __half* X_OT;      // [|O|][M]
+  const int32_t* idx;      // [K]
+  const int32_t* count;    // [1]
+  __half* Y;               // [M,N]
+  int32_t* acc_dump;       // [M,N] or nullptr
+  int32_t* part;           // [64][N] int32 partial sums, zero between launches
+  unsigned* ticket;        // [ceil(N/128)] k-steps done per n block, zero between launches
+  int* status;
+  unsigned long long timeout_ns;
+};
+// Tokens padded to the MMA N of the decode kernel: 16, 32 or 64.
+int decode_padded_tokens(int64_t M);
+// tmW maps the K-blocked weight (rows of 128 bytes) with 128-row boxes; tmX
+// maps Xq [M,K] with 128 x decode_padded_tokens(M) boxes.  With `pdl`, the first weight tiles
+// stream while the activation pass finishes.
+cudaError_t launch_gemm_decode(const CUtensorMap& tmW, const CUtensorMap& tmX, const DecodeArgs& a,
                                int num_sms, bool pdl, cudaStream_t stream);
 
 }  // namespace i8mm

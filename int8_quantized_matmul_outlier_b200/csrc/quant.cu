@@ -123,13 +123,13 @@ __global__ void __launch_bounds__(256) weight_colmax_kernel(const __half* __rest
 }
 
 // Weight prep, step 2: codes of a 128(k) x 128(n) tile, transposed through
-// shared memory so that both the fp16 reads (along n) and the int8 writes
-// (along k) are 16-byte vectors.  Blocks with blockIdx.y == 0 also write
-// c_w and 1/c_w.
+// shared memory, written to the K-blocked layout Wb[kb][n][0..128): the tile
+// is one contiguous 16 KB block (codes beyond K are 0).  Blocks with
+// blockIdx.y == 0 also write c_w and 1/c_w.
 __global__ void __launch_bounds__(256) weight_quant_kernel(const __half* __restrict__ W, int K, int N,
                                                            const uint32_t* __restrict__ colmax_bits,
-                                                           int8_t* __restrict__ Wq_t, float* __restrict__ c_w,
-                                                           float* __restrict__ inv_cw) {
+                                                           int8_t* __restrict__ Wb, int N_pad,
+                                                           float* __restrict__ c_w, float* __restrict__ inv_cw) {
   __shared__ float cs[128];
   __shared__ __align__(16) int8_t tile[128][144];  // [n][k], rows padded to 144 B
   const int tid = threadIdx.x;
@@ -168,16 +168,15 @@ __global__ void __launch_bounds__(256) weight_quant_kernel(const __half* __restr
     for (int e = 0; e < 8; ++e) tile[cg + e][kl] = q[e];
   }
   __syncthreads();
-  // 8 threads x 16 bytes per n-row, 32 rows per pass, 4 passes.
+  // 8 threads x 16 bytes per n-row, 32 rows per pass, 4 passes; the block
+  // writes 16 KB of consecutive memory.
+  int8_t* dst = Wb + (static_cast<size_t>(blockIdx.y) * N_pad + n0) * 128;
 #pragma unroll
   for (int pass = 0; pass < 4; ++pass) {
     const int nl = pass * 32 + (tid >> 3);
     const int kc = (tid & 7) * 16;
-    const int n = n0 + nl, k = k0 + kc;
-    if (n < N && k < K) {
-      *reinterpret_cast<uint4*>(Wq_t + static_cast<size_t>(n) * K + k) =
-          *reinterpret_cast<const uint4*>(&tile[nl][kc]);
-    }
+    if (n0 + nl < N)
+      *reinterpret_cast<uint4*>(dst + nl * 128 + kc) = *reinterpret_cast<const uint4*>(&tile[nl][kc]);
   }
 }
 
@@ -398,8 +397,8 @@ cudaError_t launch_row_quant_t(const __half* X, int64_t M, int64_t K, const Outl
 }  // namespace
 
 // ------------------------------------------------------------------------
-cudaError_t launch_weight_prep(const __half* W, int64_t K, int64_t N, uint32_t* colmax_bits, int8_t* Wq_t,
-                               float* c_w, float* inv_cw, int num_sms, cudaStream_t stream) {
+cudaError_t launch_weight_prep(const __half* W, int64_t K, int64_t N, uint32_t* colmax_bits, int8_t* Wb,
+                               int64_t N_pad, float* c_w, float* inv_cw, int num_sms, cudaStream_t stream) {
   cudaError_t e = cudaMemsetAsync(colmax_bits, 0, static_cast<size_t>(N) * sizeof(uint32_t), stream);
   if (e != cudaSuccess) return e;
   const int stripes = static_cast<int>((N + 255) / 256);
@@ -411,8 +410,8 @@ cudaError_t launch_weight_prep(const __half* W, int64_t K, int64_t N, uint32_t* 
       W, static_cast<int>(K), static_cast<int>(N), rows_per_chunk, colmax_bits);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   weight_quant_kernel<<<dim3(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>((K + 127) / 128)),
-                        256, 0, stream>>>(W, static_cast<int>(K), static_cast<int>(N), colmax_bits, Wq_t,
-                                          c_w, inv_cw);
+                        256, 0, stream>>>(W, static_cast<int>(K), static_cast<int>(N), colmax_bits, Wb,
+                                          static_cast<int>(N_pad), c_w, inv_cw);
   return cudaGetLastError();
 }
 

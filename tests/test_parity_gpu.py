@@ -81,6 +81,10 @@ SHAPES = [
     (33, 4096, 1024, 7, 6.0),
     (130, 2064, 2320, 9, 6.0),
     (513, 640, 4112, 3, 6.0),       # many N tiles, ragged N tail
+    (64, 1040, 784, 3, 6.0),        # largest decode-kernel M, ragged 128-column blocks
+    (65, 1040, 784, 3, 6.0),        # smallest prefill-kernel M
+    (40, 2048, 4112, 5, 6.0),       # decode kernel, stream-K splits across blocks
+    (8, 12288, 1024, 7, 6.0),       # decode, long K: whole and split blocks
 ]
 
 
@@ -127,6 +131,23 @@ def test_repeat_and_stale_state():
     b = check(p0, w=w, wq=wq)
     c = check(p1, w=w, wq=wq)
     assert (a["cnt"], b["cnt"], c["cnt"]) == (6, 0, 6)
+    assert torch.equal(a["d"]["Y"], c["d"]["Y"])
+
+
+@pytest.mark.parametrize("M", [1, 16, 40])
+def test_decode_repeat_and_stale_partials(M):
+    # split n blocks leave int32 partial sums and tickets behind for the next call
+    K, N = 2048, 1168
+    W = workloads.weight(K, N, 77)
+    pa = workloads.small(M, K, N, 4, seed=78)
+    pb = workloads.small(M, K, N, 0, seed=79)
+    pa.W = pb.W = W
+    w = m.int8mm_prepare_weight(torch.from_numpy(W).to(dev()))
+    wq = oracle.quantize_cols(W)
+    a = check(pa, w=w, wq=wq, check_w_codes=False)
+    b = check(pb, w=w, wq=wq, check_w_codes=False)
+    c = check(pa, w=w, wq=wq, check_w_codes=False)
+    assert (a["cnt"], b["cnt"], c["cnt"]) == (4, 0, 4)
     assert torch.equal(a["d"]["Y"], c["d"]["Y"])
 
 
