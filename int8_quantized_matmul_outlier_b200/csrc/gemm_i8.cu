@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float* wo = reinterpret_cast<float*>(smem + WO_OFFSET) + h * OUT_CAP * HALF_N;  // [OUT_CAP][HALF_N]
     float* rws = reinterpret_cast<float*>(smem + RW_OFFSET) + h * HALF_N;           // [HALF_N]
     const uint32_t bar_id = 1 + h;
+    const bool y32 = (reinterpret_cast<uintptr_t>(a.Y) & 31u) == 0;
     bool alive = true;
     int lt = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
@@ -345,11 +346,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const __half2 hh = __floats2half2_rn(v[2 * p], v[2 * p + 1]);
             ou[p] = *reinterpret_cast<const uint32_t*>(&hh);
           }
-          yp[0] = out[0];
-          yp[1] = out[1];
-          if (full32) {
-            yp[2] = out[2];
-            yp[3] = out[3];
+          if (y32) {  // whole 32-byte sectors per store
+            st_global_256(yp, out[0], out[1]);
+            if (full32) st_global_256(yp + 2, out[2], out[3]);
+          } else {
+            yp[0] = out[0];
+            yp[1] = out[1];
+            if (full32) {
+              yp[2] = out[2];
+              yp[3] = out[3];
+            }
           }
           if (a.acc_dump != nullptr) {
             uint4* ap = reinterpret_cast<uint4*>(a.acc_dump + static_cast<size_t>(m) * N + n);

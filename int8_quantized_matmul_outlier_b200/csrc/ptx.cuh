@@ -99,6 +99,15 @@ __device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// 32-byte global store (sm_100), not allocating in L1; p must be 32-byte aligned.
+__device__ __forceinline__ void st_global_256(void* p, const uint4& lo, const uint4& hi) {
+  asm volatile("st.global.L1::no_allocate.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+               "f"(__uint_as_float(lo.x)), "f"(__uint_as_float(lo.y)), "f"(__uint_as_float(lo.z)),
+               "f"(__uint_as_float(lo.w)), "f"(__uint_as_float(hi.x)), "f"(__uint_as_float(hi.y)),
+               "f"(__uint_as_float(hi.z)), "f"(__uint_as_float(hi.w))
+               : "memory");
+}
+
 // ----------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem_slot, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
