@@ -311,7 +311,7 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     a.acc_dump = dbg ? dbg->acc : nullptr;
     a.status = h->status;
     a.timeout_ns = h->timeout_ns;
-    if ((e = launch_gemm_decomp(h->tmA, h->tmB, a, h->num_sms, pdl, s)) != cudaSuccess)
+    if ((e = launch_gemm_decomp(h->tmA, h->tmB, h->tmW128, a, h->num_sms, pdl, s)) != cudaSuccess)
       return cuda_fail(e, "int8 GEMM launch");
   }
   rec(2);

@@ -11,12 +11,12 @@
 // int8 cuBLAS GEMM followed by a separate fp16 GEMM; here both, and the
 // dequantisation, run in one persistent kernel.
 //
-// Structure (one CTA per SM, 6 warps):
-//   warp 0      TMA producer: 128x128 A tiles (Xq) and 256x128 B tiles (Wq^T),
+// Structure (one CTA per SM, 10 warps):
+//   warp 0      TMA producer: 128x128 A tiles (Xq) and B tiles (Wq, K-blocked),
 //               128-byte swizzled, into a STAGES-deep shared-memory ring;
 //   warp 1      allocates 512 TMEM columns; one thread issues
-//               tcgen05.mma.kind::i8 (128x256x32) into a double-buffered
-//               int32 accumulator (2 x 256 columns);
+//               tcgen05.mma.kind::i8 into a double-buffered int32
+//               accumulator (2 x 256 columns);
 //   warps 2-9   epilogue, two warps per TMEM lane quarter (warp w reads lanes
 //               32*(w%4)..+31, one output row per thread), each covering one
 //               128-column half of the tile: tcgen05.ld of the accumulator,
@@ -26,6 +26,15 @@
 //               memory and load their rows' outlier activations.
 // The epilogue of tile t overlaps the main loop of tile t+1.  Every wait is
 // bounded; a timeout sets the status word and the CTA drains and exits.
+//
+// Two modes.  Single CTA (M <= 128): 128x256 tiles, B tiles of 256 rows,
+// 4 stages.  CTA pair (M > 128): a cluster of two CTAs on neighbouring SMs
+// computes a 256x256 tile with tcgen05.mma.cta_group::2 (256x256x32) issued
+// by the leader; each CTA loads its own 128 rows of A and 128 rows of B
+// (TMA completing on the leader's barrier), keeps its 128 accumulator rows in
+// its own TMEM and writes them; commits reach both CTAs' barriers.  Each SM
+// then streams 32 KB instead of 48 KB per 128x256x128 of MMA work, in a
+// 6-stage ring.  No TMA multicast is used.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -35,28 +44,38 @@ namespace i8mm {
 namespace {
 
 constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK;  // 16 KB
-constexpr int B_BYTES = BN * BK;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
-constexpr int NUM_BARS = 2 * STAGES + 5;  // full, empty, tmem_full[2], tmem_empty[2], drain
-constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
+constexpr int A_BYTES = BM * BK;  // 16 KB: 128 rows of A per CTA
 // Epilogue staging: per 128-column half of the tile, the first OUT_CAP
 // outlier rows W[idx[o], cols] and 1/c_w[cols] as fp32.
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int HALF_N = BN / 2;
 constexpr int OUT_CAP = 16;
-constexpr int WO_OFFSET = (MISC_OFFSET + 16 + 15) & ~15;
 constexpr int WO_BYTES = 2 * OUT_CAP * HALF_N * 4;
-constexpr int RW_OFFSET = WO_OFFSET + WO_BYTES;
 constexpr int RW_BYTES = 2 * HALF_N * 4;
-constexpr int SMEM_BYTES = RW_OFFSET + RW_BYTES + 1024;  // + slack to align the base to 1024
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
-static_assert(SMEM_BYTES <= 232448, "fits the 227 KB of shared memory per block");
-constexpr uint32_t IDESC = idesc_i8(BM, BN);
 static_assert(TMEM_COLS == 512, "two 128x256 int32 accumulators fill TMEM");
+
+// Single CTA: 128x256 tile, 4 stages of A (16 KB) + B (32 KB).  CTA pair:
+// 256x256 tile, each CTA holding 128 rows of A and 128 rows of B, 6 stages
+// of 32 KB: a third less operand traffic per SM for the same MMA work.
+template <bool PAIR>
+struct Cfg {
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // rows of B per CTA
+  static constexpr int B_BYTES = B_ROWS * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int TILE_M = PAIR ? 2 * BM : BM;  // rows per tile
+  static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 5;  // full, empty, tmem_full[2], tmem_empty[2], drain
+  static constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
+  static constexpr int WO_OFFSET = (MISC_OFFSET + 16 + 15) & ~15;
+  static constexpr int RW_OFFSET = WO_OFFSET + WO_BYTES;
+  static constexpr int SMEM_BYTES = RW_OFFSET + RW_BYTES + 1024;  // + slack to align the base to 1024
+  static constexpr uint32_t IDESC = idesc_i8(TILE_M, BN);
+  static_assert(SMEM_BYTES <= 232448, "fits the 227 KB of shared memory per block");
+  static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-byte aligned for the 128B swizzle");
+};
 
 __device__ __forceinline__ void fail(const GemmArgs& a, volatile int* abort_flag) {
   *abort_flag = 1;
@@ -75,22 +94,30 @@ __device__ __forceinline__ float dequant(uint32_t acc, float rx, float rw) {
   return __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(acc)), rx), rw);
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_decomp_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const GemmArgs a) {
+  using C = Cfg<PAIR>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int STAGE_BYTES = C::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFFSET);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFFSET);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFFSET);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + MISC_OFFSET + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFFSET);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFFSET + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = a.M, N = a.N, K = a.K;
-  const int num_m = (M + BM - 1) / BM;
+  // a pair of CTAs (a cluster of 2) shares each tile; rank 0 issues the MMAs
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int tile0 = PAIR ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int tstride = PAIR ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
+  const int num_m = (M + C::TILE_M - 1) / C::TILE_M;
   const int num_n = (N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = (K + BK - 1) / BK;
@@ -102,7 +129,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], NUM_EPI_WARPS);
+      mbar_init(&tempty[b], NUM_EPI_WARPS * (PAIR ? 2 : 1));
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -111,11 +138,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const unsigned long long tmo = a.timeout_ns;
@@ -127,33 +160,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
       bool ok = true;
+      // In a pair both CTAs' loads complete on the leader's full barrier, and
+      // the leader alone announces the pair's bytes.
+      auto full_of = [&](int st) { return mapa_shared(smem_u32(&full[st]), 0); };
+      auto expect = [&](int st) {
+        if (!PAIR || rank == 0) mbar_arrive_expect_tx(&full[st], (PAIR ? 2 : 1) * STAGE_BYTES);
+      };
+      auto load_a = [&](int st, int kb, int m_blk) {
+        const int row = m_blk * C::TILE_M + static_cast<int>(rank) * BM;
+        if (PAIR) tma_load_2d_pair(smem + st * STAGE_BYTES, &tmA, full_of(st), kb * BK, row);
+        else tma_load_2d(smem + st * STAGE_BYTES, &tmA, &full[st], kb * BK, row);
+      };
+      auto load_b = [&](int st, int kb, int n_blk) {
+        const int row = kb * a.N_pad + n_blk * BN + static_cast<int>(rank) * C::B_ROWS;
+        if (PAIR) tma_load_2d_pair(smem + st * STAGE_BYTES + A_BYTES, &tmB, full_of(st), 0, row);
+        else tma_load_2d(smem + st * STAGE_BYTES + A_BYTES, &tmB, &full[st], 0, row);
+      };
       // The weight tiles of the first k-blocks do not depend on the
       // activation pass: issue them before waiting for it, then the
       // matching activation tiles (all stages start empty).
-      const int first = blockIdx.x;
+      const int first = tile0;
       const int pre = first < num_tiles ? min(STAGES, num_kb) : 0;
       for (int kb = 0; kb < pre; ++kb) {
-        mbar_arrive_expect_tx(&full[kb], STAGE_BYTES);
-        tma_load_2d(smem + kb * STAGE_BYTES + A_BYTES, &tmB, &full[kb], 0, kb * a.N_pad + (first / num_m) * BN);
+        expect(kb);
+        load_b(kb, kb, first / num_m);
       }
       pdl_wait();
       for (int kb = 0; kb < pre; ++kb) {
-        tma_load_2d(smem + kb * STAGE_BYTES, &tmA, &full[kb], kb * BK, (first % num_m) * BM);
+        load_a(kb, kb, first % num_m);
         issued_mask |= 1u << kb;
       }
       stage = pre % STAGES;
       phase = pre == STAGES ? 1u : 0u;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = tile0; tile < num_tiles && ok; tile += tstride) {
         const int m_blk = tile % num_m, n_blk = tile / num_m;
         for (int kb = tile == first ? pre : 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_2d(sa, &tmA, &full[stage], kb * BK, m_blk * BM);
-          tma_load_2d(sa + A_BYTES, &tmB, &full[stage], 0, kb * a.N_pad + n_blk * BN);
+          expect(stage);
+          load_a(stage, kb, m_blk);
+          load_b(stage, kb, n_blk);
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -164,19 +212,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok) {
         fail(a, abort_flag);
-        // Let every load already issued land before the CTA can exit.
-        for (int s = 0; s < STAGES; ++s)
-          if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, tmo, nullptr);
+        // Let every load already issued land before the CTA can exit (a
+        // pair's peer cannot watch the leader's barriers: it waits a while).
+        if (!PAIR || rank == 0) {
+          for (int s = 0; s < STAGES; ++s)
+            if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, tmo, nullptr);
+        } else {
+          const uint64_t t0 = global_timer_ns();
+          while (global_timer_ns() - t0 < 200000ull) {
+          }
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && (!PAIR || rank == 0)) {
       // -------------------------------------------------------- MMA issuer
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int lt = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++lt) {
+      for (int tile = tile0; tile < num_tiles && ok; tile += tstride, ++lt) {
         const int buf = lt & 1;
         const uint32_t use = static_cast<uint32_t>(lt >> 1);
         if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, tmo, abort_flag)) {
@@ -197,20 +252,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
             // advance 32 bytes along K inside the 128-byte swizzled row
-            mma_i8(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), IDESC,
-                   (kb | kk) != 0 ? 1u : 0u);
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            if (PAIR)
+              mma_i8_pair(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2),
+                          C::IDESC, acc);
+            else
+              mma_i8(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), C::IDESC,
+                     acc);
           }
-          mma_commit(&empty[stage]);
+          if (PAIR) mma_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
+          else mma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (ok) mma_commit(&tfull[buf]);
+        if (ok) {
+          if (PAIR) mma_commit_pair(&tfull[buf], 0x3);
+          else mma_commit(&tfull[buf]);
+        }
       }
       if (!ok) {
         fail(a, abort_flag);
-        mma_commit(drain);
+        if (PAIR) mma_commit_pair(drain, 0x1);
+        else mma_commit(drain);
         mbar_wait(drain, 0, tmo, nullptr);
       }
     }
@@ -224,18 +289,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     pdl_wait();  // count, idx, X_OT and c_x come from the activation pass
     const int cnt = *a.count;
     const int cs = min(cnt, OUT_CAP);         // outliers staged in shared memory
-    float* wo = reinterpret_cast<float*>(smem + WO_OFFSET) + h * OUT_CAP * HALF_N;  // [OUT_CAP][HALF_N]
-    float* rws = reinterpret_cast<float*>(smem + RW_OFFSET) + h * HALF_N;           // [HALF_N]
+    float* wo = reinterpret_cast<float*>(smem + C::WO_OFFSET) + h * OUT_CAP * HALF_N;  // [OUT_CAP][HALF_N]
+    float* rws = reinterpret_cast<float*>(smem + C::RW_OFFSET) + h * HALF_N;           // [HALF_N]
     const uint32_t bar_id = 1 + h;
     const bool y32 = (reinterpret_cast<uintptr_t>(a.Y) & 31u) == 0;
     bool alive = true;
     int lt = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
+    for (int tile = tile0; tile < num_tiles; tile += tstride, ++lt) {
       const int m_blk = tile % num_m, n_blk = tile / num_m;
       const int buf = lt & 1;
       const uint32_t use = static_cast<uint32_t>(lt >> 1);
       const int nh = n_blk * BN + h * HALF_N;  // first column of this half
-      const int m = m_blk * BM + row_t;
+      const int m = m_blk * C::TILE_M + static_cast<int>(rank) * BM + row_t;
       const bool row_ok = m < M;
 
       // (1) stage this tile's scales and outlier weight rows; this runs
@@ -289,7 +354,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (ch == HALF_N / 32 - 1) {  // accumulator buffer no longer read: release it
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf]);
+          if (lane == 0) {
+            if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));  // the leader's barrier
+            else mbar_arrive(&tempty[buf]);
+          }
         }
         const int n = nh + cl;
         if (n >= N) continue;  // warp-uniform
@@ -370,39 +438,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync_all();  // no CTA leaves while its peer may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
-}  // namespace
-
-cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
-                               bool pdl, cudaStream_t stream) {
+template <bool PAIR>
+cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms, bool pdl,
+                     cudaStream_t stream) {
+  using C = Cfg<PAIR>;
   static unsigned long long attr_set = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_i8_decomp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(gemm_i8_decomp_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set |= bit;
   }
-  const int num_tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
-  const int grid = std::max(1, std::min(num_tiles, num_sms));
+  const int num_tiles = ((a.M + C::TILE_M - 1) / C::TILE_M) * ((a.N + BN - 1) / BN);
+  const int units = PAIR ? num_sms / 2 : num_sms;
+  const int grid = std::max(1, std::min(num_tiles, units)) * (PAIR ? 2 : 1);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr.val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemm_i8_decomp_kernel, tmA, tmB, a);
+  cudaLaunchAttribute attrs[2];
+  int n = 0;
+  if (PAIR) {
+    attrs[n].id = cudaLaunchAttributeClusterDimension;
+    attrs[n].val.clusterDim.x = 2;
+    attrs[n].val.clusterDim.y = 1;
+    attrs[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl) {
+    attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attrs;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, gemm_i8_decomp_kernel<PAIR>, tmA, tmB, a);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB256, const CUtensorMap& tmB128,
+                               const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
+  // one 128-row tile height: single CTAs; taller problems: CTA pairs
+  if (a.M <= BM) return launch_t<false>(tmA, tmB256, a, num_sms, pdl, stream);
+  return launch_t<true>(tmA, tmB128, a, num_sms, pdl, stream);
 }
 
 }  // namespace i8mm

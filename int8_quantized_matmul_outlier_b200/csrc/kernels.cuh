@@ -77,10 +77,12 @@ struct GemmArgs {
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 128;
-// With `pdl`, launched as a programmatic dependent of the row pass: its
-// prologue and the first weight-tile loads overlap that pass.
-cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
-                               int num_sms, bool pdl, cudaStream_t stream);
+// tmB256 / tmB128 map the weight with 256- and 128-row boxes (the second is
+// used by the CTA-pair mode, for M > 128).  With `pdl`, launched as a
+// programmatic dependent of the row pass: its prologue and the first
+// weight-tile loads overlap that pass.
+cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB256, const CUtensorMap& tmB128,
+                               const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream);
 
 // Largest K any kernel here accepts (the row kernels keep a row in registers).
 constexpr int64_t kMaxK = 65536;
