@@ -57,6 +57,8 @@ def parse_args():
     ap.add_argument("--cpu-rows", type=int, default=0,
                     help="rows of the oracle CPU sample (0: sized to about 10 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=200,
+                    help="timed steps per decode shape (0 skips the decode measurement)")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -245,6 +247,49 @@ def job_throughput(ops_per_step: float, steps: int, world: int, max_total_ms: fl
     return ops_per_step * steps * world / (max_total_ms * 1e-3) / 1e12
 
 
+DECODE_K, DECODE_N, DECODE_MS = 12288, 49152, (1, 8, 32)
+
+
+def decode_algorithmic_bytes(M: int, K: int, N: int, n_out: int) -> int:
+    """Bytes a decode forward must move: the int8 weight, its fp32 scales, the
+    fp16 outlier rows of W, X in and Y out (intermediates excluded)."""
+    return N * K + 4 * N + 2 * n_out * N + 2 * M * K + 2 * M * N
+
+
+def run_decode(m, torch, dev, stream, scrub, steps: int, peaks: dict, max_over, rank: int):
+    """Decode steps (few tokens against the 175B-scale weight): each step one
+    forward, timed with events around it only, so the GEMM stays a
+    programmatic dependent launch of the activation pass."""
+    Wnp = workloads.weight(DECODE_K, DECODE_N, 3 * 1000 + 500_000 + rank)
+    W = torch.from_numpy(Wnp).to(dev)
+    del Wnp
+    w = m.int8mm_prepare_weight(W)
+    out = []
+    for M in DECODE_MS:
+        p = workloads.decode(M, repeat=rank, with_weight=False)
+        X = torch.from_numpy(p.X).to(dev)
+        Y = torch.empty((M, DECODE_N), dtype=torch.float16, device=dev)
+        for _ in range(5):
+            m.int8mm_forward(w, X, p.alpha, Y)
+            scrub.zero_()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        for e0, e1 in ev:
+            e0.record(stream)
+            m.int8mm_forward(w, X, p.alpha, Y)
+            e1.record(stream)
+            scrub.zero_()
+        torch.cuda.synchronize()
+        ms = max_over(float(np.mean([e0.elapsed_time(e1) for e0, e1 in ev])))
+        nbytes = decode_algorithmic_bytes(M, DECODE_K, DECODE_N, int(p.planted.size))
+        gbps = nbytes / (ms * 1e-3) / 1e9
+        out.append({"M": M, "K": DECODE_K, "N": DECODE_N, "ms_per_step": ms, "GBps": gbps,
+                    "frac_hbm": gbps / peaks["hbm_gbs"], "algorithmic_bytes": nbytes,
+                    "gpu_launches_per_step": 2})
+    m.int8mm_free(w)
+    return out
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -386,6 +431,14 @@ def run_ours(args):
         "clocks": clocks.summary(),
         "wall_s_timed_region": wall,
     }
+    if args.decode_steps > 0:
+        line["decode"] = {
+            "workload": "decode: M in (1, 8, 32) tokens x K=12288 x N=49152, 7 outlier columns in every row",
+            "timing": "CUDA events around each whole forward (no event between its kernels), L2 scrubbed "
+                      "between steps; GB/s = algorithmic bytes / step time, vs measured HBM copy bandwidth",
+            "hbm_peak_gbs": peaks["hbm_gbs"],
+            "shapes": run_decode(m, torch, dev, stream, scrub, args.decode_steps, peaks,
+                                 lambda x: max_over_ranks(x, dev), rank)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(p, args.cpu_rows)
     m.int8mm_free(w)
