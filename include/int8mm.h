@@ -94,11 +94,15 @@ int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream);
  * alpha: outlier threshold (6.0 in the pages); INFINITY disables the fp16
  *   path (pure vector-wise int8); any value below every |x| makes every
  *   column an outlier.  NaN is an argument error.
- * M == 0 is a no-op.  Three kernels run on `stream` (outlier detection, row
- * quantisation, fused int8 GEMM), the last two as programmatic dependent
- * launches that start while their predecessor finishes; the outlier count
- * never leaves the device, so the call does not synchronise.  Grows the workspace when M exceeds
- * every earlier M (stream-ordered allocation).
+ * M == 0 is a no-op.  Two or three kernels run on `stream`: the activation
+ * pass (outlier detection, row quantisation and the outlier gather) and the
+ * fused int8 GEMM, a programmatic dependent launch that starts while the
+ * activation pass finishes.  The activation pass is one kernel when X fits
+ * in the GPU's shared memory (rows split evenly over one block per SM, K <=
+ * 32768) or M <= 64, else two (detection, then quantisation); see
+ * int8mm_launches_per_forward.  The outlier count never leaves the device,
+ * so the call does not synchronise.  Grows the workspace when M exceeds every
+ * earlier M (stream-ordered allocation).
  */
 int8mm_status int8mm_forward(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
                              void* Y_fp16_dev, void* stream);
@@ -116,10 +120,10 @@ int8mm_status int8mm_forward_host(int8mm_weight_t h, const void* X_fp16_host, in
 /*
  * Same as int8mm_forward, and records three caller-created CUDA events
  * (cudaEvent_t, passed as void*; NULL entries are skipped) on `stream`:
- * before the activation passes, between them and the GEMM, and after the
+ * before the activation pass, between it and the GEMM, and after the
  * GEMM, so that the GEMM can be timed on the stream it runs on.  A middle
  * event makes the GEMM an ordinary launch instead of a programmatic
- * dependent of the row pass (its prologue then no longer overlaps that pass).
+ * dependent of the activation pass (its prologue then no longer overlaps it).
  */
 int8mm_status int8mm_forward_events(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
                                     void* Y_fp16_dev, void* stream, void* const events[3]);
@@ -159,6 +163,10 @@ int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns);
 
 /* Device bytes held by the handle (codes, scales, workspace). */
 int8mm_status int8mm_weight_bytes(int8mm_weight_t h, size_t* bytes);
+
+/* Number of kernels a forward of M rows launches with this handle (0 for
+ * M == 0, else 2 or 3).  Host-side only; nothing is enqueued. */
+int8mm_status int8mm_launches_per_forward(int8mm_weight_t h, int64_t M, int* count);
 
 /*
  * Outlier-column detection (step 1 above) that allocates no device memory.

@@ -44,6 +44,7 @@ SIGNATURES = {
     "int8mm_get_status": (_ST, [_P]),
     "int8mm_set_wait_limit": (_ST, [_P, ctypes.c_uint64]),
     "int8mm_weight_bytes": (_ST, [_P, ctypes.POINTER(ctypes.c_size_t)]),
+    "int8mm_launches_per_forward": (_ST, [_P, _I64, ctypes.POINTER(ctypes.c_int)]),
     "int8mm_free": (None, [_P]),
     "int8mm_last_error": (ctypes.c_char_p, []),
     "int8mm_outlier_columns_noalloc": (_ST, [_P, _I64, _I64, ctypes.c_float, _P, _P, _P, _P]),
@@ -234,6 +235,12 @@ def int8mm_set_wait_limit(w: Weight, timeout_ns: int) -> None:
 def int8mm_weight_bytes(w: Weight) -> int:
     n = ctypes.c_size_t()
     _check(lib().int8mm_weight_bytes(w.handle, ctypes.byref(n)))
+    return int(n.value)
+
+
+def int8mm_launches_per_forward(w: Weight, M: int) -> int:
+    n = ctypes.c_int()
+    _check(lib().int8mm_launches_per_forward(w.handle, int(M), ctypes.byref(n)))
     return int(n.value)
 
 

@@ -40,6 +40,10 @@ struct int8mm_weight {
   unsigned* ticket = nullptr;            // [1]
   uint32_t* mask = nullptr;
   int32_t* pre = nullptr;
+  // single-launch activation pass: two bitmasks (by generation parity) and
+  // the grid barrier's arrival counter and generation
+  uint32_t* omask = nullptr;  // [2][ceil(K/32)]
+  uint32_t* xsync = nullptr;  // [4]: arrivals by generation parity, generation
   int32_t* idx = nullptr;
   int32_t* count = nullptr;
   float* colmax = nullptr;
@@ -159,6 +163,8 @@ void free_all(int8mm_weight* h) {
   release(&h->ticket);
   release(&h->mask);
   release(&h->pre);
+  release(&h->omask);
+  release(&h->xsync);
   release(&h->idx);
   release(&h->count);
   release(&h->colmax);
@@ -265,6 +271,27 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     SmallActArgs sa{Xh, static_cast<int>(M), static_cast<int>(h->K), alpha, h->Xq, h->c_x, h->X_OT,
                     h->colmax, h->idx, h->count};
     if ((e = launch_small_act(sa, s)) != cudaSuccess) return cuda_fail(e, "activation pass launch");
+  } else if (!decode && row_act_fits(M, h->K, h->num_sms)) {
+    RowActArgs ra;
+    ra.X = Xh;
+    ra.M = static_cast<int>(M);
+    ra.K = static_cast<int>(h->K);
+    ra.rows_per_block = 0;
+    ra.col_threads = 0;
+    ra.thr = half_magnitude_threshold(alpha);
+    ra.Xq = h->Xq;
+    ra.c_x = h->c_x;
+    ra.X_OT = h->X_OT;
+    ra.idx = h->idx;
+    ra.count = h->count;
+    ra.omask = h->omask;
+    ra.sync = h->xsync;
+    ra.epoch = h->epoch;
+    ra.colkey = dbg ? h->colkey : nullptr;  // column maxima only for the debug dump
+    ra.colmax = h->colmax;
+    ra.status = h->status;
+    ra.timeout_ns = h->timeout_ns;
+    if ((e = launch_row_act(ra, h->num_sms, s)) != cudaSuccess) return cuda_fail(e, "activation pass launch");
   } else {
     if ((e = launch_outlier_detect(Xh, M, h->K, alpha, sc, s)) != cudaSuccess)
       return cuda_fail(e, "outlier detection launch");
@@ -382,7 +409,8 @@ int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N
       (e = alloc(&h->inv_cw, Nz, s, tot)) != cudaSuccess || (e = alloc(&h->colmax_bits, Nz, s, tot)) != cudaSuccess ||
       (e = alloc(&h->colkey, Kz, s, tot)) != cudaSuccess || (e = alloc(&h->epoch, 1, s, tot)) != cudaSuccess ||
       (e = alloc(&h->ticket, 1, s, tot)) != cudaSuccess || (e = alloc(&h->mask, words, s, tot)) != cudaSuccess ||
-      (e = alloc(&h->pre, words, s, tot)) != cudaSuccess || (e = alloc(&h->idx, Kz, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->pre, words, s, tot)) != cudaSuccess || (e = alloc(&h->omask, 2 * words, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->xsync, 4, s, tot)) != cudaSuccess || (e = alloc(&h->idx, Kz, s, tot)) != cudaSuccess ||
       (e = alloc(&h->count, 1, s, tot)) != cudaSuccess || (e = alloc(&h->colmax, Kz, s, tot)) != cudaSuccess ||
       (e = alloc(&h->status, 1, s, tot)) != cudaSuccess) {
     cudaStreamSynchronize(s);
@@ -395,6 +423,8 @@ int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N
       (e = cudaMemsetAsync(h->epoch, 0, 8, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->ticket, 0, 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->mask, 0, words * 4, s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(h->omask, 0, 2 * words * 4, s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(h->xsync, 0, 16, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->count, 0, 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->status, 0, 4, s)) != cudaSuccess ||
       (e = launch_weight_prep(h->W, K, N, h->colmax_bits, h->Wb, h->N_pad, h->c_w, h->inv_cw, h->num_sms, s)) !=
@@ -494,9 +524,12 @@ int8mm_status int8mm_get_status(int8mm_weight_t h) {
   if ((e = cudaMemset(h->status, 0, 4)) != cudaSuccess) return cuda_fail(e, "status reset");
   if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "device synchronise");
   if (word & kStatusTimeout) {
-    // an aborted decode GEMM may leave partial sums and tickets behind
+    // an aborted decode GEMM may leave partial sums and tickets behind,
     if (h->part) cudaMemset(h->part, 0, static_cast<size_t>(kDecodeMaxM) * h->N * 4);
     if (h->dticket) cudaMemset(h->dticket, 0, static_cast<size_t>((h->N + 127) / 128) * 4);
+    // and an aborted single-launch activation pass its barrier counts and bitmasks
+    cudaMemset(h->xsync, 0, 16);
+    cudaMemset(h->omask, 0, static_cast<size_t>((h->K + 31) / 32) * 8);
     cudaDeviceSynchronize();
     return fail(INT8MM_ERR_TIMEOUT, "a device wait ran out of time");
   }
@@ -513,6 +546,15 @@ int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns) {
 int8mm_status int8mm_weight_bytes(int8mm_weight_t h, size_t* bytes) {
   if (!live(h) || bytes == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "invalid handle or NULL output");
   *bytes = h->bytes;
+  return INT8MM_OK;
+}
+
+int8mm_status int8mm_launches_per_forward(int8mm_weight_t h, int64_t M, int* count) {
+  if (!live(h) || count == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "invalid handle or NULL output");
+  if (M < 0) return fail(INT8MM_ERR_INVALID_ARG, "M=%lld is negative", (long long)M);
+  if (M == 0) *count = 0;
+  else if (M <= kDecodeMaxM) *count = small_act_fits(M, h->K) ? 2 : 3;
+  else *count = row_act_fits(M, h->K, h->num_sms) ? 2 : 3;
   return INT8MM_OK;
 }
 

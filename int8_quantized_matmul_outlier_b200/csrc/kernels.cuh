@@ -110,6 +110,39 @@ constexpr size_t kSmallActSmemMax = 200 * 1024;
 bool small_act_fits(int64_t M, int64_t K);
 cudaError_t launch_small_act(const SmallActArgs& a, cudaStream_t stream);
 
+// ---- activation pass in one launch (rows held in shared memory) -----------
+// Detection, quantisation and the outlier gather for an X whose rows, split
+// into equal runs across one block per SM, fit in shared memory
+// (csrc/xact_rows.cu).  A cooperative launch with one grid barrier; writes
+// idx, count, Xq, c_x and X_OT (and colmax when colkey is given).
+struct RowActArgs {
+  const __half* X;     // [M, K]
+  int M, K;
+  int rows_per_block;  // set by the launcher
+  int col_threads;     // set by the launcher: threads per row group
+  int thr;             // half_magnitude_threshold(alpha)
+  int8_t* Xq;          // [M, K]
+  float* c_x;          // [M]
+  __half* X_OT;        // [|O|][M]
+  int32_t* idx;        // [K]
+  int32_t* count;      // [1]
+  uint32_t* omask;     // [2][ceil(K/32)] bitmasks; the one of the current generation is zero
+  uint32_t* sync;      // [3] arrivals for generation parity 0 and 1, generation
+  unsigned long long* epoch;   // epoch of the colkey tags, advanced by every launch
+  unsigned long long* colkey;  // [K] or nullptr; with it, colmax is written too
+  float* colmax;               // [K]
+  int* status;
+  unsigned long long timeout_ns;
+};
+constexpr int64_t kRowActMaxK = 32768;
+constexpr int64_t kRowActMaxRows = 256;
+constexpr size_t kRowActSmemMax = 220 * 1024;
+// Largest binary16 magnitude pattern (0 .. 0x7c00) whose value is <= alpha,
+// or -1 when alpha < 0: |x| > alpha exactly when |x|'s bits exceed it.
+int half_magnitude_threshold(float alpha);
+bool row_act_fits(int64_t M, int64_t K, int num_sms);
+cudaError_t launch_row_act(const RowActArgs& a, int num_sms, cudaStream_t stream);
+
 // ---- decode-shape GEMM (M <= 64 tokens) -----------------------------------
 struct DecodeArgs {
   int M, N, K;

@@ -12,80 +12,15 @@
 // fp16); "LLM.int8()" (brain.gartu.xyz), "Seuil de détection α"; the Fig. 2
 // caption of the AI 十大核心论文解读 article (split, then scale).
 //
-// All loads of X and W are 16-byte vectors; |x| is handled as the binary16
-// magnitude bits (h & 0x7fff), whose unsigned order equals the order of |x|,
-// so maxima are exact and two lanes are compared per instruction (vmax2).
+// All loads of X and W are 16-byte vectors; maxima are taken on the binary16
+// magnitude bits (actq.cuh).
+#include "actq.cuh"
 #include "kernels.cuh"
 
 #include <algorithm>
 
 namespace i8mm {
 namespace {
-
-__device__ __forceinline__ int8_t quant_rne(float x, float c) {
-  // fp32 product rounded once, then round-to-nearest-even, clamped to +-127.
-  int q = __float2int_rn(__fmul_rn(x, c));
-  q = max(-127, min(127, q));
-  return static_cast<int8_t>(q);
-}
-
-__device__ __forceinline__ float scale_from_absmax_bits(uint32_t bits) {
-  const float a = __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
-  return a == 0.0f ? 0.0f : __fdiv_rn(127.0f, a);
-}
-
-__device__ __forceinline__ uint32_t max_pair(uint32_t m) { return max(m & 0xffffu, m >> 16); }
-
-// rne(x * c) as int8 in the low byte.  |x| <= absmax and c = 127/absmax
-// bound |x * c| by 127 (1 + 2^-24), which rounds to at most 127, so the
-// saturating conversion equals the clamp to [-127, 127] exactly.
-__device__ __forceinline__ uint32_t q8(float x, float c) {
-  int32_t q;
-  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(q) : "f"(__fmul_rn(x, c)));
-  return static_cast<uint32_t>(q);
-}
-
-// Eight halves -> eight int8 codes, as two little-endian words.
-__device__ __forceinline__ uint2 quant8(const uint4& v, float c) {
-  const __half2* h = reinterpret_cast<const __half2*>(&v);
-  const float2 f0 = __half22float2(h[0]), f1 = __half22float2(h[1]);
-  const float2 f2 = __half22float2(h[2]), f3 = __half22float2(h[3]);
-  const uint32_t a01 = __byte_perm(q8(f0.x, c), q8(f0.y, c), 0x0040);
-  const uint32_t a23 = __byte_perm(q8(f1.x, c), q8(f1.y, c), 0x0040);
-  const uint32_t b01 = __byte_perm(q8(f2.x, c), q8(f2.y, c), 0x0040);
-  const uint32_t b23 = __byte_perm(q8(f3.x, c), q8(f3.y, c), 0x0040);
-  return make_uint2(__byte_perm(a01, a23, 0x5410), __byte_perm(b01, b23, 0x5410));
-}
-
-// Bits 0..3 of n -> 0xff in bytes 0..3 of the result.
-__device__ __forceinline__ uint32_t expand_nibble(uint32_t n) {
-  return ((n * 0x00204081u) & 0x01010101u) * 0xffu;
-}
-
-// Max of the magnitudes of the halves of v whose flag bit is clear.
-__device__ __forceinline__ uint32_t masked_absmax2(uint32_t m, const uint4& v, uint32_t fl) {
-  if (fl == 0) {
-    m = __vmaxu2(m, v.x & 0x7fff7fffu);
-    m = __vmaxu2(m, v.y & 0x7fff7fffu);
-    m = __vmaxu2(m, v.z & 0x7fff7fffu);
-    return __vmaxu2(m, v.w & 0x7fff7fffu);
-  }
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const uint32_t keep = (((fl >> (2 * p)) & 1u) ? 0u : 0x0000ffffu) | (((fl >> (2 * p + 1)) & 1u) ? 0u : 0xffff0000u);
-    m = __vmaxu2(m, w[p] & 0x7fff7fffu & keep);
-  }
-  return m;
-}
-
-// Programmatic dependent launch: let the next kernel of the stream start its
-// prologue, and wait until the previous kernel's results are visible.  Both
-// are no-ops for a kernel launched without the programmatic attribute.
-__device__ __forceinline__ void pdl_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ------------------------------------------------------------------------
 // Weight prep, step 1: column absmax of W[K,N] into colmax_bits[N] (atomicMax

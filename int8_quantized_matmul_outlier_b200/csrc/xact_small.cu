@@ -23,6 +23,7 @@
 //   3. the codes and the outlier entries of the slice;    cluster barrier
 // The forward uses this kernel while the slice fits (M <= 64 and
 // M * K/16 * 2 bytes within kSmallActSmemMax).
+#include "actq.cuh"
 #include "kernels.cuh"
 
 #include <cooperative_groups.h>
@@ -33,43 +34,6 @@ namespace i8mm {
 namespace {
 
 constexpr int NT = 256;
-
-__device__ __forceinline__ uint32_t q8(float x, float c) {
-  int32_t q;
-  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(q) : "f"(__fmul_rn(x, c)));
-  return static_cast<uint32_t>(q);
-}
-
-__device__ __forceinline__ uint2 quant8(const uint4& v, float c) {
-  const __half2* h = reinterpret_cast<const __half2*>(&v);
-  const float2 f0 = __half22float2(h[0]), f1 = __half22float2(h[1]);
-  const float2 f2 = __half22float2(h[2]), f3 = __half22float2(h[3]);
-  const uint32_t a01 = __byte_perm(q8(f0.x, c), q8(f0.y, c), 0x0040);
-  const uint32_t a23 = __byte_perm(q8(f1.x, c), q8(f1.y, c), 0x0040);
-  const uint32_t b01 = __byte_perm(q8(f2.x, c), q8(f2.y, c), 0x0040);
-  const uint32_t b23 = __byte_perm(q8(f3.x, c), q8(f3.y, c), 0x0040);
-  return make_uint2(__byte_perm(a01, a23, 0x5410), __byte_perm(b01, b23, 0x5410));
-}
-
-__device__ __forceinline__ uint32_t expand_nibble(uint32_t n) {
-  return ((n * 0x00204081u) & 0x01010101u) * 0xffu;
-}
-
-__device__ __forceinline__ uint32_t masked_absmax2(uint32_t m, const uint4& v, uint32_t fl) {
-  if (fl == 0) {
-    m = __vmaxu2(m, v.x & 0x7fff7fffu);
-    m = __vmaxu2(m, v.y & 0x7fff7fffu);
-    m = __vmaxu2(m, v.z & 0x7fff7fffu);
-    return __vmaxu2(m, v.w & 0x7fff7fffu);
-  }
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const uint32_t keep = (((fl >> (2 * p)) & 1u) ? 0u : 0x0000ffffu) | (((fl >> (2 * p + 1)) & 1u) ? 0u : 0xffff0000u);
-    m = __vmaxu2(m, w[p] & 0x7fff7fffu & keep);
-  }
-  return m;
-}
 
 __global__ void __launch_bounds__(NT) xact_small_kernel(SmallActArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
@@ -85,7 +49,7 @@ __global__ void __launch_bounds__(NT) xact_small_kernel(SmallActArgs a) {
   const int nw = (nv + 3) / 4;  // mask words of this slice
 
   // the decode GEMM may start its prologue and weight prefetch right away
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_launch_dependents();
 
   extern __shared__ uint4 dsm[];
   uint4* xs = dsm;                                               // [M][vpb] the slice of X
@@ -218,8 +182,7 @@ __global__ void __launch_bounds__(NT) xact_small_kernel(SmallActArgs a) {
   for (int r = warp; r < M; r += NT / 32) {
     uint32_t m = lane < CL ? *cluster.map_shared_rank(&s_rowmax[r], lane) : 0u;
     m = __reduce_max_sync(0xffffffffu, m);
-    const float am = __half2float(__ushort_as_half(static_cast<unsigned short>(m)));
-    const float c = am == 0.0f ? 0.0f : __fdiv_rn(127.0f, am);
+    const float c = scale_from_absmax_bits(m);
     if (lane == 0) {
       s_c[r] = c;
       if (rank == 0) a.c_x[r] = c;

@@ -85,6 +85,11 @@ SHAPES = [
     (65, 1040, 784, 3, 6.0),        # smallest prefill-kernel M
     (40, 2048, 4112, 5, 6.0),       # decode kernel, stream-K splits across blocks
     (8, 12288, 1024, 7, 6.0),       # decode, long K: whole and split blocks
+    (96, 512, 256, 6, 0.0),         # alpha = 0 on the single-launch activation pass
+    (100, 256, 128, 0, -1.0),       # alpha < 0: every column is an outlier
+    (300, 16, 32, 1, 6.0),          # smallest K, three rows per block
+    (149, 32768, 256, 3, 6.0),      # largest K of the single-launch pass, one row per block
+    (3000, 5120, 256, 7, 6.0),      # 21 rows (210 KB) of X per block
 ]
 
 
@@ -104,6 +109,27 @@ def test_threshold_ties_on_gpu():
     p.X[5, 3] = 6.0
     p.X[9, 10] = -6.0
     p.X[11, 20] = np.float16(6.00390625)
+    p.X[0, 63] = -100
+    out = check(p)
+    assert out["cnt"] == 2
+
+
+@pytest.mark.parametrize("alpha", [6.001, 5.9999, 1e-7, 3e-5, 65504.0, 70000.0])
+def test_thresholds_between_fp16_values(alpha):
+    # alpha need not be an fp16 value: |x| > alpha is decided in fp32 on both sides
+    p = workloads.small(100, 256, 64, 3, seed=31, alpha=alpha)
+    p.X[7, 5] = np.float16(6.0)
+    p.X[8, 6] = np.float16(6.00390625)
+    p.X[9, 7] = np.float16(2.98e-5)
+    p.X[10, 8] = np.float16(65504.0)
+    check(p)
+
+
+def test_threshold_ties_single_launch_pass():
+    p = workloads.small(100, 64, 32, 0, seed=4)
+    p.X[5, 3] = 6.0
+    p.X[90, 10] = -6.0
+    p.X[99, 20] = np.float16(6.00390625)
     p.X[0, 63] = -100
     out = check(p)
     assert out["cnt"] == 2
@@ -132,6 +158,51 @@ def test_repeat_and_stale_state():
     c = check(p1, w=w, wq=wq)
     assert (a["cnt"], b["cnt"], c["cnt"]) == (6, 0, 6)
     assert torch.equal(a["d"]["Y"], c["d"]["Y"])
+
+
+def test_activation_paths_alternate_on_one_handle():
+    # the single-launch pass (rows in shared memory) and the two-pass kernels
+    # share the handle's epoch; outlier sets must not leak between them
+    K, N = 5120, 512
+    W = workloads.weight(K, N, 41)
+    w = m.int8mm_prepare_weight(torch.from_numpy(W).to(dev()))
+    wq = oracle.quantize_cols(W)
+    runs = [(2048, 7), (2048, 0), (4096, 3), (2048, 5), (4096, 0), (3000, 2), (2048, 7), (2048, 1)]
+    counts = []
+    for i, (M, n_out) in enumerate(runs):
+        p = workloads.small(M, K, N, n_out, seed=400 + i)
+        p.W = W
+        out = check(p, w=w, wq=wq, rows=sample_rows(M, 16, seed=i), check_w_codes=False)
+        counts.append(out["cnt"])
+    assert counts == [n for _, n in runs]
+
+
+def test_launches_per_forward():
+    W = torch.from_numpy(workloads.weight(5120, 256, 43)).to(dev())
+    w = m.int8mm_prepare_weight(W)
+    assert m.int8mm_launches_per_forward(w, 0) == 0
+    assert m.int8mm_launches_per_forward(w, 1) == 2       # single-cluster activation pass + decode GEMM
+    assert m.int8mm_launches_per_forward(w, 2048) == 2    # rows fit in shared memory
+    assert m.int8mm_launches_per_forward(w, 4096) == 3    # two activation kernels
+    with pytest.raises(m.Int8mmError):
+        m.int8mm_launches_per_forward(w, -1)
+
+
+def test_single_launch_pass_many_generations():
+    # the product forward (no column maxima) over many launches with changing
+    # outlier sets, against the debug forward of the same inputs
+    K, N = 1024, 256
+    W = workloads.weight(K, N, 42)
+    w = m.int8mm_prepare_weight(torch.from_numpy(W).to(dev()))
+    for i in range(9):
+        p = workloads.small(200, K, N, i % 4, seed=500 + i)
+        X = torch.from_numpy(p.X).to(dev())
+        y = m.int8mm_forward(w, X, 6.0)
+        d = m.int8mm_forward_debug(w, X, 6.0)
+        torch.cuda.synchronize()
+        assert int(d["outlier_count"].item()) == i % 4
+        assert torch.equal(y, d["Y"])
+    assert m.int8mm_get_status(w) == m.INT8MM_OK
 
 
 @pytest.mark.parametrize("M", [1, 16, 40])
