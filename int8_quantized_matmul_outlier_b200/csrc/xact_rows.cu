@@ -243,22 +243,32 @@ __global__ void __launch_bounds__(kMaxThreads, 1) xact_rows_kernel(RowActArgs a)
       slot[i] = pre_s[w] + __popc(mask_s[w] & ((1u << sh) - 1u));
     }
   }
-  // row maxima over the non-outlier columns (vectors past K have keep = 0)
-  for (int j = g; j < nr; j += RG) {
-    const uint4* row = xs + static_cast<size_t>(j) * nvec;
-    uint32_t m = 0;
+  // row maxima over the non-outlier columns (vectors past K have keep = 0),
+  // four rows at a time so that their loads and reductions overlap
+  for (int k0 = 0; g + RG * k0 < nr; k0 += 4) {
+    uint32_t m[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      const int v = min(t + i * CT, nvec - 1);
-      const uint4 x = row[v];
-      // the byte masks widened to 16-bit lanes, with the sign bits cleared
-      m = __vmaxu2(m, x.x & __byte_perm(keep[i][0], 0u, 0x1100) & 0x7fff7fffu);
-      m = __vmaxu2(m, x.y & __byte_perm(keep[i][0], 0u, 0x3322) & 0x7fff7fffu);
-      m = __vmaxu2(m, x.z & __byte_perm(keep[i][1], 0u, 0x1100) & 0x7fff7fffu);
-      m = __vmaxu2(m, x.w & __byte_perm(keep[i][1], 0u, 0x3322) & 0x7fff7fffu);
+    for (int u = 0; u < 4; ++u) {
+      const int j = g + RG * (k0 + u);
+      if (j < nr) {
+        const uint4* row = xs + static_cast<size_t>(j) * nvec;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+          const uint4 x = row[min(t + i * CT, nvec - 1)];
+          // the byte masks widened to 16-bit lanes, with the sign bits cleared
+          m[u] = __vmaxu2(m[u], x.x & __byte_perm(keep[i][0], 0u, 0x1100) & 0x7fff7fffu);
+          m[u] = __vmaxu2(m[u], x.y & __byte_perm(keep[i][0], 0u, 0x3322) & 0x7fff7fffu);
+          m[u] = __vmaxu2(m[u], x.z & __byte_perm(keep[i][1], 0u, 0x1100) & 0x7fff7fffu);
+          m[u] = __vmaxu2(m[u], x.w & __byte_perm(keep[i][1], 0u, 0x3322) & 0x7fff7fffu);
+        }
+      }
     }
-    m = __reduce_max_sync(0xffffffffu, max_pair(m));
-    if (lane == 0) atomicMax(&rowmax_s[j], m);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = g + RG * (k0 + u);  // the same for the whole warp
+      const uint32_t r = __reduce_max_sync(0xffffffffu, max_pair(m[u]));
+      if (lane == 0 && j < nr) atomicMax(&rowmax_s[j], r);
+    }
   }
   __syncthreads();
   if (tid < nr) {
