@@ -20,12 +20,19 @@
 //   warps 2-9   epilogue, two warps per TMEM lane quarter (warp w reads lanes
 //               32*(w%4)..+31, one output row per thread), each covering one
 //               128-column half of the tile: tcgen05.ld of the accumulator,
-//               scale by 1/c_x and 1/c_w, add the |O| outlier FMAs, write fp16.
-//               While the tile still accumulates, the four warps of a half
-//               stage 1/c_w and the outlier weight rows W[O, half] in shared
-//               memory and load their rows' outlier activations.
+//               scale by 1/c_x and 1/c_w, add the fp16 outlier product, write
+//               fp16.
 // The epilogue of tile t overlaps the main loop of tile t+1.  Every wait is
 // bounded; a timeout sets the status word and the CTA drains and exits.
+//
+// The outlier product X[:,O] W[O,:] (CTA pairs, the first kOutMma outliers)
+// runs on the tensor cores too: the epilogue writes the dequantised tile
+// back into TMEM as fp32, the MMA warp adds X_O W_O^T onto it with
+// tcgen05.mma.kind::f16 (X_O [M][64] and W_O [N][64] fp16, prepared by the
+// activation pass, loaded by TMA like the int8 operands), and the epilogue
+// reads the sums.  The MMA warp issues that product between the int8 k-blocks
+// of the next tile.  Single CTAs (M <= 128) and outliers past kOutMma use
+// CUDA-core FMAs in the epilogue (W rows staged in shared memory).
 //
 // Two modes.  Single CTA (M <= 128): 128x256 tiles, B tiles of 256 rows,
 // 4 stages.  CTA pair (M > 128): a cluster of two CTAs on neighbouring SMs
@@ -67,11 +74,19 @@ struct Cfg {
   static constexpr int STAGES = PAIR ? 6 : 4;
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;  // rows per tile
   static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 5;  // full, empty, tmem_full[2], tmem_empty[2], drain
+  // full, empty, tmem_full[2], tmem_empty[2], drain, and for the outlier
+  // product: operands loaded, operands free, tile dequantised[2], product done[2]
+  static constexpr int NUM_BARS = 2 * STAGES + 5 + 6;
   static constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
-  static constexpr int WO_OFFSET = (MISC_OFFSET + 16 + 15) & ~15;
-  static constexpr int RW_OFFSET = WO_OFFSET + WO_BYTES;
+  // pairs: the outlier product's operand tiles (128 rows of 128 bytes each:
+  // 64 fp16 outliers of 128 rows of X_O, and of 128 rows of W_O); single CTAs:
+  // the staged outlier weight rows
+  static constexpr int OA_OFFSET = (MISC_OFFSET + 16 + 1023) & ~1023;
+  static constexpr int OB_OFFSET = OA_OFFSET + (PAIR ? A_BYTES : 0);
+  static constexpr int WO_OFFSET = OB_OFFSET + (PAIR ? A_BYTES : 0);
+  static constexpr int RW_OFFSET = WO_OFFSET + (PAIR ? 0 : WO_BYTES);
   static constexpr int SMEM_BYTES = RW_OFFSET + RW_BYTES + 1024;  // + slack to align the base to 1024
+  static constexpr uint32_t IDESC_F16 = idesc_f16_f32(TILE_M, BN);
   static constexpr uint32_t IDESC = idesc_i8(TILE_M, BN);
   static_assert(SMEM_BYTES <= 232448, "fits the 227 KB of shared memory per block");
   static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-byte aligned for the 128B swizzle");
@@ -97,6 +112,7 @@ __device__ __forceinline__ float dequant(uint32_t acc, float rx, float rw) {
 template <bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_decomp_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmXO, const __grid_constant__ CUtensorMap tmWO,
                           const GemmArgs a) {
   using C = Cfg<PAIR>;
   constexpr int STAGES = C::STAGES;
@@ -108,6 +124,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
+  uint64_t* ofull = drain + 1;   // outlier operand tiles landed (leader)
+  uint64_t* oempty = ofull + 1;  // outlier operand tiles read by the product
+  uint64_t* tdeq = oempty + 1;   // [2] tile dequantised into TMEM (leader)
+  uint64_t* tout = tdeq + 2;     // [2] outlier product added
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFFSET);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFFSET + 4);
 
@@ -132,10 +152,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&tempty[b], NUM_EPI_WARPS * (PAIR ? 2 : 1));
     }
     mbar_init(drain, 1);
+    mbar_init(ofull, 1);
+    mbar_init(oempty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tdeq[b], NUM_EPI_WARPS * (PAIR ? 2 : 1));
+      mbar_init(&tout[b], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (PAIR) {
+      tma_prefetch_desc(&tmXO);
+      tma_prefetch_desc(&tmWO);
+    }
   }
   if (warp == 1) {
     if (PAIR) {
@@ -192,8 +222,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       stage = pre % STAGES;
       phase = pre == STAGES ? 1u : 0u;
+      // Operand tiles of the outlier product of a tile (pairs with |O| > 0):
+      // loaded at the start of the next tile, once the previous product has
+      // read the single buffer.
+      const bool outl = PAIR && *a.count > 0;
+      uint32_t ouse = 0;
+      auto load_outl = [&](int tile) -> bool {
+        if (!mbar_wait(oempty, (ouse & 1u) ^ 1u, tmo, abort_flag)) return false;
+        if (rank == 0) mbar_arrive_expect_tx(ofull, 4 * A_BYTES);  // two CTAs x (X_O + W_O tiles)
+        const uint32_t ob = mapa_shared(smem_u32(ofull), 0);
+        tma_load_2d_pair(smem + C::OA_OFFSET, &tmXO, ob, 0, (tile % num_m) * C::TILE_M + static_cast<int>(rank) * BM);
+        tma_load_2d_pair(smem + C::OB_OFFSET, &tmWO, ob, 0, (tile / num_m) * BN + static_cast<int>(rank) * C::B_ROWS);
+        ++ouse;
+        return true;
+      };
+      int prev = -1;
       for (int tile = tile0; tile < num_tiles && ok; tile += tstride) {
         const int m_blk = tile % num_m, n_blk = tile / num_m;
+        if (outl && prev >= 0 && !load_outl(prev)) {
+          ok = false;
+          break;
+        }
+        prev = tile;
         for (int kb = tile == first ? pre : 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
             ok = false;
@@ -210,6 +260,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      if (ok && outl && prev >= 0 && !load_outl(prev)) ok = false;
       if (!ok) {
         fail(a, abort_flag);
         // Let every load already issued land before the CTA can exit (a
@@ -217,6 +268,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!PAIR || rank == 0) {
           for (int s = 0; s < STAGES; ++s)
             if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, tmo, nullptr);
+          if (ouse > 0) mbar_wait(ofull, (ouse - 1u) & 1u, tmo, nullptr);
         } else {
           const uint64_t t0 = global_timer_ns();
           while (global_timer_ns() - t0 < 200000ull) {
@@ -231,6 +283,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       int lt = 0;
+      // Outlier product of a finished tile (pairs with |O| > 0): once the
+      // epilogue has written the dequantised tile back to TMEM and the
+      // operand tiles have landed, D += X_O W_O^T in min(|O|, 64)/16 steps of
+      // K = 16, issued between the int8 k-blocks of the next tile.
+      pdl_wait();
+      const int cnt = PAIR ? *a.count : 0;
+      const int nk = cnt > 0 ? (min(cnt, kOutMma) + 15) / 16 : 0;
+      uint32_t ouse = 0, pend_use = 0;
+      int pend = -1;  // accumulator buffer whose outlier product is due
+      auto issue_outl = [&](bool block) -> bool {
+        if (block) {
+          if (!mbar_wait(&tdeq[pend], pend_use & 1u, tmo, abort_flag) || !mbar_wait(ofull, ouse & 1u, tmo, abort_flag))
+            return false;
+        } else if (!mbar_test_wait(&tdeq[pend], pend_use & 1u) || !mbar_test_wait(ofull, ouse & 1u)) {
+          return true;  // not yet
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(pend * BN);
+        const uint64_t adesc = smem_desc_k_sw128(smem_u32(smem + C::OA_OFFSET));
+        const uint64_t bdesc = smem_desc_k_sw128(smem_u32(smem + C::OB_OFFSET));
+        for (int kk = 0; kk < nk; ++kk)  // 32 bytes (16 fp16) along K per step
+          mma_f16_pair(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2),
+                       C::IDESC_F16, 1u);
+        mma_commit_pair(oempty, 0x3);
+        mma_commit_pair(&tout[pend], 0x3);
+        ++ouse;
+        pend = -1;
+        return true;
+      };
       for (int tile = tile0; tile < num_tiles && ok; tile += tstride, ++lt) {
         const int buf = lt & 1;
         const uint32_t use = static_cast<uint32_t>(lt >> 1);
@@ -266,12 +347,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             stage = 0;
             phase ^= 1u;
           }
+          if (pend >= 0) issue_outl(false);
         }
         if (ok) {
           if (PAIR) mma_commit_pair(&tfull[buf], 0x3);
           else mma_commit(&tfull[buf]);
         }
+        if (ok && pend >= 0 && !issue_outl(true)) ok = false;
+        if (nk > 0) {
+          pend = buf;
+          pend_use = use;
+        }
       }
+      if (ok && pend >= 0 && !issue_outl(true)) ok = false;
       if (!ok) {
         fail(a, abort_flag);
         if (PAIR) mma_commit_pair(drain, 0x1);
@@ -288,7 +376,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row_t = q * 32 + lane;
     pdl_wait();  // count, idx, X_OT and c_x come from the activation pass
     const int cnt = *a.count;
-    const int cs = min(cnt, OUT_CAP);         // outliers staged in shared memory
+    // pairs: the first kOutMma outliers are added on the tensor cores; single
+    // CTAs: the first OUT_CAP outliers from staged weight rows; both: any
+    // further outliers from global memory
+    const bool outl = PAIR && cnt > 0;
+    const int cs = PAIR ? 0 : min(cnt, OUT_CAP);  // outliers staged in shared memory
+    const int o_tail = PAIR ? kOutMma : OUT_CAP;
     float* wo = reinterpret_cast<float*>(smem + C::WO_OFFSET) + h * OUT_CAP * HALF_N;  // [OUT_CAP][HALF_N]
     float* rws = reinterpret_cast<float*>(smem + C::RW_OFFSET) + h * HALF_N;           // [HALF_N]
     const uint32_t bar_id = 1 + h;
@@ -345,6 +438,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(buf * BN + h * HALF_N);
+      if (outl) {
+        // (3) dequantise in place (int32 -> fp32 in TMEM), hand the tile to
+        //     the MMA warp for the outlier product, and wait for it
+#pragma unroll 1
+        for (int ch = 0; ch < HALF_N / 32; ++ch) {
+          const int cl = ch * 32;
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(cl), r);
+          tmem_wait_ld();
+          const int n = nh + cl;
+          if (a.acc_dump != nullptr && row_ok && n < N) {
+            uint4* ap = reinterpret_cast<uint4*>(a.acc_dump + static_cast<size_t>(m) * N + n);
+#pragma unroll
+            for (int t4 = 0; t4 < 8; ++t4)
+              if (n + 32 <= N || t4 < 4) ap[t4] = make_uint4(r[4 * t4], r[4 * t4 + 1], r[4 * t4 + 2], r[4 * t4 + 3]);
+          }
+          const float4* rw4 = reinterpret_cast<const float4*>(rws + cl);
+#pragma unroll
+          for (int t4 = 0; t4 < 8; ++t4) {
+            const float4 w = rw4[t4];
+            r[4 * t4 + 0] = __float_as_uint(dequant(r[4 * t4 + 0], rx, w.x));
+            r[4 * t4 + 1] = __float_as_uint(dequant(r[4 * t4 + 1], rx, w.y));
+            r[4 * t4 + 2] = __float_as_uint(dequant(r[4 * t4 + 2], rx, w.z));
+            r[4 * t4 + 3] = __float_as_uint(dequant(r[4 * t4 + 3], rx, w.w));
+          }
+          tmem_st_32x32b_x32(t_row + static_cast<uint32_t>(cl), r);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tdeq[buf]), 0));  // the leader's barrier
+        alive = __all_sync(0xffffffffu, mbar_wait(&tout[buf], use & 1u, tmo, abort_flag));
+        if (!alive) {
+          if (lane == 0) fail(a, abort_flag);
+          continue;
+        }
+        tc_fence_after();
+      }
 #pragma unroll 1
       for (int ch = 0; ch < HALF_N / 32; ++ch) {
         const int cl = ch * 32;
@@ -363,14 +494,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (n >= N) continue;  // warp-uniform
         const bool full32 = n + 32 <= N;
         float v[32];
-        const float4* rw4 = reinterpret_cast<const float4*>(rws + cl);
+        if (outl) {  // already dequantised, outlier product included
 #pragma unroll
-        for (int t4 = 0; t4 < 8; ++t4) {
-          const float4 w = rw4[t4];
-          v[4 * t4 + 0] = dequant(r[4 * t4 + 0], rx, w.x);
-          v[4 * t4 + 1] = dequant(r[4 * t4 + 1], rx, w.y);
-          v[4 * t4 + 2] = dequant(r[4 * t4 + 2], rx, w.z);
-          v[4 * t4 + 3] = dequant(r[4 * t4 + 3], rx, w.w);
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+        } else {
+          const float4* rw4 = reinterpret_cast<const float4*>(rws + cl);
+#pragma unroll
+          for (int t4 = 0; t4 < 8; ++t4) {
+            const float4 w = rw4[t4];
+            v[4 * t4 + 0] = dequant(r[4 * t4 + 0], rx, w.x);
+            v[4 * t4 + 1] = dequant(r[4 * t4 + 1], rx, w.y);
+            v[4 * t4 + 2] = dequant(r[4 * t4 + 2], rx, w.z);
+            v[4 * t4 + 3] = dequant(r[4 * t4 + 3], rx, w.w);
+          }
         }
         // fp16 outlier product X[m, O] . W[O, n..n+31] with fp32 accumulation,
         // in ascending order of O: staged rows first, then any beyond OUT_CAP.
@@ -388,7 +524,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        for (int o = OUT_CAP; o < cnt; ++o) {
+        for (int o = o_tail; o < cnt; ++o) {
           const int j = __ldg(a.idx + o);
           const float x1 = row_ok ? __half2float(a.X_OT[static_cast<size_t>(o) * M + m]) : 0.0f;
           const uint4* wr = reinterpret_cast<const uint4*>(a.W + static_cast<size_t>(j) * N + n);
@@ -425,7 +561,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               yp[3] = out[3];
             }
           }
-          if (a.acc_dump != nullptr) {
+          if (a.acc_dump != nullptr && !outl) {
             uint4* ap = reinterpret_cast<uint4*>(a.acc_dump + static_cast<size_t>(m) * N + n);
 #pragma unroll
             for (int t4 = 0; t4 < 8; ++t4)
@@ -447,8 +583,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 template <bool PAIR>
-cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms, bool pdl,
-                     cudaStream_t stream) {
+cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmXO, const CUtensorMap& tmWO,
+                     const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
   using C = Cfg<PAIR>;
   static unsigned long long attr_set = 0;  // one bit per device
   int dev = 0;
@@ -484,16 +620,17 @@ cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmA
   }
   cfg.attrs = attrs;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, gemm_i8_decomp_kernel<PAIR>, tmA, tmB, a);
+  return cudaLaunchKernelEx(&cfg, gemm_i8_decomp_kernel<PAIR>, tmA, tmB, tmXO, tmWO, a);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB256, const CUtensorMap& tmB128,
-                               const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
+                               const CUtensorMap& tmXO, const CUtensorMap& tmWO, const GemmArgs& a, int num_sms,
+                               bool pdl, cudaStream_t stream) {
   // one 128-row tile height: single CTAs; taller problems: CTA pairs
-  if (a.M <= BM) return launch_t<false>(tmA, tmB256, a, num_sms, pdl, stream);
-  return launch_t<true>(tmA, tmB128, a, num_sms, pdl, stream);
+  if (a.M <= BM) return launch_t<false>(tmA, tmB256, tmXO, tmWO, a, num_sms, pdl, stream);
+  return launch_t<true>(tmA, tmB128, tmXO, tmWO, a, num_sms, pdl, stream);
 }
 
 }  // namespace i8mm
