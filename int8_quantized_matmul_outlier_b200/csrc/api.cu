@@ -31,9 +31,6 @@ struct int8mm_weight {
   uint32_t* colmax_bits = nullptr;  // [N] prep scratch
   CUtensorMap tmB;     // Wb, 256-row boxes (prefill GEMM operand B)
   CUtensorMap tmW128;  // Wb, 128-row boxes (decode GEMM operand A)
-  // operands of the prefill GEMM's tensor-core outlier product
-  __half* w_o = nullptr;  // [N_pad][kOutMma]
-  CUtensorMap tmWO;
   // decode (M <= 64) scratch: int32 partial sums and per-n-block tickets
   int32_t* part = nullptr;
   unsigned* dticket = nullptr;
@@ -56,10 +53,6 @@ struct int8mm_weight {
   int8_t* Xq = nullptr;
   float* c_x = nullptr;
   __half* X_OT = nullptr;
-  __half* x_o = nullptr;  // [rows][kOutMma]
-  CUtensorMap tmXO;       // for the current (x_o, M)
-  const void* tmXO_ptr = nullptr;
-  int64_t tmXO_rows = -1;
   // tensor map of Xq for the current (pointer, M, box rows)
   CUtensorMap tmA;
   const void* tmA_ptr = nullptr;
@@ -150,12 +143,9 @@ void free_workspace(int8mm_weight* h) {
   release(&h->Xq);
   release(&h->c_x);
   release(&h->X_OT);
-  release(&h->x_o);
   h->ws_rows = 0;
   h->tmA_ptr = nullptr;
   h->tmA_rows = -1;
-  h->tmXO_ptr = nullptr;
-  h->tmXO_rows = -1;
 }
 
 void free_all(int8mm_weight* h) {
@@ -165,7 +155,6 @@ void free_all(int8mm_weight* h) {
   release(&h->part);
   release(&h->dticket);
   release(&h->Wb);
-  release(&h->w_o);
   release(&h->c_w);
   release(&h->inv_cw);
   release(&h->colmax_bits);
@@ -185,8 +174,7 @@ void free_all(int8mm_weight* h) {
 size_t ws_bytes(const int8mm_weight* h, int64_t rows) {
   return static_cast<size_t>(rows) * h->K                  // Xq
          + static_cast<size_t>(rows) * 4                   // c_x
-         + static_cast<size_t>(rows) * h->K * 2            // X_OT
-         + static_cast<size_t>(rows) * kOutMma * 2;        // x_o
+         + static_cast<size_t>(rows) * h->K * 2;           // X_OT
 }
 
 int8mm_status ensure_workspace(int8mm_weight* h, int64_t M, cudaStream_t s) {
@@ -199,19 +187,16 @@ int8mm_status ensure_workspace(int8mm_weight* h, int64_t M, cudaStream_t s) {
     cudaFreeAsync(h->Xq, s);
     cudaFreeAsync(h->c_x, s);
     cudaFreeAsync(h->X_OT, s);
-    cudaFreeAsync(h->x_o, s);
     h->bytes -= ws_bytes(h, h->ws_rows);
     h->Xq = nullptr;
     h->c_x = nullptr;
     h->X_OT = nullptr;
-    h->x_o = nullptr;
     h->ws_rows = 0;
   }
   cudaError_t e;
   if ((e = alloc(&h->Xq, static_cast<size_t>(rows) * h->K, s, nullptr)) != cudaSuccess ||
       (e = alloc(&h->c_x, static_cast<size_t>(rows), s, nullptr)) != cudaSuccess ||
-      (e = alloc(&h->X_OT, static_cast<size_t>(rows) * h->K, s, nullptr)) != cudaSuccess ||
-      (e = alloc(&h->x_o, static_cast<size_t>(rows) * kOutMma, s, nullptr)) != cudaSuccess) {
+      (e = alloc(&h->X_OT, static_cast<size_t>(rows) * h->K, s, nullptr)) != cudaSuccess) {
     cudaStreamSynchronize(s);
     free_workspace(h);
     return cuda_fail(e, "workspace allocation");
@@ -220,8 +205,6 @@ int8mm_status ensure_workspace(int8mm_weight* h, int64_t M, cudaStream_t s) {
   h->bytes += ws_bytes(h, rows);
   h->tmA_ptr = nullptr;
   h->tmA_rows = -1;
-  h->tmXO_ptr = nullptr;
-  h->tmXO_rows = -1;
   return INT8MM_OK;
 }
 
@@ -263,11 +246,6 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     h->tmA_ptr = h->Xq;
     h->tmA_rows = M;
     h->tmA_box = box_rows;
-  }
-  if (!decode && (h->tmXO_ptr != h->x_o || h->tmXO_rows != M)) {
-    if ((st = make_tmap_i8(&h->tmXO, h->x_o, kOutMma * 2, M, kOutMma * 2, kGemmBM)) != INT8MM_OK) return st;
-    h->tmXO_ptr = h->x_o;
-    h->tmXO_rows = M;
   }
   if (decode && h->part == nullptr) {
     const size_t nb = static_cast<size_t>((h->N + 127) / 128);
@@ -313,17 +291,11 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     ra.colmax = h->colmax;
     ra.status = h->status;
     ra.timeout_ns = h->timeout_ns;
-    ra.W = h->W;
-    ra.N = static_cast<int>(h->N);
-    ra.N_pad = static_cast<int>(h->N_pad);
-    ra.x_o = h->x_o;
-    ra.w_o = h->w_o;
     if ((e = launch_row_act(ra, h->num_sms, s)) != cudaSuccess) return cuda_fail(e, "activation pass launch");
   } else {
     if ((e = launch_outlier_detect(Xh, M, h->K, alpha, sc, s)) != cudaSuccess)
       return cuda_fail(e, "outlier detection launch");
-    OutlierOperands oo{h->idx, h->count, h->W, static_cast<int>(h->N), static_cast<int>(h->N_pad), h->x_o, h->w_o};
-    if ((e = launch_row_quant(Xh, M, h->K, sc, h->Xq, h->c_x, h->X_OT, oo, /*pdl=*/true, s)) != cudaSuccess)
+    if ((e = launch_row_quant(Xh, M, h->K, sc, h->Xq, h->c_x, h->X_OT, /*pdl=*/true, s)) != cudaSuccess)
       return cuda_fail(e, "row quantisation launch");
   }
   rec(1);
@@ -366,7 +338,7 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     a.acc_dump = dbg ? dbg->acc : nullptr;
     a.status = h->status;
     a.timeout_ns = h->timeout_ns;
-    if ((e = launch_gemm_decomp(h->tmA, h->tmB, h->tmW128, h->tmXO, h->tmWO, a, h->num_sms, pdl, s)) != cudaSuccess)
+    if ((e = launch_gemm_decomp(h->tmA, h->tmB, h->tmW128, a, h->num_sms, pdl, s)) != cudaSuccess)
       return cuda_fail(e, "int8 GEMM launch");
   }
   rec(2);
@@ -435,7 +407,6 @@ int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N
   const size_t wb_bytes = kblocks * static_cast<size_t>(h->N_pad) * 128;
   if ((e = alloc(&h->Wb, wb_bytes, s, tot)) != cudaSuccess || (e = alloc(&h->c_w, Nz, s, tot)) != cudaSuccess ||
       (e = alloc(&h->inv_cw, Nz, s, tot)) != cudaSuccess || (e = alloc(&h->colmax_bits, Nz, s, tot)) != cudaSuccess ||
-      (e = alloc(&h->w_o, static_cast<size_t>(h->N_pad) * kOutMma, s, tot)) != cudaSuccess ||
       (e = alloc(&h->colkey, Kz, s, tot)) != cudaSuccess || (e = alloc(&h->epoch, 1, s, tot)) != cudaSuccess ||
       (e = alloc(&h->ticket, 1, s, tot)) != cudaSuccess || (e = alloc(&h->mask, words, s, tot)) != cudaSuccess ||
       (e = alloc(&h->pre, words, s, tot)) != cudaSuccess || (e = alloc(&h->omask, 2 * words, s, tot)) != cudaSuccess ||
@@ -466,8 +437,6 @@ int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N
   const uint64_t wb_rows = kblocks * static_cast<uint64_t>(h->N_pad);
   int8mm_status st = make_tmap_i8(&h->tmB, h->Wb, 128, wb_rows, kGemmBK, kGemmBN);
   if (st == INT8MM_OK) st = make_tmap_i8(&h->tmW128, h->Wb, 128, wb_rows, kGemmBK, 128);
-  if (st == INT8MM_OK)
-    st = make_tmap_i8(&h->tmWO, h->w_o, kOutMma * 2, static_cast<uint64_t>(h->N_pad), kOutMma * 2, 128);
   if (st != INT8MM_OK) {
     cudaStreamSynchronize(s);
     free_all(h);

@@ -26,13 +26,15 @@
 // bounded; a timeout sets the status word and the CTA drains and exits.
 //
 // The outlier product X[:,O] W[O,:] (CTA pairs, the first kOutMma outliers)
-// runs on the tensor cores too: the epilogue writes the dequantised tile
-// back into TMEM as fp32, the MMA warp adds X_O W_O^T onto it with
-// tcgen05.mma.kind::f16 (X_O [M][64] and W_O [N][64] fp16, prepared by the
-// activation pass, loaded by TMA like the int8 operands), and the epilogue
-// reads the sums.  The MMA warp issues that product between the int8 k-blocks
-// of the next tile.  Single CTAs (M <= 128) and outliers past kOutMma use
-// CUDA-core FMAs in the epilogue (W rows staged in shared memory).
+// runs on the tensor cores too.  While a tile accumulates, the epilogue warps
+// write its operand blocks into shared memory in the 128-byte-swizzled
+// K-major layout the int8 tiles use: X_O (this CTA's 128 rows x the outliers,
+// from X_OT) and W_O (its 128 columns x the outliers, from the rows W[O,:]).
+// Once the tile is done they write the dequantised tile back into TMEM as
+// fp32; the MMA warp adds X_O W_O^T onto it with tcgen05.mma.kind::f16
+// (K = 16 per step), between the int8 k-blocks of the next tile; the
+// epilogue reads the sums.  Single CTAs (M <= 128) and outliers past
+// kOutMma use CUDA-core FMAs in the epilogue (W rows staged in shared memory).
 //
 // Two modes.  Single CTA (M <= 128): 128x256 tiles, B tiles of 256 rows,
 // 4 stages.  CTA pair (M > 128): a cluster of two CTAs on neighbouring SMs
@@ -57,6 +59,10 @@ constexpr int A_BYTES = BM * BK;  // 16 KB: 128 rows of A per CTA
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int HALF_N = BN / 2;
 constexpr int OUT_CAP = 16;
+// The outlier product of tile t is issued after this many int8 k-blocks of
+// tile t+1 (by then the epilogue has written tile t back to TMEM), splitting
+// the k-block loop in two tight loops.
+constexpr int OUT_ISSUE_KB = 16;
 constexpr int WO_BYTES = 2 * OUT_CAP * HALF_N * 4;
 constexpr int RW_BYTES = 2 * HALF_N * 4;
 constexpr int TMEM_COLS = 2 * BN;
@@ -75,12 +81,12 @@ struct Cfg {
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;  // rows per tile
   static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
   // full, empty, tmem_full[2], tmem_empty[2], drain, and for the outlier
-  // product: operands loaded, operands free, tile dequantised[2], product done[2]
-  static constexpr int NUM_BARS = 2 * STAGES + 5 + 6;
+  // product: tile dequantised (operands staged)[2], product done[2]
+  static constexpr int NUM_BARS = 2 * STAGES + 5 + 4;
   static constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
-  // pairs: the outlier product's operand tiles (128 rows of 128 bytes each:
-  // 64 fp16 outliers of 128 rows of X_O, and of 128 rows of W_O); single CTAs:
-  // the staged outlier weight rows
+  // pairs: the outlier product's operand blocks (128 rows of 128 bytes each:
+  // up to 64 fp16 outliers for 128 rows of X_O, and for 128 columns of W_O);
+  // single CTAs: the staged outlier weight rows
   static constexpr int OA_OFFSET = (MISC_OFFSET + 16 + 1023) & ~1023;
   static constexpr int OB_OFFSET = OA_OFFSET + (PAIR ? A_BYTES : 0);
   static constexpr int WO_OFFSET = OB_OFFSET + (PAIR ? A_BYTES : 0);
@@ -112,7 +118,6 @@ __device__ __forceinline__ float dequant(uint32_t acc, float rx, float rw) {
 template <bool PAIR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_decomp_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                          const __grid_constant__ CUtensorMap tmXO, const __grid_constant__ CUtensorMap tmWO,
                           const GemmArgs a) {
   using C = Cfg<PAIR>;
   constexpr int STAGES = C::STAGES;
@@ -124,10 +129,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* ofull = drain + 1;   // outlier operand tiles landed (leader)
-  uint64_t* oempty = ofull + 1;  // outlier operand tiles read by the product
-  uint64_t* tdeq = oempty + 1;   // [2] tile dequantised into TMEM (leader)
-  uint64_t* tout = tdeq + 2;     // [2] outlier product added
+  uint64_t* tdeq = drain + 1;  // [2] operands staged and tile dequantised into TMEM (leader)
+  uint64_t* tout = tdeq + 2;   // [2] outlier product added
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFFSET);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFFSET + 4);
 
@@ -152,8 +155,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&tempty[b], NUM_EPI_WARPS * (PAIR ? 2 : 1));
     }
     mbar_init(drain, 1);
-    mbar_init(ofull, 1);
-    mbar_init(oempty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tdeq[b], NUM_EPI_WARPS * (PAIR ? 2 : 1));
       mbar_init(&tout[b], 1);
@@ -162,10 +163,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (PAIR) {
-      tma_prefetch_desc(&tmXO);
-      tma_prefetch_desc(&tmWO);
-    }
+
   }
   if (warp == 1) {
     if (PAIR) {
@@ -222,28 +220,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       stage = pre % STAGES;
       phase = pre == STAGES ? 1u : 0u;
-      // Operand tiles of the outlier product of a tile (pairs with |O| > 0):
-      // loaded at the start of the next tile, once the previous product has
-      // read the single buffer.
-      const bool outl = PAIR && *a.count > 0;
-      uint32_t ouse = 0;
-      auto load_outl = [&](int tile) -> bool {
-        if (!mbar_wait(oempty, (ouse & 1u) ^ 1u, tmo, abort_flag)) return false;
-        if (rank == 0) mbar_arrive_expect_tx(ofull, 4 * A_BYTES);  // two CTAs x (X_O + W_O tiles)
-        const uint32_t ob = mapa_shared(smem_u32(ofull), 0);
-        tma_load_2d_pair(smem + C::OA_OFFSET, &tmXO, ob, 0, (tile % num_m) * C::TILE_M + static_cast<int>(rank) * BM);
-        tma_load_2d_pair(smem + C::OB_OFFSET, &tmWO, ob, 0, (tile / num_m) * BN + static_cast<int>(rank) * C::B_ROWS);
-        ++ouse;
-        return true;
-      };
-      int prev = -1;
       for (int tile = tile0; tile < num_tiles && ok; tile += tstride) {
         const int m_blk = tile % num_m, n_blk = tile / num_m;
-        if (outl && prev >= 0 && !load_outl(prev)) {
-          ok = false;
-          break;
-        }
-        prev = tile;
         for (int kb = tile == first ? pre : 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
             ok = false;
@@ -260,7 +238,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (ok && outl && prev >= 0 && !load_outl(prev)) ok = false;
       if (!ok) {
         fail(a, abort_flag);
         // Let every load already issued land before the CTA can exit (a
@@ -268,7 +245,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!PAIR || rank == 0) {
           for (int s = 0; s < STAGES; ++s)
             if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, tmo, nullptr);
-          if (ouse > 0) mbar_wait(ofull, (ouse - 1u) & 1u, tmo, nullptr);
         } else {
           const uint64_t t0 = global_timer_ns();
           while (global_timer_ns() - t0 < 200000ull) {
@@ -284,21 +260,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       int lt = 0;
       // Outlier product of a finished tile (pairs with |O| > 0): once the
-      // epilogue has written the dequantised tile back to TMEM and the
-      // operand tiles have landed, D += X_O W_O^T in min(|O|, 64)/16 steps of
-      // K = 16, issued between the int8 k-blocks of the next tile.
+      // epilogue has staged the operand blocks and written the dequantised
+      // tile back to TMEM, D += X_O W_O^T in min(|O|, 64)/16 steps of K = 16,
+      // issued after OUT_ISSUE_KB int8 k-blocks of the next tile.
       pdl_wait();
       const int cnt = PAIR ? *a.count : 0;
       const int nk = cnt > 0 ? (min(cnt, kOutMma) + 15) / 16 : 0;
-      uint32_t ouse = 0, pend_use = 0;
+      uint32_t pend_use = 0;
       int pend = -1;  // accumulator buffer whose outlier product is due
-      auto issue_outl = [&](bool block) -> bool {
-        if (block) {
-          if (!mbar_wait(&tdeq[pend], pend_use & 1u, tmo, abort_flag) || !mbar_wait(ofull, ouse & 1u, tmo, abort_flag))
-            return false;
-        } else if (!mbar_test_wait(&tdeq[pend], pend_use & 1u) || !mbar_test_wait(ofull, ouse & 1u)) {
-          return true;  // not yet
-        }
+      auto issue_outl = [&]() -> bool {
+        if (!mbar_wait(&tdeq[pend], pend_use & 1u, tmo, abort_flag)) return false;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(pend * BN);
         const uint64_t adesc = smem_desc_k_sw128(smem_u32(smem + C::OA_OFFSET));
@@ -306,9 +277,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kk = 0; kk < nk; ++kk)  // 32 bytes (16 fp16) along K per step
           mma_f16_pair(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2),
                        C::IDESC_F16, 1u);
-        mma_commit_pair(oempty, 0x3);
         mma_commit_pair(&tout[pend], 0x3);
-        ++ouse;
         pend = -1;
         return true;
       };
@@ -321,11 +290,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, tmo, abort_flag)) {
-            ok = false;
-            break;
-          }
+        auto kblock = [&](int kb) -> bool {
+          if (!mbar_wait(&full[stage], phase, tmo, abort_flag)) return false;
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint64_t adesc = smem_desc_k_sw128(sa);
@@ -347,19 +313,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             stage = 0;
             phase ^= 1u;
           }
-          if (pend >= 0) issue_outl(false);
-        }
+          return true;
+        };
+        const int ksplit = pend >= 0 ? min(num_kb, OUT_ISSUE_KB) : num_kb;
+        for (int kb = 0; kb < ksplit && ok; ++kb) ok = kblock(kb);
+        if (ok && pend >= 0) ok = issue_outl();
+        for (int kb = ksplit; kb < num_kb && ok; ++kb) ok = kblock(kb);
         if (ok) {
           if (PAIR) mma_commit_pair(&tfull[buf], 0x3);
           else mma_commit(&tfull[buf]);
         }
-        if (ok && pend >= 0 && !issue_outl(true)) ok = false;
         if (nk > 0) {
           pend = buf;
           pend_use = use;
         }
       }
-      if (ok && pend >= 0 && !issue_outl(true)) ok = false;
+      if (ok && pend >= 0) ok = issue_outl();
       if (!ok) {
         fail(a, abort_flag);
         if (PAIR) mma_commit_pair(drain, 0x1);
@@ -420,6 +389,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int o = 0; o < OUT_CAP; ++o)
         xo[o] = (o < cs && row_ok) ? __half2float(a.X_OT[static_cast<size_t>(o) * M + m]) : 0.0f;
+      if (outl) {
+        // this tile's outlier-product operand blocks, as fp16 rows of the
+        // 128-byte-swizzled K-major layout (16-byte chunk c of row r stored at
+        // chunk c ^ (r % 8), groups of 8 rows 1024 bytes apart): half 0 writes
+        // row tl of X_O (X[m, O_o]), half 1 row tl of W_O (W[O_o, n]); only
+        // the chunks the product reads, zero past |O|.  The previous tile's
+        // product has completed (waited for below), so the blocks are free.
+        const int no = min(cnt, kOutMma), nch = 2 * ((no + 15) / 16);
+        uint8_t* rowp = smem + (h == 0 ? C::OA_OFFSET : C::OB_OFFSET) + (tl >> 3) * 1024 + (tl & 7) * 128;
+        const int mrow = m_blk * C::TILE_M + static_cast<int>(rank) * BM + tl;
+        const int ncol = n_blk * BN + static_cast<int>(rank) * C::B_ROWS + tl;
+        const bool ok_rc = h == 0 ? mrow < M : ncol < N;
+        const uint16_t* src = h == 0 ? reinterpret_cast<const uint16_t*>(a.X_OT) + mrow
+                                     : reinterpret_cast<const uint16_t*>(a.W) + ncol;
+        for (int c = 0; c < nch; ++c) {
+          uint32_t w2[4];
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const int o = 8 * c + 2 * p;
+            uint32_t lo = 0u, hi = 0u;
+            if (ok_rc && o < no)
+              lo = __ldg(src + (h == 0 ? static_cast<size_t>(o) * M : static_cast<size_t>(__ldg(a.idx + o)) * N));
+            if (ok_rc && o + 1 < no)
+              hi = __ldg(src + (h == 0 ? static_cast<size_t>(o + 1) * M : static_cast<size_t>(__ldg(a.idx + o + 1)) * N));
+            w2[p] = lo | (hi << 16);
+          }
+          *reinterpret_cast<uint4*>(rowp + ((c ^ (tl & 7)) << 4)) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
+      }
       float rx = 0.0f;
       if (row_ok) {
         const float c = a.c_x[m];
@@ -583,8 +582,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 template <bool PAIR>
-cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmXO, const CUtensorMap& tmWO,
-                     const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
+cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms, bool pdl,
+                     cudaStream_t stream) {
   using C = Cfg<PAIR>;
   static unsigned long long attr_set = 0;  // one bit per device
   int dev = 0;
@@ -620,17 +619,16 @@ cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUten
   }
   cfg.attrs = attrs;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, gemm_i8_decomp_kernel<PAIR>, tmA, tmB, tmXO, tmWO, a);
+  return cudaLaunchKernelEx(&cfg, gemm_i8_decomp_kernel<PAIR>, tmA, tmB, a);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB256, const CUtensorMap& tmB128,
-                               const CUtensorMap& tmXO, const CUtensorMap& tmWO, const GemmArgs& a, int num_sms,
-                               bool pdl, cudaStream_t stream) {
+                               const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
   // one 128-row tile height: single CTAs; taller problems: CTA pairs
-  if (a.M <= BM) return launch_t<false>(tmA, tmB256, tmXO, tmWO, a, num_sms, pdl, stream);
-  return launch_t<true>(tmA, tmB128, tmXO, tmWO, a, num_sms, pdl, stream);
+  if (a.M <= BM) return launch_t<false>(tmA, tmB256, a, num_sms, pdl, stream);
+  return launch_t<true>(tmA, tmB128, a, num_sms, pdl, stream);
 }
 
 }  // namespace i8mm

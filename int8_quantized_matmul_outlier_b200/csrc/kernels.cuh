@@ -13,9 +13,9 @@ namespace i8mm {
 // Status bits in the device status word.
 constexpr int kStatusTimeout = 1;
 
-// Outliers whose fp16 product the prefill GEMM computes on the tensor cores
-// (kind::f16, from X_O [M][kOutMma] and W_O [N_pad][kOutMma], rows of 128
-// bytes); the GEMM's epilogue adds any further outliers with FMAs.
+// Outliers whose fp16 product the prefill GEMM (CTA pairs) computes on the
+// tensor cores (kind::f16, K = 16 per step, operand rows of 128 bytes); its
+// epilogue adds any further outliers with FMAs.
 constexpr int kOutMma = 64;
 
 // Sets the message returned by int8mm_last_error() on this host thread.
@@ -51,28 +51,13 @@ struct OutlierScratch {
 cudaError_t launch_outlier_detect(const __half* X, int64_t M, int64_t K, float alpha,
                                   const OutlierScratch& s, cudaStream_t stream);
 
-// Operands of the prefill GEMM's tensor-core outlier product, written by the
-// activation pass for the first kOutMma outliers (fp16, kOutMma per row;
-// columns up to the next multiple of 16 are written, zero past |O|):
-// x_o[m][o] = X[m, O_o] and w_o[n][o] = W[O_o, n] (zero for n >= N).
-struct OutlierOperands {
-  const int32_t* idx;    // [K] ascending outlier columns
-  const int32_t* count;  // [1] |O|
-  const __half* W;       // [K, N]
-  int N, N_pad;
-  __half* x_o;           // [M][kOutMma]
-  __half* w_o;           // [N_pad][kOutMma]
-};
-
 // Pass 2: per row, absmax over non-outlier columns, c_x = 127/absmax, int8
-// codes (outlier columns 0), the fp16 outlier values scattered as
-// X_OT[o][i] = X[i, idx[o]] (o-major, M entries per o), and the outlier
-// product's operands (block i also writes rows [i p, i p + p) of w_o, p =
-// ceil(N_pad / M)).  With `pdl`, launched as a programmatic dependent of
-// pass 1: it loads its row of X while that pass finishes.
+// codes (outlier columns 0), and the fp16 outlier values scattered as
+// X_OT[o][i] = X[i, idx[o]] (o-major, M entries per o).  With `pdl`,
+// launched as a programmatic dependent of pass 1: it loads its row of X
+// while that pass finishes.
 cudaError_t launch_row_quant(const __half* X, int64_t M, int64_t K, const OutlierScratch& s,
-                             int8_t* Xq, float* c_x, __half* X_OT, const OutlierOperands& oo, bool pdl,
-                             cudaStream_t stream);
+                             int8_t* Xq, float* c_x, __half* X_OT, bool pdl, cudaStream_t stream);
 
 // ---- fused tcgen05 GEMM ---------------------------------------------------
 struct GemmArgs {
@@ -98,14 +83,11 @@ constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 128;
 // tmB256 / tmB128 map the weight with 256- and 128-row boxes (the second is
-// used by the CTA-pair mode, for M > 128).  tmXO / tmWO map the outlier
-// product's operands x_o [M][kOutMma] and w_o [N_pad][kOutMma] (rows of 128
-// bytes, 128-row boxes; pair mode).  With `pdl`, launched as a programmatic
-// dependent of the activation pass: its prologue and the first weight-tile
-// loads overlap that pass.
+// used by the CTA-pair mode, for M > 128).  With `pdl`, launched as a
+// programmatic dependent of the activation pass: its prologue and the first
+// weight-tile loads overlap that pass.
 cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB256, const CUtensorMap& tmB128,
-                               const CUtensorMap& tmXO, const CUtensorMap& tmWO, const GemmArgs& a, int num_sms,
-                               bool pdl, cudaStream_t stream);
+                               const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream);
 
 // Largest K any kernel here accepts (the row kernels keep a row in registers).
 constexpr int64_t kMaxK = 65536;
@@ -156,11 +138,6 @@ struct RowActArgs {
   float* colmax;               // [K]
   int* status;
   unsigned long long timeout_ns;
-  // operands of the GEMM's tensor-core outlier product (first kOutMma outliers)
-  const __half* W;     // [K, N] fp16 weight
-  int N, N_pad;
-  __half* x_o;         // [M][kOutMma]: X[m, O_o]
-  __half* w_o;         // [N_pad][kOutMma]: W[O_o, n]
 };
 constexpr int64_t kRowActMaxK = 32768;
 constexpr int64_t kRowActMaxRows = 256;

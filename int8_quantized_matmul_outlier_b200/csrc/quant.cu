@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(NT) row_quant_kernel(const __half* __restrict_
                                                        const uint32_t* __restrict__ mask,
                                                        const int32_t* __restrict__ pre,
                                                        int8_t* __restrict__ Xq, float* __restrict__ c_x,
-                                                       __half* __restrict__ X_OT, OutlierOperands oo) {
+                                                       __half* __restrict__ X_OT) {
   const int row = blockIdx.x, tid = threadIdx.x;
   const int nvec = K / 8;
   const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(row) * K);
@@ -309,49 +309,12 @@ __global__ void __launch_bounds__(NT) row_quant_kernel(const __half* __restrict_
       *reinterpret_cast<uint2*>(qr + c8 * 8) = q;
     }
   }
-  // operands of the GEMM's tensor-core outlier product: this row of X_O, and
-  // this block's share of the rows of W_O (see RowActArgs)
-  const int cnt = __ldcg(oo.count);
-  if (cnt > 0) {
-    const int no = min(cnt, kOutMma);
-    const int nch = 2 * ((no + 15) / 16);
-    const uint16_t* Xh = reinterpret_cast<const uint16_t*>(X) + static_cast<size_t>(row) * K;
-    if (tid < nch) {
-      uint32_t w2[4];
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const int o = 8 * tid + 2 * p;
-        const uint32_t lo = o < no ? __ldg(Xh + __ldcg(oo.idx + o)) : 0u;
-        const uint32_t hi = o + 1 < no ? __ldg(Xh + __ldcg(oo.idx + o + 1)) : 0u;
-        w2[p] = lo | (hi << 16);
-      }
-      *reinterpret_cast<uint4*>(oo.x_o + static_cast<size_t>(row) * kOutMma + 8 * tid) =
-          make_uint4(w2[0], w2[1], w2[2], w2[3]);
-    }
-    const int per = (oo.N_pad + M - 1) / M;
-    const int n0 = row * per, n1 = min(oo.N_pad, n0 + per);
-    const uint16_t* Wh = reinterpret_cast<const uint16_t*>(oo.W);
-    for (int it = tid; it < (n1 - n0) * nch; it += NT) {
-      const int n = n0 + it / nch, c = it % nch;
-      uint32_t w2[4];
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const int o = 8 * c + 2 * p;
-        const uint32_t lo = (o < no && n < oo.N) ? __ldg(Wh + static_cast<size_t>(__ldcg(oo.idx + o)) * oo.N + n) : 0u;
-        const uint32_t hi =
-            (o + 1 < no && n < oo.N) ? __ldg(Wh + static_cast<size_t>(__ldcg(oo.idx + o + 1)) * oo.N + n) : 0u;
-        w2[p] = lo | (hi << 16);
-      }
-      *reinterpret_cast<uint4*>(oo.w_o + static_cast<size_t>(n) * kOutMma + 8 * c) =
-          make_uint4(w2[0], w2[1], w2[2], w2[3]);
-    }
-  }
   pdl_launch_dependents();
 }
 
 template <int VPT, int NT>
 cudaError_t launch_row_quant_t(const __half* X, int64_t M, int64_t K, const OutlierScratch& s, int8_t* Xq,
-                               float* c_x, __half* X_OT, const OutlierOperands& oo, bool pdl, cudaStream_t stream) {
+                               float* c_x, __half* X_OT, bool pdl, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(M));
   cfg.blockDim = dim3(NT);
@@ -363,7 +326,7 @@ cudaError_t launch_row_quant_t(const __half* X, int64_t M, int64_t K, const Outl
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, row_quant_kernel<VPT, NT>, X, static_cast<int>(M), static_cast<int>(K),
                             static_cast<const uint32_t*>(s.mask), static_cast<const int32_t*>(s.pre), Xq, c_x,
-                            X_OT, oo);
+                            X_OT);
 }
 
 }  // namespace
@@ -397,12 +360,12 @@ cudaError_t launch_outlier_detect(const __half* X, int64_t M, int64_t K, float a
 }
 
 cudaError_t launch_row_quant(const __half* X, int64_t M, int64_t K, const OutlierScratch& s, int8_t* Xq,
-                             float* c_x, __half* X_OT, const OutlierOperands& oo, bool pdl, cudaStream_t stream) {
+                             float* c_x, __half* X_OT, bool pdl, cudaStream_t stream) {
   // 128 threads per row up to K = 16384, then 256 and 512; each thread
   // keeps VPT vectors of 8 halves of its row in registers.
   const int64_t nvec = K / 8;
 #define I8MM_ROWQ(V, T) \
-  if (nvec <= int64_t(V) * (T)) return launch_row_quant_t<V, T>(X, M, K, s, Xq, c_x, X_OT, oo, pdl, stream)
+  if (nvec <= int64_t(V) * (T)) return launch_row_quant_t<V, T>(X, M, K, s, Xq, c_x, X_OT, pdl, stream)
   I8MM_ROWQ(1, 128);
   I8MM_ROWQ(2, 128);
   I8MM_ROWQ(3, 128);

@@ -70,8 +70,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1) xact_rows_kernel(RowActArgs a)
   __shared__ uint32_t s_gen;
   __shared__ unsigned long long s_epoch;
   __shared__ int s_ok;
-  __shared__ int s_cnt;               // |O|
-  __shared__ int idx_s[kOutMma];      // the first kOutMma outlier columns
 
   // The GEMM that follows may launch now; its blocks take the SMs this
   // kernel leaves.
@@ -203,21 +201,17 @@ __global__ void __launch_bounds__(kMaxThreads, 1) xact_rows_kernel(RowActArgs a)
     int pos = incl - cnt;
     for (int w = w0; w < w1; ++w) {
       pre_s[w] = pos;
-      uint32_t bits = mask_s[w];
-      int o = pos;
-      while (bits && (blockIdx.x == 0 || o < kOutMma)) {
-        const int col = w * 32 + __ffs(bits) - 1;
-        if (blockIdx.x == 0) a.idx[o] = col;
-        if (o < kOutMma) idx_s[o] = col;
-        ++o;
-        bits &= bits - 1;
+      if (blockIdx.x == 0) {
+        uint32_t bits = mask_s[w];
+        int o = pos;
+        while (bits) {
+          a.idx[o++] = w * 32 + __ffs(bits) - 1;
+          bits &= bits - 1;
+        }
       }
       pos += __popc(mask_s[w]);
     }
-    if (lane == 31) {
-      s_cnt = incl;
-      if (blockIdx.x == 0) *a.count = incl;
-    }
+    if (blockIdx.x == 0 && lane == 31) *a.count = incl;
   }
   if (blockIdx.x == 0) {
     uint32_t* next = a.omask + static_cast<size_t>((gen + 1u) & 1u) * KW;
@@ -231,46 +225,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1) xact_rows_kernel(RowActArgs a)
       }
   }
   __syncthreads();
-  // the first kOutMma outlier columns in the operand layouts of the GEMM's
-  // tensor-core outlier product: X_O[m][o] = X[m, O_o] for this block's rows
-  // and, for this block's share of the weight rows, W_O[n][o] = W[O_o, n]
-  // (fp16, 64 per row; columns up to the next multiple of 16 are written,
-  // zero past |O|)
-  if (s_cnt > 0) {
-    const int no = min(s_cnt, kOutMma);
-    const int nch = 2 * ((no + 15) / 16);  // 16-byte chunks per row
-    const __half* xh = reinterpret_cast<const __half*>(xs);
-    for (int it = tid; it < nr * nch; it += NT) {
-      const int j = it / nch, c = it - j * nch;
-      uint32_t w2[4];
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const int o = 8 * c + 2 * p;
-        const uint32_t lo = o < no ? __half_as_ushort(xh[static_cast<size_t>(j) * K + idx_s[o]]) : 0u;
-        const uint32_t hi = o + 1 < no ? __half_as_ushort(xh[static_cast<size_t>(j) * K + idx_s[o + 1]]) : 0u;
-        w2[p] = lo | (hi << 16);
-      }
-      *reinterpret_cast<uint4*>(a.x_o + static_cast<size_t>(r0 + j) * kOutMma + 8 * c) =
-          make_uint4(w2[0], w2[1], w2[2], w2[3]);
-    }
-    const int per = (a.N_pad + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
-    const int n0 = static_cast<int>(blockIdx.x) * per, n1 = min(a.N_pad, n0 + per);
-    const uint16_t* Wh = reinterpret_cast<const uint16_t*>(a.W);
-    for (int n = n0 + tid; n < n1; n += NT) {
-      for (int c = 0; c < nch; ++c) {
-        uint32_t w2[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const int o = 8 * c + 2 * p;
-          const uint32_t lo = (o < no && n < a.N) ? __ldg(Wh + static_cast<size_t>(idx_s[o]) * a.N + n) : 0u;
-          const uint32_t hi = (o + 1 < no && n < a.N) ? __ldg(Wh + static_cast<size_t>(idx_s[o + 1]) * a.N + n) : 0u;
-          w2[p] = lo | (hi << 16);
-        }
-        *reinterpret_cast<uint4*>(a.w_o + static_cast<size_t>(n) * kOutMma + 8 * c) =
-            make_uint4(w2[0], w2[1], w2[2], w2[3]);
-      }
-    }
-  }
   // per owned vector: outlier flags, the masks that keep its non-outlier codes,
   // and the X_OT slot of its first outlier column
   uint32_t fl[VPT], keep[VPT][2];
