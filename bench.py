@@ -290,6 +290,35 @@ def run_decode(m, torch, dev, stream, scrub, steps: int, peaks: dict, max_over, 
     return out
 
 
+def accuracy_report(torch, dev, X, W, Y, rows: int = 32, seed: int = 0) -> dict:
+    """Error of the GPU's Y against the exact matmul of the fp16 inputs (fp64,
+    on seeded sampled rows), next to tensor-wise absmax int8 (one scale for X,
+    one for W, no decomposition) on the same rows.  Plain torch reference
+    arithmetic, outside the timed regions."""
+    M = X.shape[0]
+    g = np.random.default_rng(seed)
+    r = np.unique(np.concatenate([[0, M - 1], g.choice(M, size=min(M, rows) - 2, replace=False)]))
+    ri = torch.from_numpy(r).to(dev)
+    Xr = X.index_select(0, ri).double()
+    Wd = W.double()
+    exact = Xr @ Wd
+    y = Y.index_select(0, ri).double()
+    cx = 127.0 / X.abs().max().double()
+    cw = 127.0 / W.abs().max().double()
+    qx = torch.round(Xr * cx).clamp(-127, 127)   # round half to even
+    qw = torch.round(Wd * cw).clamp(-127, 127)
+    tw = (qx @ qw) / (cx * cw)
+    del Wd, qw
+
+    def err(v):
+        d = v - exact
+        return {"max_abs": float(d.abs().max()), "rel_fro": float(d.norm() / exact.norm())}
+    e_gpu, e_tw = err(y), err(tw)
+    return {"rows_sampled": int(r.size), "reference": "fp64 matmul of the fp16 inputs",
+            "decomposed_gpu": e_gpu, "tensorwise_absmax_int8": e_tw,
+            "rel_fro_ratio_tensorwise_over_decomposed": e_tw["rel_fro"] / max(e_gpu["rel_fro"], 1e-30)}
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -449,6 +478,7 @@ def run_ours(args):
         "clocks": clocks.summary(),
         "wall_s_timed_region": wall,
     }
+    line["accuracy"] = accuracy_report(torch, dev, X, W, Y)
     if args.decode_steps > 0:
         line["decode"] = {
             "workload": "decode: M in (1, 8, 32) tokens x K=12288 x N=49152, 7 outlier columns in every row",

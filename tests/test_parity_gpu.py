@@ -135,6 +135,23 @@ def test_threshold_ties_single_launch_pass():
     assert out["cnt"] == 2
 
 
+@pytest.mark.parametrize("K", [4102, 4096])
+def test_worked_example_error_vs_exact_matmul(K):
+    # the pages' worked example (7 outlier channels among K-7 ordinary ones):
+    # the GPU's decomposed Y against the exact fp16-input matmul, next to the
+    # tensor-wise absmax int8 comparator on the same inputs
+    p = workloads.worked_example(K=K, M=512, N=256)
+    out = check(p)
+    assert out["cnt"] == 7
+    y = out["d"]["Y"].cpu().numpy().astype(np.float64)
+    exact = oracle.matmul_f64(p.X, p.W)
+    tw = oracle.tensorwise_absmax(p.X, p.W)["Y"].astype(np.float64)
+    fro = lambda v: np.linalg.norm(v - exact) / np.linalg.norm(exact)
+    e_gpu, e_tw = fro(y), fro(tw)
+    assert e_gpu * 10 < e_tw, (e_gpu, e_tw)
+    assert np.abs(y - exact).max() < np.abs(tw - exact).max()
+
+
 def test_zero_rows_and_columns():
     p = workloads.small(20, 128, 64, 2, seed=5)
     p.X[4, :] = 0
