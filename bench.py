@@ -220,11 +220,20 @@ def cpu_baseline(p: workloads.Problem, rows: int) -> dict:
         rows = cpu_rows_for(p, 10.0, wq)
     t, _ = oracle_rows_sample(p, rows, wq)
     M, K, N = p.shape
-    return {"value": 2.0 * rows * N * K / t / 1e12, "unit": "TOPS", "cores": oracle.num_threads(),
+    cores = oracle.num_threads()
+    # the Tiny configuration on one thread, for scale
+    tiny = workloads.tiny()
+    oracle.set_num_threads(1)
+    try:
+        t1, _ = oracle_rows_sample(tiny, tiny.shape[0])
+    finally:
+        oracle.set_num_threads(cores)
+    return {"value": 2.0 * rows * N * K / t / 1e12, "unit": "TOPS", "cores": cores,
             "kind": "oracle",
             "sample": f"batch of the first {rows} of {M} rows, whole forward on it; "
                       f"weight codes prepared outside the timed region",
-            "seconds": t}
+            "seconds": t,
+            "single_thread_tiny_forward_s": t1}
 
 
 # --------------------------------------------------------------------------

@@ -63,6 +63,17 @@ def check(p: workloads.Problem, rows=None, w=None, wq=None, check_w_codes=True):
 
 # ---------------------------------------------------------------- small cases
 
+def test_oracle_half_decoder_matches_gpu_conversion():
+    # the oracle's own binary16 decoder against the GPU's fp16 -> fp32
+    # conversion, on all 65 536 codes (NaNs compared as NaN)
+    codes = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    mine = oracle.half_to_double(codes)
+    gpu = torch.from_numpy(codes.view(np.int16)).to(dev()).view(torch.float16).float().cpu().numpy()
+    nan = np.isnan(mine)
+    assert (np.isnan(gpu) == nan).all()
+    assert (mine[~nan] == gpu[~nan].astype(np.float64)).all()
+
+
 def test_tiny():
     out = check(workloads.tiny())
     assert out["cnt"] == 2
