@@ -2,7 +2,7 @@
 // magnitude maxima, the scale c = 127/absmax, round-to-nearest-even int8
 // codes, programmatic-dependent-launch controls, and the few memory
 // operations the single-launch activation pass needs (bulk copies into shared
-// memory, acquire/release flags).
+// memory, release flags; the acquire load is in ptx.cuh).
 //
 // Method: "LLM.int8() — 大模型激活值里藏着几个超大异常通道", 方法1 (one scale
 // per row of X and per column of W, c = 127/absmax, codes rounded to int8).
@@ -112,12 +112,6 @@ __device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gsrc, u
                    static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
                "l"(gsrc), "r"(bytes), "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
                : "memory");
-}
-
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
 }
 
 __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {

@@ -13,10 +13,15 @@
 // Work split (stream-K): the N/128 x K/128 sequence of (n block, k block)
 // steps is cut into gridDim.x equal contiguous ranges, one per persistent CTA,
 // so every SM streams the same number of weight bytes.  A range covers whole
-// n blocks (finished straight from TMEM) and at most two partial ones, whose
-// int32 sums are added exactly into a global buffer; the CTA that brings an
-// n block's k-step count to K/128 (ticket) finishes it and clears the buffer
-// and the ticket again.  Integer sums make the result independent of order.
+// n blocks (finished straight from TMEM) and at most two partial ones.  The
+// piece of a split n block that holds k block 0 owns it: it is the last
+// segment of its CTA's range, while the other pieces are first segments of
+// the following CTAs, done early.  Those add their int32 sums exactly into a
+// global buffer and count their k steps on the block's ticket; the owner
+// waits (bounded) until the ticket shows the rest of K, adds the buffer to
+// its own sums, clears buffer and ticket, and finishes the block.  Owners
+// wait only on pieces that wait on nothing.  Integer sums make the result
+// independent of order.
 //
 // Warps: 0 TMA producer (weight tile + token tile per stage, 6-deep ring,
 // weight loads marked evict-first in L2; the first weight tiles are issued
@@ -279,9 +284,9 @@ __global__ void __launch_bounds__(D_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
 
-      if (sg.kb0 != 0 || sg.kb1 != num_kb) {
-        // partial n block: add into the global sums; the CTA that completes
-        // the block's K range finishes it
+      if (sg.kb0 != 0) {
+        // a later piece of a split n block: add into the global sums and
+        // count the k steps for the block's owner
         if (n_ok) {
 #pragma unroll
           for (int m = 0; m < MP; ++m)
@@ -289,21 +294,37 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         }
         __threadfence();
         dbar_sync(1, 128);
+        if (et == 0) atomicAdd(a.ticket + sg.nb, static_cast<unsigned>(sg.kb1 - sg.kb0));
+        continue;
+      }
+      if (sg.kb1 != num_kb) {
+        // the owner of a split n block: wait for the other pieces' k steps,
+        // then add their sums
         if (et == 0) {
-          const unsigned add = static_cast<unsigned>(sg.kb1 - sg.kb0);
-          *s_flag = (atomicAdd(a.ticket + sg.nb, add) + add == static_cast<unsigned>(num_kb)) ? 1 : 0;
+          const unsigned need = static_cast<unsigned>(num_kb - sg.kb1);
+          int got = 1;
+          if (ld_acquire_gpu_u32(a.ticket + sg.nb) != need) {
+            const uint64_t t0 = global_timer_ns();
+            for (uint32_t it = 1; ld_acquire_gpu_u32(a.ticket + sg.nb) != need; ++it) {
+              if ((it & 15u) == 0 && (*abort_flag || global_timer_ns() - t0 > tmo)) {
+                got = 0;
+                break;
+              }
+            }
+          }
+          if (!got) dfail(a, abort_flag);
+          *s_flag = got;
         }
         dbar_sync(1, 128);
-        const int last = *s_flag;
+        const int got = *s_flag;
         dbar_sync(1, 128);  // s_flag is reused by the next segment
-        if (!last) continue;
-        __threadfence();
+        if (!got) continue;
         if (n_ok) {
 #pragma unroll
           for (int m = 0; m < MP; ++m)
             if (m < M) {
               int32_t* p = a.part + static_cast<size_t>(m) * N + n;
-              r[m] = static_cast<uint32_t>(__ldcg(p));
+              r[m] = static_cast<uint32_t>(static_cast<int>(r[m]) + __ldcg(p));
               *p = 0;
             }
         }

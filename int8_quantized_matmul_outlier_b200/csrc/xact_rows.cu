@@ -156,9 +156,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) xact_rows_kernel(RowActArgs a)
     uint32_t* arrivals = a.sync + (gen & 1u);
     red_release_add_gpu(arrivals, 1u);
     int bar_ok = 1;
-    if (ld_acquire_gpu(arrivals) < gridDim.x) {
+    if (ld_acquire_gpu_u32(arrivals) < gridDim.x) {
       const uint64_t t0 = global_timer_ns();
-      for (uint32_t it = 1; ld_acquire_gpu(arrivals) < gridDim.x; ++it) {
+      for (uint32_t it = 1; ld_acquire_gpu_u32(arrivals) < gridDim.x; ++it) {
         if ((it & 15u) == 0 && global_timer_ns() - t0 > a.timeout_ns) {
           bar_ok = 0;
           break;
