@@ -320,13 +320,16 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         dbar_sync(1, 128);  // s_flag is reused by the next segment
         if (!got) continue;
         if (n_ok) {
+          // all loads first: a store between them would serialise the round
+          // trips (the compiler cannot tell the addresses apart)
+          int32_t v[MP];
+#pragma unroll
+          for (int m = 0; m < MP; ++m) v[m] = m < M ? __ldcg(a.part + static_cast<size_t>(m) * N + n) : 0;
 #pragma unroll
           for (int m = 0; m < MP; ++m)
-            if (m < M) {
-              int32_t* p = a.part + static_cast<size_t>(m) * N + n;
-              r[m] = static_cast<uint32_t>(static_cast<int>(r[m]) + __ldcg(p));
-              *p = 0;
-            }
+            if (m < M) a.part[static_cast<size_t>(m) * N + n] = 0;
+#pragma unroll
+          for (int m = 0; m < MP; ++m) r[m] = static_cast<uint32_t>(static_cast<int>(r[m]) + v[m]);
         }
         if (et == 0) a.ticket[sg.nb] = 0u;
       }
