@@ -61,7 +61,7 @@ def lib():
         L.orc_quantize_cols.argtypes = [P, I64, I64, P, P]
         L.orc_int8_matmul.argtypes = [P, P, I64, I64, I64, P]
         L.orc_int8_matmul.restype = ctypes.c_int
-        L.orc_dequant_add_outliers.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P, P]
+        L.orc_dequant_add_outliers.argtypes = [P, P, P, P, P, I64, I64, I64, P, I64, P, P, P]
         L.orc_matmul_f64.argtypes = [P, P, I64, I64, I64, P]
         L.orc_tensorwise_absmax.argtypes = [P, P, I64, I64, I64, P, P, P, P, P]
         L.orc_tensorwise_absmax.restype = ctypes.c_int
@@ -155,8 +155,9 @@ def int8_matmul(qx: np.ndarray, qw: np.ndarray) -> np.ndarray:
     return acc
 
 
-def dequant_add_outliers(acc, c_x, c_w, X, W, idx):
-    """Steps 4-5: fp16 Y [M,N] and the unrounded double value."""
+def dequant_add_outliers(acc, c_x, c_w, X, W, idx, bias=None):
+    """Steps 4-5 (plus the layer's optional fp16 bias [N]): fp16 Y [M,N] and
+    the unrounded double value."""
     X = _f16(X)
     W = _f16(W)
     acc = np.ascontiguousarray(acc, dtype=np.int32)
@@ -165,17 +166,19 @@ def dequant_add_outliers(acc, c_x, c_w, X, W, idx):
     idx = np.ascontiguousarray(idx, dtype=np.int32)
     M, K = X.shape
     N = W.shape[1]
+    b = None if bias is None else _f16(np.asarray(bias).reshape(N))
     Y = np.empty((M, N), np.uint16)
     Yx = np.empty((M, N), np.float64)
     lib().orc_dequant_add_outliers(_p(acc), _p(c_x), _p(c_w), _p(X), _p(W), M, K, N,
-                                   _p(idx), idx.size, _p(Y), _p(Yx))
+                                   _p(idx), idx.size, None if b is None else _p(b), _p(Y), _p(Yx))
     return Y.view(np.float16), Yx
 
 
-def decomp_matmul(X: np.ndarray, W: np.ndarray, alpha: float, rows=None, wq=None):
+def decomp_matmul(X: np.ndarray, W: np.ndarray, alpha: float, rows=None, wq=None, bias=None):
     """The whole method.  Outlier detection always uses all rows of X; with
     ``rows`` given, only those rows of the output (and of the X codes) are
-    computed.  ``wq`` may pass a previous ``quantize_cols(W)`` result."""
+    computed.  ``wq`` may pass a previous ``quantize_cols(W)`` result;
+    ``bias`` is the layer's optional fp16 bias [N]."""
     X = _f16(X)
     W = _f16(W)
     colmax, idx = outlier_columns(X, alpha)
@@ -183,7 +186,7 @@ def decomp_matmul(X: np.ndarray, W: np.ndarray, alpha: float, rows=None, wq=None
     qx, c_x = quantize_rows(Xr, idx)
     qw, c_w = quantize_cols(W) if wq is None else wq
     acc = int8_matmul(qx, qw)
-    Y, Yx = dequant_add_outliers(acc, c_x, c_w, Xr, W, idx)
+    Y, Yx = dequant_add_outliers(acc, c_x, c_w, Xr, W, idx, bias)
     return dict(colmax=colmax, idx=idx, qx=qx, c_x=c_x, qw=qw, c_w=c_w,
                 acc=acc, Y=Y, Y_exact=Yx)
 

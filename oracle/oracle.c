@@ -218,11 +218,15 @@ int orc_int8_matmul(const int8_t *qx, const int8_t *qw, int64_t M, int64_t K, in
 /* the fp16 outlier product ([estelledc] 方法1/方法2; [gartu] La solution):  */
 /*   y[i,j] = acc[i,j] / (c_x[i] * c_w[j]) + sum_{k in O} X[i,k] * W[k,j]    */
 /* in double, rounded once to fp16.  A zero scale means a zero int8 term.   */
+/* bias (optional, fp16 [N]) is the layer's bias b[j] ([gartu] Exemple      */
+/* pratique: the int8 layer that replaces nn.Linear keeps bias=True), added */
+/* to the double sum before the rounding.                                   */
 /* Y_exact (optional) receives the unrounded double.                         */
 void orc_dequant_add_outliers(const int32_t *acc, const float *cx, const float *cw,
                               const uint16_t *X, const uint16_t *W,
                               int64_t M, int64_t K, int64_t N,
                               const int32_t *idx, int64_t n_out,
+                              const uint16_t *bias,
                               uint16_t *Y, double *Y_exact)
 {
     #pragma omp parallel
@@ -240,6 +244,8 @@ void orc_dequant_add_outliers(const int32_t *acc, const float *cx, const float *
                 for (int64_t j = 0; j < N; ++j)
                     row[j] += x * orc_half_to_double(W[k * N + j]);
             }
+            if (bias)  /* the layer's bias, added before the one rounding */
+                for (int64_t j = 0; j < N; ++j) row[j] += orc_half_to_double(bias[j]);
             for (int64_t j = 0; j < N; ++j) {
                 Y[i * N + j] = orc_double_to_half(row[j]);
                 if (Y_exact) Y_exact[i * N + j] = row[j];

@@ -176,6 +176,25 @@ def test_T3_alpha_zero_is_exact_fp16_matmul():
     assert (r["Y"].view(np.uint16) == ref.view(np.uint16)).all()
 
 
+def test_T3_with_bias_adds_before_the_single_rounding():
+    # the layer's bias (gartu "Exemple pratique": the int8 layer replacing
+    # nn.Linear keeps its bias) joins the exact double sum before the one
+    # fp16 rounding: with alpha = 0 the result is fp16(X W + b) bit for bit
+    rng = np.random.default_rng(33)
+    M, K, N = 9, 40, 17
+    X = (rng.integers(-256, 256, (M, K)) / 64.0).astype(np.float16)
+    W = (rng.integers(-256, 256, (K, N)) / 64.0).astype(np.float16)
+    b = (rng.integers(-4096, 4096, N) / 1024.0 + 1.0 / 4096).astype(np.float16)
+    r = oracle.decomp_matmul(X, W, 0.0, bias=b)
+    exact = X.astype(np.float64) @ W.astype(np.float64) + b.astype(np.float64)
+    assert (r["Y"].view(np.uint16) == exact.astype(np.float16).view(np.uint16)).all()
+    assert (r["Y_exact"] == exact).all()
+    # and with alpha = inf the bias shifts the unrounded value by exactly b
+    r0 = oracle.decomp_matmul(X, W, np.inf)
+    r1 = oracle.decomp_matmul(X, W, np.inf, bias=b)
+    assert np.allclose(r1["Y_exact"] - r0["Y_exact"], b.astype(np.float64)[None, :], rtol=0, atol=1e-12)
+
+
 # --------------------------------------------------------------------------
 # T5: the pages' worked example (estelledc 案例1): 7 outlier channels among
 # ordinary ones destroy tensor-wise absmax resolution but not the decomposition
