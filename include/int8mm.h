@@ -108,6 +108,19 @@ int8mm_status int8mm_forward(int8mm_weight_t h, const void* X_fp16_dev, int64_t 
                              void* Y_fp16_dev, void* stream);
 
 /*
+ * Forward of a linear layer with bias: as int8mm_forward, plus the layer's
+ * bias b[j] added to each output before the single rounding to fp16,
+ * Y = fp16(X_int8 W_int8 / scales + X_fp16 W_fp16 + b) ("LLM.int8()",
+ * brain.gartu.xyz, "Exemple pratique": the int8 layer that replaces
+ * nn.Linear keeps its bias).
+ *
+ * bias_fp16_dev: [N] fp16, 16-byte aligned, read-only; NULL means no bias
+ *   (the same as int8mm_forward).  A misaligned bias is an alignment error.
+ */
+int8mm_status int8mm_forward_bias(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
+                                  const void* bias_fp16_dev, void* Y_fp16_dev, void* stream);
+
+/*
  * Same as int8mm_forward for host-resident X and Y: copies X_fp16_host
  * [M, K] into a handle-owned device buffer, runs the forward, and copies Y
  * back into Y_fp16_host [M, N], all enqueued on `stream`.  Y_fp16_host is

@@ -39,6 +39,7 @@ SIGNATURES = {
     "int8mm_reserve": (_ST, [_P, _I64, _P]),
     "int8mm_forward": (_ST, [_P, _P, _I64, ctypes.c_float, _P, _P]),
     "int8mm_forward_host": (_ST, [_P, _P, _I64, ctypes.c_float, _P, _P]),
+    "int8mm_forward_bias": (_ST, [_P, _P, _I64, ctypes.c_float, _P, _P, _P]),
     "int8mm_forward_events": (_ST, [_P, _P, _I64, ctypes.c_float, _P, _P, ctypes.POINTER(_P)]),
     "int8mm_forward_debug": (_ST, [_P, _P, _I64, ctypes.c_float, _P, _P, _P]),
     "int8mm_get_status": (_ST, [_P]),
@@ -141,6 +142,26 @@ def int8mm_forward(w: Weight, X: torch.Tensor, alpha: float = 6.0, Y: torch.Tens
         Y = torch.empty((M, w.N), dtype=torch.float16, device=X.device)
     _dev_f16_2d(Y, "Y")
     _check(lib().int8mm_forward(w.handle, X.data_ptr(), M, float(alpha), Y.data_ptr(), _stream(stream)))
+    return Y
+
+
+def int8mm_forward_bias(w: Weight, X: torch.Tensor, alpha: float = 6.0, bias: torch.Tensor | None = None,
+                        Y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """int8mm_forward plus the layer's fp16 bias [N] (None: no bias)."""
+    _dev_f16_2d(X, "X")
+    M = X.shape[0]
+    if X.shape[1] != w.K:
+        raise ValueError(f"X has {X.shape[1]} columns, the weight has K={w.K}")
+    bp = None
+    if bias is not None:
+        if (not bias.is_cuda or bias.dtype != torch.float16 or not bias.is_contiguous()
+                or bias.numel() != w.N or bias.device != X.device):
+            raise ValueError("bias must be a contiguous float16 tensor of N elements on X's device")
+        bp = bias.data_ptr()
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.float16, device=X.device)
+    _dev_f16_2d(Y, "Y")
+    _check(lib().int8mm_forward_bias(w.handle, X.data_ptr(), M, float(alpha), bp, Y.data_ptr(), _stream(stream)))
     return Y
 
 
@@ -249,3 +270,5 @@ def int8mm_free(w: Weight) -> None:
     if h:
         lib().int8mm_free(h)
 
+
+from .linear import Linear8bitLt  # noqa: E402  (the layer over the functions above)

@@ -233,7 +233,7 @@ int8mm_status set_device(const int8mm_weight* h) {
 }
 
 int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alpha, void* Y, cudaStream_t s,
-                           void* const* events, const int8mm_debug_bufs* dbg) {
+                           void* const* events, const int8mm_debug_bufs* dbg, const void* bias = nullptr) {
   int8mm_status st = check_forward_args(h, X, M, alpha, Y);
   if (st != INT8MM_OK) return st;
   if (M == 0) return INT8MM_OK;
@@ -315,6 +315,7 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     d.idx = h->idx;
     d.count = h->count;
     d.Y = static_cast<__half*>(Y);
+    d.bias = static_cast<const __half*>(bias);
     d.acc_dump = dbg ? dbg->acc : nullptr;
     d.part = h->part;
     d.ticket = h->dticket;
@@ -335,6 +336,7 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     a.idx = h->idx;
     a.count = h->count;
     a.Y = static_cast<__half*>(Y);
+    a.bias = static_cast<const __half*>(bias);
     a.acc_dump = dbg ? dbg->acc : nullptr;
     a.status = h->status;
     a.timeout_ns = h->timeout_ns;
@@ -462,6 +464,14 @@ int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream) {
 int8mm_status int8mm_forward(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha, void* Y_fp16_dev,
                              void* stream) {
   return forward_impl(h, X_fp16_dev, M, alpha, Y_fp16_dev, static_cast<cudaStream_t>(stream), nullptr, nullptr);
+}
+
+int8mm_status int8mm_forward_bias(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
+                                  const void* bias_fp16_dev, void* Y_fp16_dev, void* stream) {
+  if (bias_fp16_dev != nullptr && !aligned16(bias_fp16_dev))
+    return fail(INT8MM_ERR_ALIGNMENT, "bias must be 16-byte aligned");
+  return forward_impl(h, X_fp16_dev, M, alpha, Y_fp16_dev, static_cast<cudaStream_t>(stream), nullptr, nullptr,
+                      bias_fp16_dev);
 }
 
 int8mm_status int8mm_forward_events(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,

@@ -1,7 +1,8 @@
 // Fused int8 GEMM of the LLM.int8() decomposed matmul for sm_100a.
 //
-//   Y[i,j] = fp16( Acc[i,j] / (c_x[i] c_w[j]) + sum_{k in O} X[i,k] W[k,j] )
+//   Y[i,j] = fp16( Acc[i,j] / (c_x[i] c_w[j]) + sum_{k in O} X[i,k] W[k,j] [+ b[j]] )
 //   Acc    = Xq Wq^T, int8 x int8 -> int32 on the 5th-generation tensor cores
+//   b      = the layer's optional fp16 bias, added before the one rounding
 //
 // Method: "LLM.int8() — 大模型激活值里藏着几个超大异常通道", 方法1 (the int8
 // product is dequantised by the outer product of the row and column scales)
@@ -113,6 +114,27 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 
 __device__ __forceinline__ float dequant(uint32_t acc, float rx, float rw) {
   return __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(acc)), rx), rw);
+}
+
+// The layer bias of 32 columns n.. (16 when only those are inside N), as
+// fp32; zero without a bias.  The same addresses for every lane of the warp.
+__device__ __forceinline__ void load_bias32(const __half* bias, int n, bool full32, float (&b)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) b[i] = 0.0f;
+  if (bias == nullptr) return;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if (c < 2 || full32) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(bias + n) + c);
+      const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float2 f = __half22float2(h2[p]);
+        b[8 * c + 2 * p] = f.x;
+        b[8 * c + 2 * p + 1] = f.y;
+      }
+    }
+  }
 }
 
 template <bool PAIR>
@@ -453,14 +475,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int t4 = 0; t4 < 8; ++t4)
               if (n + 32 <= N || t4 < 4) ap[t4] = make_uint4(r[4 * t4], r[4 * t4 + 1], r[4 * t4 + 2], r[4 * t4 + 3]);
           }
+          float bb[32];
+          load_bias32(n < N ? a.bias : nullptr, n, n + 32 <= N, bb);
           const float4* rw4 = reinterpret_cast<const float4*>(rws + cl);
 #pragma unroll
           for (int t4 = 0; t4 < 8; ++t4) {
             const float4 w = rw4[t4];
-            r[4 * t4 + 0] = __float_as_uint(dequant(r[4 * t4 + 0], rx, w.x));
-            r[4 * t4 + 1] = __float_as_uint(dequant(r[4 * t4 + 1], rx, w.y));
-            r[4 * t4 + 2] = __float_as_uint(dequant(r[4 * t4 + 2], rx, w.z));
-            r[4 * t4 + 3] = __float_as_uint(dequant(r[4 * t4 + 3], rx, w.w));
+            r[4 * t4 + 0] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 0], rx, w.x), bb[4 * t4 + 0]));
+            r[4 * t4 + 1] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 1], rx, w.y), bb[4 * t4 + 1]));
+            r[4 * t4 + 2] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 2], rx, w.z), bb[4 * t4 + 2]));
+            r[4 * t4 + 3] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 3], rx, w.w), bb[4 * t4 + 3]));
           }
           tmem_st_32x32b_x32(t_row + static_cast<uint32_t>(cl), r);
         }
@@ -497,14 +521,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
         } else {
+          load_bias32(a.bias, n, full32, v);
           const float4* rw4 = reinterpret_cast<const float4*>(rws + cl);
 #pragma unroll
           for (int t4 = 0; t4 < 8; ++t4) {
             const float4 w = rw4[t4];
-            v[4 * t4 + 0] = dequant(r[4 * t4 + 0], rx, w.x);
-            v[4 * t4 + 1] = dequant(r[4 * t4 + 1], rx, w.y);
-            v[4 * t4 + 2] = dequant(r[4 * t4 + 2], rx, w.z);
-            v[4 * t4 + 3] = dequant(r[4 * t4 + 3], rx, w.w);
+            v[4 * t4 + 0] = __fadd_rn(dequant(r[4 * t4 + 0], rx, w.x), v[4 * t4 + 0]);
+            v[4 * t4 + 1] = __fadd_rn(dequant(r[4 * t4 + 1], rx, w.y), v[4 * t4 + 1]);
+            v[4 * t4 + 2] = __fadd_rn(dequant(r[4 * t4 + 2], rx, w.z), v[4 * t4 + 2]);
+            v[4 * t4 + 3] = __fadd_rn(dequant(r[4 * t4 + 3], rx, w.w), v[4 * t4 + 3]);
           }
         }
         // fp16 outlier product X[m, O] . W[O, n..n+31] with fp32 accumulation,

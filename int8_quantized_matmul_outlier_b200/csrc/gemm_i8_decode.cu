@@ -1,6 +1,6 @@
 // Decode-shape variant of the fused int8 GEMM (few tokens, M <= 64) for sm_100a.
 //
-//   Y[m,n] = fp16( Acc[m,n] / (c_x[m] c_w[n]) + sum_{k in O} X[m,k] W[k,n] ),  Acc = Xq Wq^T
+//   Y[m,n] = fp16( Acc[m,n] / (c_x[m] c_w[n]) + sum_{k in O} X[m,k] W[k,n] [+ b[n]] ),  Acc = Xq Wq^T
 //
 // Method: as the prefill kernel ("LLM.int8() — 大模型激活值里藏着几个超大异常通道",
 // 方法1 and 方法2; the Fig. 2 caption of the AI 十大核心论文解读 article).
@@ -336,10 +336,12 @@ __global__ void __launch_bounds__(D_THREADS, 1)
       if (!n_ok) continue;
       // dequantise, add the fp16 outlier product, write fp16 (coalesced over n)
       const float rw = __ldg(a.inv_cw + n);
+      const float bn = a.bias != nullptr ? __half2float(a.bias[n]) : 0.0f;
       float y[MP];
 #pragma unroll
       for (int m = 0; m < MP; ++m)
-        y[m] = m < M ? __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[m])), rx_s[m]), rw) : 0.0f;
+        y[m] = m < M ? __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[m])), rx_s[m]), rw), bn)
+                     : 0.0f;
 #pragma unroll
       for (int o = 0; o < C::WCAP; ++o)
         if (o < cs) {

@@ -70,6 +70,7 @@ struct GemmArgs {
   const int32_t* idx;      // [K] ascending outlier columns
   const int32_t* count;    // [1] |O|
   __half* Y;               // [M,N] fp16 output
+  const __half* bias;      // [N] fp16 layer bias added before the rounding, or nullptr
   int32_t* acc_dump;       // [M,N] int32 accumulators, or nullptr
   int* status;             // device status word
   unsigned long long timeout_ns;
@@ -159,6 +160,7 @@ struct DecodeArgs {
   const int32_t* idx;      // [K]
   const int32_t* count;    // [1]
   __half* Y;               // [M,N]
+  const __half* bias;      // [N] or nullptr
   int32_t* acc_dump;       // [M,N] or nullptr
   int32_t* part;           // [64][N] int32 partial sums, zero between launches
   unsigned* ticket;        // [ceil(N/128)] k-steps done per n block, zero between launches

@@ -165,6 +165,62 @@ def test_worked_example_error_vs_exact_matmul(K):
     assert np.abs(y - exact).max() < np.abs(tw - exact).max()
 
 
+BIAS_SHAPES = [
+    # M, K, N, planted outliers, alpha
+    (300, 1040, 784, 5, 6.0),      # CTA pairs: bias joins the tensor-core outlier product
+    (257, 384, 512, 3, math.inf),  # CTA pairs, no outliers: direct epilogue
+    (100, 512, 272, 4, 6.0),       # single CTAs: FMA epilogue, ragged N tail
+    (8, 2048, 1168, 4, 6.0),       # decode kernel with split n blocks
+    (40, 1040, 784, 0, 6.0),       # decode kernel, no outliers
+]
+
+
+@pytest.mark.parametrize("M,K,N,n_out,alpha", BIAS_SHAPES)
+def test_forward_with_bias(M, K, N, n_out, alpha):
+    p = workloads.small(M, K, N, n_out, seed=M + 3 * K + N, alpha=alpha)
+    b = (np.random.default_rng(M + N).standard_normal(N) * 0.5).astype(np.float16)
+    w = m.int8mm_prepare_weight(torch.from_numpy(p.W).to(dev()))
+    y = m.int8mm_forward_bias(w, torch.from_numpy(p.X).to(dev()), alpha, torch.from_numpy(b).to(dev()))
+    y0 = m.int8mm_forward(w, torch.from_numpy(p.X).to(dev()), alpha)
+    torch.cuda.synchronize()
+    r = oracle.decomp_matmul(p.X, p.W, alpha, bias=b)
+    assert_y_close(y.cpu().numpy(), r["Y"], p.X, p.W, r["idx"])
+    assert not torch.equal(y, y0)
+    # no bias pointer is the plain forward
+    y1 = m.int8mm_forward_bias(w, torch.from_numpy(p.X).to(dev()), alpha, None)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y0)
+
+
+def test_linear8bitlt_module():
+    torch.manual_seed(0)
+    K, N = 1040, 784
+    lin = torch.nn.Linear(K, N, bias=True).to(dev()).half()
+    with torch.no_grad():
+        lin.weight.normal_(0.0, 0.02)
+        lin.bias.normal_(0.0, 0.5)
+    q = m.Linear8bitLt.from_linear(lin, threshold=6.0)
+    p = workloads.small(2 * 75, K, N, 4, seed=9)
+    x = torch.from_numpy(p.X).to(dev()).reshape(2, 75, K)
+    y = q(x)
+    torch.cuda.synchronize()
+    assert y.shape == (2, 75, N) and y.dtype == torch.float16
+    W = lin.weight.detach().t().contiguous().cpu().numpy()
+    b = lin.bias.detach().cpu().numpy()
+    r = oracle.decomp_matmul(p.X, W, 6.0, bias=b)
+    assert_y_close(y.reshape(-1, N).cpu().numpy(), r["Y"], p.X, W, r["idx"])
+    # the same layer without bias, and the layer's fp16 reference stays close
+    q0 = m.Linear8bitLt(K, N, bias=False, device=dev())
+    with torch.no_grad():
+        q0.weight.copy_(lin.weight.t())
+    y0 = q0(x)
+    ref = (x.float() @ lin.weight.float().t() + lin.bias.float())
+    assert (y.float() - ref).norm() / ref.norm() < 0.02
+    assert torch.allclose(y0.float() + lin.bias.float(), y.float(), atol=2e-2, rtol=1e-2)
+    with pytest.raises(TypeError):
+        q(x.float())
+
+
 def test_zero_rows_and_columns():
     p = workloads.small(20, 128, 64, 2, seed=5)
     p.X[4, :] = 0
