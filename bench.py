@@ -328,6 +328,35 @@ def accuracy_report(torch, dev, X, W, Y, rows: int = 32, seed: int = 0) -> dict:
             "rel_fro_ratio_tensorwise_over_decomposed": e_tw["rel_fro"] / max(e_gpu["rel_fro"], 1e-30)}
 
 
+def run_ffn_contraction(m, torch, dev, stream, scrub, steps: int, peak_tops: float, max_over, rank: int) -> dict:
+    """The FFN's second layer at OPT-13B size (K = 20480 > N = 5120): whole
+    forwards timed with events around each (the GEMM a programmatic
+    dependent), L2 scrubbed between them."""
+    p = workloads.opt13b_contraction(repeat=rank)
+    M, K, N = p.shape
+    X = torch.from_numpy(p.X).to(dev)
+    W = torch.from_numpy(p.W).to(dev)
+    w = m.int8mm_prepare_weight(W)
+    Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    for _ in range(5):
+        m.int8mm_forward(w, X, p.alpha, Y)
+        scrub.zero_()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        e0.record(stream)
+        m.int8mm_forward(w, X, p.alpha, Y)
+        e1.record(stream)
+        scrub.zero_()
+    torch.cuda.synchronize()
+    ms = max_over(float(np.mean([e0.elapsed_time(e1) for e0, e1 in ev])))
+    tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+    out = {"workload": p.name, "M": M, "K": K, "N": N, "ms_per_step": ms, "TOPS": tops,
+           "frac_int8_peak": tops / peak_tops, "gpu_launches_per_step": m.int8mm_launches_per_forward(w, M)}
+    m.int8mm_free(w)
+    return out
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -489,6 +518,8 @@ def run_ours(args):
     }
     line["accuracy"] = accuracy_report(torch, dev, X, W, Y)
     if args.decode_steps > 0:
+        line["ffn_contraction"] = run_ffn_contraction(m, torch, dev, stream, scrub, min(args.decode_steps, 100),
+                                                      peak_tops, lambda x: max_over_ranks(x, dev), rank)
         line["decode"] = {
             "workload": "decode: M in (1, 8, 32) tokens x K=12288 x N=49152, 7 outlier columns in every row",
             "timing": "CUDA events around each whole forward (no event between its kernels), L2 scrubbed "

@@ -137,7 +137,9 @@ __device__ __forceinline__ void load_bias32(const __half* bias, int n, bool full
   }
 }
 
-template <bool PAIR>
+// BIAS: the layer bias is added (a separate instantiation, so that the
+// common bias-free path carries none of its code).
+template <bool PAIR, bool BIAS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_decomp_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const GemmArgs a) {
@@ -475,16 +477,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int t4 = 0; t4 < 8; ++t4)
               if (n + 32 <= N || t4 < 4) ap[t4] = make_uint4(r[4 * t4], r[4 * t4 + 1], r[4 * t4 + 2], r[4 * t4 + 3]);
           }
-          float bb[32];
-          load_bias32(n < N ? a.bias : nullptr, n, n + 32 <= N, bb);
           const float4* rw4 = reinterpret_cast<const float4*>(rws + cl);
+          if (BIAS) {
+            float bb[32];
+            load_bias32(n < N ? a.bias : nullptr, n, n + 32 <= N, bb);
 #pragma unroll
-          for (int t4 = 0; t4 < 8; ++t4) {
-            const float4 w = rw4[t4];
-            r[4 * t4 + 0] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 0], rx, w.x), bb[4 * t4 + 0]));
-            r[4 * t4 + 1] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 1], rx, w.y), bb[4 * t4 + 1]));
-            r[4 * t4 + 2] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 2], rx, w.z), bb[4 * t4 + 2]));
-            r[4 * t4 + 3] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 3], rx, w.w), bb[4 * t4 + 3]));
+            for (int t4 = 0; t4 < 8; ++t4) {
+              const float4 w = rw4[t4];
+              r[4 * t4 + 0] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 0], rx, w.x), bb[4 * t4 + 0]));
+              r[4 * t4 + 1] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 1], rx, w.y), bb[4 * t4 + 1]));
+              r[4 * t4 + 2] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 2], rx, w.z), bb[4 * t4 + 2]));
+              r[4 * t4 + 3] = __float_as_uint(__fadd_rn(dequant(r[4 * t4 + 3], rx, w.w), bb[4 * t4 + 3]));
+            }
+          } else {
+#pragma unroll
+            for (int t4 = 0; t4 < 8; ++t4) {
+              const float4 w = rw4[t4];
+              r[4 * t4 + 0] = __float_as_uint(dequant(r[4 * t4 + 0], rx, w.x));
+              r[4 * t4 + 1] = __float_as_uint(dequant(r[4 * t4 + 1], rx, w.y));
+              r[4 * t4 + 2] = __float_as_uint(dequant(r[4 * t4 + 2], rx, w.z));
+              r[4 * t4 + 3] = __float_as_uint(dequant(r[4 * t4 + 3], rx, w.w));
+            }
           }
           tmem_st_32x32b_x32(t_row + static_cast<uint32_t>(cl), r);
         }
@@ -521,15 +534,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
         } else {
-          load_bias32(a.bias, n, full32, v);
           const float4* rw4 = reinterpret_cast<const float4*>(rws + cl);
 #pragma unroll
           for (int t4 = 0; t4 < 8; ++t4) {
             const float4 w = rw4[t4];
-            v[4 * t4 + 0] = __fadd_rn(dequant(r[4 * t4 + 0], rx, w.x), v[4 * t4 + 0]);
-            v[4 * t4 + 1] = __fadd_rn(dequant(r[4 * t4 + 1], rx, w.y), v[4 * t4 + 1]);
-            v[4 * t4 + 2] = __fadd_rn(dequant(r[4 * t4 + 2], rx, w.z), v[4 * t4 + 2]);
-            v[4 * t4 + 3] = __fadd_rn(dequant(r[4 * t4 + 3], rx, w.w), v[4 * t4 + 3]);
+            v[4 * t4 + 0] = dequant(r[4 * t4 + 0], rx, w.x);
+            v[4 * t4 + 1] = dequant(r[4 * t4 + 1], rx, w.y);
+            v[4 * t4 + 2] = dequant(r[4 * t4 + 2], rx, w.z);
+            v[4 * t4 + 3] = dequant(r[4 * t4 + 3], rx, w.w);
+          }
+          if (BIAS) {
+            float bb[32];
+            load_bias32(a.bias, n, full32, bb);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __fadd_rn(v[i], bb[i]);
           }
         }
         // fp16 outlier product X[m, O] . W[O, n..n+31] with fp32 accumulation,
@@ -606,7 +624,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <bool PAIR>
+template <bool PAIR, bool BIAS>
 cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms, bool pdl,
                      cudaStream_t stream) {
   using C = Cfg<PAIR>;
@@ -615,7 +633,7 @@ cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmA
   cudaGetDevice(&dev);
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_i8_decomp_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemm_i8_decomp_kernel<PAIR, BIAS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set |= bit;
@@ -644,7 +662,7 @@ cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmA
   }
   cfg.attrs = attrs;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, gemm_i8_decomp_kernel<PAIR>, tmA, tmB, a);
+  return cudaLaunchKernelEx(&cfg, gemm_i8_decomp_kernel<PAIR, BIAS>, tmA, tmB, a);
 }
 
 }  // namespace
@@ -652,8 +670,12 @@ cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmA
 cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB256, const CUtensorMap& tmB128,
                                const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
   // one 128-row tile height: single CTAs; taller problems: CTA pairs
-  if (a.M <= BM) return launch_t<false>(tmA, tmB256, a, num_sms, pdl, stream);
-  return launch_t<true>(tmA, tmB128, a, num_sms, pdl, stream);
+  const bool bias = a.bias != nullptr;
+  if (a.M <= BM)
+    return bias ? launch_t<false, true>(tmA, tmB256, a, num_sms, pdl, stream)
+                : launch_t<false, false>(tmA, tmB256, a, num_sms, pdl, stream);
+  return bias ? launch_t<true, true>(tmA, tmB128, a, num_sms, pdl, stream)
+              : launch_t<true, false>(tmA, tmB128, a, num_sms, pdl, stream);
 }
 
 }  // namespace i8mm

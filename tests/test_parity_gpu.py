@@ -381,6 +381,18 @@ def test_opt13b_prefill_full_size():
     m.int8mm_free(out["w"])
 
 
+def test_opt13b_ffn_contraction_full_size():
+    # the FFN's second layer (K = 20480 > N = 5120): the activation (84 MB)
+    # exceeds the SMs' shared memory, so the two-kernel activation path runs
+    p = workloads.opt13b_contraction()
+    W = torch.from_numpy(p.W).to(dev())
+    w = m.int8mm_prepare_weight(W)
+    assert m.int8mm_launches_per_forward(w, p.X.shape[0]) == 3
+    out = check(p, w=w, rows=sample_rows(p.X.shape[0], 16, seed=2))
+    assert out["cnt"] == 7
+    m.int8mm_free(w)
+
+
 def test_175b_prefill_full_size(w175):
     p, w, wq = w175
     out = check(p, rows=sample_rows(p.X.shape[0], 8, seed=2), w=w, wq=wq)

@@ -127,6 +127,13 @@ def gpt175b_prefill(repeat: int = 0, M: int = 2048, with_weight: bool = True) ->
     return _ffn_prefill(f"175b_ffn1_m{M}_k12288_n49152", 2, M, 12288, 49152, repeat, with_weight)
 
 
+def opt13b_contraction(repeat: int = 0, M: int = 2048, with_weight: bool = True) -> Problem:
+    """OPT-13B FFN contraction, the layer after the expansion: M=2048 tokens,
+    K=20480, N=5120 (K > N), the same activation statistics (7 outlier
+    columns, mean |x| 65, max 130, in 75% of rows; ordinary mean |x| 0.5)."""
+    return _ffn_prefill(f"opt13b_ffn2_m{M}_k20480_n5120", 6, M, 20480, 5120, repeat, with_weight)
+
+
 def decode(M: int, repeat: int = 0, K: int = 12288, N: int = 49152,
            with_weight: bool = True) -> Problem:
     """Decode step: M in {1, 8, 32} tokens, K=12288, N=49152.  The 7 outlier
@@ -172,4 +179,5 @@ WORKLOADS = {
     "tiny": tiny,
     "opt13b": opt13b_prefill,
     "175b": gpt175b_prefill,
+    "opt13b_ffn2": opt13b_contraction,
 }
