@@ -277,6 +277,8 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     ra.M = static_cast<int>(M);
     ra.K = static_cast<int>(h->K);
     ra.rows_per_block = 0;
+    ra.chunk_rows = 0;
+    ra.slots = 0;
     ra.col_threads = 0;
     ra.thr = half_magnitude_threshold(alpha);
     ra.Xq = h->Xq;

@@ -116,15 +116,18 @@ constexpr size_t kSmallActSmemMax = 200 * 1024;
 bool small_act_fits(int64_t M, int64_t K);
 cudaError_t launch_small_act(const SmallActArgs& a, cudaStream_t stream);
 
-// ---- activation pass in one launch (rows held in shared memory) -----------
-// Detection, quantisation and the outlier gather for an X whose rows, split
-// into equal runs across one block per SM, fit in shared memory
-// (csrc/xact_rows.cu).  A cooperative launch with one grid barrier; writes
-// idx, count, Xq, c_x and X_OT (and colmax when colkey is given).
+// ---- activation pass in one launch --------------------------------------
+// Detection, quantisation and the outlier gather (csrc/xact_rows.cu) for K <=
+// kRowActMaxK: the rows, split into equal runs across one block per SM, are
+// held in shared memory when they fit, else streamed through it twice (in
+// chunks, double-buffered).  A cooperative launch with one grid barrier;
+// writes idx, count, Xq, c_x and X_OT (and colmax when colkey is given).
 struct RowActArgs {
   const __half* X;     // [M, K]
   int M, K;
   int rows_per_block;  // set by the launcher
+  int chunk_rows;      // set by the launcher: rows per chunk (= rows_per_block when all fit)
+  int slots;           // set by the launcher: row slots in shared memory
   int col_threads;     // set by the launcher: threads per row group
   int thr;             // half_magnitude_threshold(alpha)
   int8_t* Xq;          // [M, K]

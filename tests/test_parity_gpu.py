@@ -101,6 +101,9 @@ SHAPES = [
     (300, 16, 32, 1, 6.0),          # smallest K, three rows per block
     (149, 32768, 256, 3, 6.0),      # largest K of the single-launch pass, one row per block
     (3000, 5120, 256, 7, 6.0),      # 21 rows (210 KB) of X per block
+    (4000, 5120, 256, 5, 6.0),      # streamed: 28 rows per block in chunks of 10, a short last chunk
+    (600, 20480, 256, 7, 6.0),      # streamed, two 40 KB rows per chunk
+    (130, 40960, 256, 3, 6.0),      # K > 32768: two-kernel activation path
 ]
 
 
@@ -247,8 +250,9 @@ def test_repeat_and_stale_state():
 
 
 def test_activation_paths_alternate_on_one_handle():
-    # the single-launch pass (rows in shared memory) and the two-pass kernels
-    # share the handle's epoch; outlier sets must not leak between them
+    # the single-launch pass with rows held (M = 2048, 3000) and streamed
+    # (M = 4096) in shared memory: generation-parity state and outlier sets
+    # must not leak between calls
     K, N = 5120, 512
     W = workloads.weight(K, N, 41)
     w = m.int8mm_prepare_weight(torch.from_numpy(W).to(dev()))
@@ -268,8 +272,10 @@ def test_launches_per_forward():
     w = m.int8mm_prepare_weight(W)
     assert m.int8mm_launches_per_forward(w, 0) == 0
     assert m.int8mm_launches_per_forward(w, 1) == 2       # single-cluster activation pass + decode GEMM
-    assert m.int8mm_launches_per_forward(w, 2048) == 2    # rows fit in shared memory
-    assert m.int8mm_launches_per_forward(w, 4096) == 3    # two activation kernels
+    assert m.int8mm_launches_per_forward(w, 2048) == 2    # rows held in shared memory
+    assert m.int8mm_launches_per_forward(w, 4096) == 2    # rows streamed through it
+    w2 = m.int8mm_prepare_weight(torch.from_numpy(workloads.weight(40960, 256, 44)).to(dev()))
+    assert m.int8mm_launches_per_forward(w2, 2048) == 3   # K > 32768: two activation kernels
     with pytest.raises(m.Int8mmError):
         m.int8mm_launches_per_forward(w, -1)
 
@@ -383,11 +389,11 @@ def test_opt13b_prefill_full_size():
 
 def test_opt13b_ffn_contraction_full_size():
     # the FFN's second layer (K = 20480 > N = 5120): the activation (84 MB)
-    # exceeds the SMs' shared memory, so the two-kernel activation path runs
+    # exceeds the SMs' shared memory and is streamed through it twice
     p = workloads.opt13b_contraction()
     W = torch.from_numpy(p.W).to(dev())
     w = m.int8mm_prepare_weight(W)
-    assert m.int8mm_launches_per_forward(w, p.X.shape[0]) == 3
+    assert m.int8mm_launches_per_forward(w, p.X.shape[0]) == 2
     out = check(p, w=w, rows=sample_rows(p.X.shape[0], 16, seed=2))
     assert out["cnt"] == 7
     m.int8mm_free(w)
