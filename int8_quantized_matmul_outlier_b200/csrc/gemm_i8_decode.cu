@@ -26,7 +26,8 @@
 // Warps: 0 TMA producer (weight tile + token tile per stage, 6-deep ring,
 // weight loads marked evict-first in L2; the first weight tiles are issued
 // before waiting on the activation pass), 1 MMA issuer and TMEM owner (double-buffered 128 x MP int32
-// accumulator), 2-5 epilogue (one output column n per thread, all tokens).
+// accumulator), 2-9 epilogue (one output column n per thread, half of the
+// tokens: two warps share each TMEM lane quarter).
 // Every wait is bounded; a timeout sets the status word and the CTA exits.
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -42,7 +43,8 @@ constexpr int DBK = 128;  // K bytes per stage
 // rings (4: slower, 11: 12% slower): more outstanding reads only congest HBM.
 constexpr int D_STAGES = 6;
 constexpr int D_OUT_STAGE = 64;  // outliers whose activations are staged in smem
-constexpr int D_THREADS = 192;
+constexpr int D_EPI = 256;  // epilogue threads: eight warps
+constexpr int D_THREADS = 64 + D_EPI;
 
 template <int MP>
 struct DCfg {
@@ -58,7 +60,7 @@ struct DCfg {
   static constexpr int IDX_OFF = RX_OFF + 64 * 4;                  // int [D_OUT_STAGE]
   static constexpr int SMEM = IDX_OFF + D_OUT_STAGE * 4 + 1024;
   // outlier weight values prefetched into registers per segment
-  static constexpr int WCAP = MP == 64 ? 8 : 16;
+  static constexpr int WCAP = 16;
   static constexpr int TMEM_COLS = 2 * MP < 32 ? 32 : 2 * MP;
   static constexpr uint32_t IDESC = idesc_i8(DBM, MP);
   static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned for the 128B swizzle");
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(D_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], D_EPI / 32);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -237,22 +239,26 @@ __global__ void __launch_bounds__(D_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may read
+    // Two warps per TMEM lane quarter (warp w may read lanes 32 (w % 4) ..):
+    // warps 2-5 take tokens [0, HM), warps 6-9 tokens [HM, MP).
+    constexpr int HM = MP / 2;
+    const int q = warp & 3;
+    const int m0 = ((warp - 2) >> 2) * HM;
     const int n_local = q * 32 + lane;
-    const int et = threadIdx.x - 64;  // 0..127
+    const int et = threadIdx.x - 64;  // 0 .. D_EPI-1
     dpdl_wait();  // count, idx, X_OT and c_x come from the activation pass
     const int cnt = *a.count;
     const int cs = min(cnt, D_OUT_STAGE);
-    for (int e = et; e < cs * M; e += 128) {
+    for (int e = et; e < cs * M; e += D_EPI) {
       const int o = e / M, m = e % M;
       xo_s[o * 64 + m] = a.X_OT[static_cast<size_t>(o) * M + m];
     }
-    for (int o = et; o < cs; o += 128) idx_s[o] = a.idx[o];
+    for (int o = et; o < cs; o += D_EPI) idx_s[o] = a.idx[o];
     if (et < M) {
       const float c = a.c_x[et];
       rx_s[et] = c == 0.0f ? 0.0f : __frcp_rn(c);
     }
-    dbar_sync(1, 128);
+    dbar_sync(1, D_EPI);
     int lt = 0;
     for (long long u = u_begin; u < u_end; ++lt) {
       const Seg sg = segment_at(u, u_end, num_kb);
@@ -267,18 +273,23 @@ __global__ void __launch_bounds__(D_THREADS, 1)
 #pragma unroll
       for (int o = 0; o < C::WCAP; ++o)
         wo[o] = (o < cs && n_ok) ? __half2float(a.W[static_cast<size_t>(idx_s[o]) * N + n]) : 0.0f;
-      // all lanes wait; the decision to go on is then made once for all 4 warps
+      // all lanes wait; the decision to go on is then made once for all warps
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], use & 1u, tmo, abort_flag));
       if (!ok && lane == 0) dfail(a, abort_flag);
-      dbar_sync(1, 128);
+      dbar_sync(1, D_EPI);
       if (et == 0) *s_flag = *abort_flag ? 0 : 1;
-      dbar_sync(1, 128);
+      dbar_sync(1, D_EPI);
       if (!*s_flag) continue;
       tc_fence_after();
-      uint32_t r[MP];
-      const uint32_t t = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * MP);
+      uint32_t r[HM];
+      const uint32_t t =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * MP + m0);
+      if constexpr (HM >= 16) {
 #pragma unroll
-      for (int j = 0; j < MP / 16; ++j) tmem_ld_32x32b_x16(t + 16 * j, r + 16 * j);
+        for (int j = 0; j < HM / 16; ++j) tmem_ld_32x32b_x16(t + 16 * j, r + 16 * j);
+      } else {
+        tmem_ld_32x32b_x8(t, r);
+      }
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -289,11 +300,11 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         // count the k steps for the block's owner
         if (n_ok) {
 #pragma unroll
-          for (int m = 0; m < MP; ++m)
-            if (m < M) atomicAdd(a.part + static_cast<size_t>(m) * N + n, static_cast<int>(r[m]));
+          for (int j = 0; j < HM; ++j)
+            if (m0 + j < M) atomicAdd(a.part + static_cast<size_t>(m0 + j) * N + n, static_cast<int>(r[j]));
         }
         __threadfence();
-        dbar_sync(1, 128);
+        dbar_sync(1, D_EPI);
         if (et == 0) atomicAdd(a.ticket + sg.nb, static_cast<unsigned>(sg.kb1 - sg.kb0));
         continue;
       }
@@ -315,21 +326,22 @@ __global__ void __launch_bounds__(D_THREADS, 1)
           if (!got) dfail(a, abort_flag);
           *s_flag = got;
         }
-        dbar_sync(1, 128);
+        dbar_sync(1, D_EPI);
         const int got = *s_flag;
-        dbar_sync(1, 128);  // s_flag is reused by the next segment
+        dbar_sync(1, D_EPI);  // s_flag is reused by the next segment
         if (!got) continue;
         if (n_ok) {
           // all loads first: a store between them would serialise the round
           // trips (the compiler cannot tell the addresses apart)
-          int32_t v[MP];
+          int32_t v[HM];
 #pragma unroll
-          for (int m = 0; m < MP; ++m) v[m] = m < M ? __ldcg(a.part + static_cast<size_t>(m) * N + n) : 0;
+          for (int j = 0; j < HM; ++j)
+            v[j] = m0 + j < M ? __ldcg(a.part + static_cast<size_t>(m0 + j) * N + n) : 0;
 #pragma unroll
-          for (int m = 0; m < MP; ++m)
-            if (m < M) a.part[static_cast<size_t>(m) * N + n] = 0;
+          for (int j = 0; j < HM; ++j)
+            if (m0 + j < M) a.part[static_cast<size_t>(m0 + j) * N + n] = 0;
 #pragma unroll
-          for (int m = 0; m < MP; ++m) r[m] = static_cast<uint32_t>(static_cast<int>(r[m]) + v[m]);
+          for (int j = 0; j < HM; ++j) r[j] = static_cast<uint32_t>(static_cast<int>(r[j]) + v[j]);
         }
         if (et == 0) a.ticket[sg.nb] = 0u;
       }
@@ -337,35 +349,36 @@ __global__ void __launch_bounds__(D_THREADS, 1)
       // dequantise, add the fp16 outlier product, write fp16 (coalesced over n)
       const float rw = __ldg(a.inv_cw + n);
       const float bn = a.bias != nullptr ? __half2float(a.bias[n]) : 0.0f;
-      float y[MP];
+      float y[HM];
 #pragma unroll
-      for (int m = 0; m < MP; ++m)
-        y[m] = m < M ? __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[m])), rx_s[m]), rw), bn)
-                     : 0.0f;
+      for (int j = 0; j < HM; ++j)
+        y[j] = m0 + j < M
+                   ? __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), rx_s[m0 + j]), rw), bn)
+                   : 0.0f;
 #pragma unroll
       for (int o = 0; o < C::WCAP; ++o)
         if (o < cs) {
 #pragma unroll
-          for (int m = 0; m < MP; ++m)
-            if (m < M) y[m] = __fmaf_rn(__half2float(xo_s[o * 64 + m]), wo[o], y[m]);
+          for (int j = 0; j < HM; ++j)
+            if (m0 + j < M) y[j] = __fmaf_rn(__half2float(xo_s[o * 64 + m0 + j]), wo[o], y[j]);
         }
       for (int o = C::WCAP; o < cnt; ++o) {
         const float w1 = __half2float(a.W[static_cast<size_t>(__ldg(a.idx + o)) * N + n]);
 #pragma unroll
-        for (int m = 0; m < MP; ++m)
-          if (m < M) {
-            const float xo = o < cs ? __half2float(xo_s[o * 64 + m])
-                                    : __half2float(a.X_OT[static_cast<size_t>(o) * M + m]);
-            y[m] = __fmaf_rn(xo, w1, y[m]);
+        for (int j = 0; j < HM; ++j)
+          if (m0 + j < M) {
+            const float xo = o < cs ? __half2float(xo_s[o * 64 + m0 + j])
+                                    : __half2float(a.X_OT[static_cast<size_t>(o) * M + m0 + j]);
+            y[j] = __fmaf_rn(xo, w1, y[j]);
           }
       }
 #pragma unroll
-      for (int m = 0; m < MP; ++m)
-        if (m < M) a.Y[static_cast<size_t>(m) * N + n] = __float2half_rn(y[m]);
+      for (int j = 0; j < HM; ++j)
+        if (m0 + j < M) a.Y[static_cast<size_t>(m0 + j) * N + n] = __float2half_rn(y[j]);
       if (a.acc_dump != nullptr) {
 #pragma unroll
-        for (int m = 0; m < MP; ++m)
-          if (m < M) a.acc_dump[static_cast<size_t>(m) * N + n] = static_cast<int32_t>(r[m]);
+        for (int j = 0; j < HM; ++j)
+          if (m0 + j < M) a.acc_dump[static_cast<size_t>(m0 + j) * N + n] = static_cast<int32_t>(r[j]);
       }
     }
   }
