@@ -174,6 +174,18 @@ int8mm_status int8mm_get_status(int8mm_weight_t h);
  */
 int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns);
 
+/*
+ * Split of the prefill GEMM along K (forwards with M > 128, whose 256 x 256
+ * output tiles are computed by pairs of SMs).  0 (the default) lets the
+ * library choose: it cuts each tile's K range into the S in 1..4 pieces that
+ * best fill the pairs' rounds of work (K-heavy shapes with few tiles, such
+ * as an FFN contraction, get S > 1).  1..4 forces S (capped at the number of
+ * 128-deep k-blocks).  Piece sums are exact int32, so every S gives the
+ * same results.  With S > 1 the handle holds a workspace of (S-1) x 256 KB
+ * per tile.  INT8MM_ERR_INVALID_ARG for a value outside 0..4.
+ */
+int8mm_status int8mm_set_split_k(int8mm_weight_t h, int split);
+
 /* Device bytes held by the handle (codes, scales, workspace). */
 int8mm_status int8mm_weight_bytes(int8mm_weight_t h, size_t* bytes);
 

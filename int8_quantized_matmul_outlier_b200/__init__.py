@@ -44,6 +44,7 @@ SIGNATURES = {
     "int8mm_forward_debug": (_ST, [_P, _P, _I64, ctypes.c_float, _P, _P, _P]),
     "int8mm_get_status": (_ST, [_P]),
     "int8mm_set_wait_limit": (_ST, [_P, ctypes.c_uint64]),
+    "int8mm_set_split_k": (_ST, [_P, ctypes.c_int]),
     "int8mm_weight_bytes": (_ST, [_P, ctypes.POINTER(ctypes.c_size_t)]),
     "int8mm_launches_per_forward": (_ST, [_P, _I64, ctypes.POINTER(ctypes.c_int)]),
     "int8mm_free": (None, [_P]),
@@ -251,6 +252,11 @@ def int8mm_get_status(w: Weight) -> int:
 
 def int8mm_set_wait_limit(w: Weight, timeout_ns: int) -> None:
     _check(lib().int8mm_set_wait_limit(w.handle, int(timeout_ns)))
+
+
+def int8mm_set_split_k(w: Weight, split: int) -> None:
+    """Pieces along K per prefill GEMM tile: 0 automatic, 1..4 forced."""
+    _check(lib().int8mm_set_split_k(w.handle, int(split)))
 
 
 def int8mm_weight_bytes(w: Weight) -> int:

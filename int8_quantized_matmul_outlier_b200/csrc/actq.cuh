@@ -2,7 +2,8 @@
 // magnitude maxima, the scale c = 127/absmax, round-to-nearest-even int8
 // codes, programmatic-dependent-launch controls, and the few memory
 // operations the single-launch activation pass needs (bulk copies into shared
-// memory, release flags; the acquire load is in ptx.cuh).
+// memory, release stores; the acquire load and the release add are in
+// ptx.cuh).
 //
 // Method: "LLM.int8() — 大模型激活值里藏着几个超大异常通道", 方法1 (one scale
 // per row of X and per column of W, c = 127/absmax, codes rounded to int8).
@@ -116,11 +117,6 @@ __device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gsrc, u
 
 __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Atomic add with release semantics at GPU scope, no result returned.
-__device__ __forceinline__ void red_release_add_gpu(uint32_t* p, uint32_t v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 }  // namespace i8mm

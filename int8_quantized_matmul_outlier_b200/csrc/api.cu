@@ -34,6 +34,12 @@ struct int8mm_weight {
   // decode (M <= 64) scratch: int32 partial sums and per-n-block tickets
   int32_t* part = nullptr;
   unsigned* dticket = nullptr;
+  // prefill split-K scratch: partial tiles and per-(tile, CTA, half) tickets
+  int split_override = 0;        // 0: automatic
+  int32_t* sk_ws = nullptr;
+  size_t sk_ws_elems = 0;
+  uint32_t* sk_ticket = nullptr;
+  size_t sk_ticket_n = 0;
   // fixed-size scratch of the outlier pass
   unsigned long long* colkey = nullptr;  // [K]
   unsigned long long* epoch = nullptr;   // [1]
@@ -154,6 +160,8 @@ void free_all(int8mm_weight* h) {
   release(&h->dY);
   release(&h->part);
   release(&h->dticket);
+  release(&h->sk_ws);
+  release(&h->sk_ticket);
   release(&h->Wb);
   release(&h->c_w);
   release(&h->inv_cw);
@@ -326,6 +334,47 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     if ((e = launch_gemm_decode(h->tmW128, h->tmA, d, h->num_sms, pdl, s)) != cudaSuccess)
       return cuda_fail(e, "int8 decode GEMM launch");
   } else {
+    // split K for the CTA-pair tiles; the scratch grows on demand
+    int split = 1;
+    if (M > kGemmBM) {
+      const int64_t num_kb = (h->K + kGemmBK - 1) / kGemmBK;
+      split = h->split_override > 0 ? static_cast<int>(std::min<int64_t>(h->split_override, num_kb))
+                                    : gemm_split_for(M, h->N, h->K, h->num_sms);
+    }
+    if (split > 1) {
+      const size_t tiles = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM)) *
+                           static_cast<size_t>((h->N + kGemmBN - 1) / kGemmBN);
+      const size_t ws = static_cast<size_t>(split - 1) * tiles * 2 * kGemmBM * kGemmBN;
+      if (ws > h->sk_ws_elems) {
+        if (h->sk_ws) {
+          cudaFreeAsync(h->sk_ws, s);
+          h->bytes -= h->sk_ws_elems * 4;
+          h->sk_ws = nullptr;
+          h->sk_ws_elems = 0;
+        }
+        if ((e = alloc(&h->sk_ws, ws, s, &h->bytes)) != cudaSuccess) {
+          cudaStreamSynchronize(s);
+          release(&h->sk_ws);
+          return cuda_fail(e, "split-K workspace allocation");
+        }
+        h->sk_ws_elems = ws;
+      }
+      if (tiles * 4 > h->sk_ticket_n) {
+        if (h->sk_ticket) {
+          cudaFreeAsync(h->sk_ticket, s);
+          h->bytes -= h->sk_ticket_n * 4;
+          h->sk_ticket = nullptr;
+          h->sk_ticket_n = 0;
+        }
+        if ((e = alloc(&h->sk_ticket, tiles * 4, s, &h->bytes)) != cudaSuccess ||
+            (e = cudaMemsetAsync(h->sk_ticket, 0, tiles * 16, s)) != cudaSuccess) {
+          cudaStreamSynchronize(s);
+          release(&h->sk_ticket);
+          return cuda_fail(e, "split-K ticket allocation");
+        }
+        h->sk_ticket_n = tiles * 4;
+      }
+    }
     GemmArgs a;
     a.M = static_cast<int>(M);
     a.N = static_cast<int>(h->N);
@@ -340,6 +389,9 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     a.Y = static_cast<__half*>(Y);
     a.bias = static_cast<const __half*>(bias);
     a.acc_dump = dbg ? dbg->acc : nullptr;
+    a.split = split;
+    a.sk_ws = h->sk_ws;
+    a.sk_ticket = h->sk_ticket;
     a.status = h->status;
     a.timeout_ns = h->timeout_ns;
     if ((e = launch_gemm_decomp(h->tmA, h->tmB, h->tmW128, a, h->num_sms, pdl, s)) != cudaSuccess)
@@ -539,6 +591,8 @@ int8mm_status int8mm_get_status(int8mm_weight_t h) {
     // an aborted decode GEMM may leave partial sums and tickets behind,
     if (h->part) cudaMemset(h->part, 0, static_cast<size_t>(kDecodeMaxM) * h->N * 4);
     if (h->dticket) cudaMemset(h->dticket, 0, static_cast<size_t>((h->N + 127) / 128) * 4);
+    // an aborted split-K GEMM its tile tickets,
+    if (h->sk_ticket) cudaMemset(h->sk_ticket, 0, h->sk_ticket_n * 4);
     // and an aborted single-launch activation pass its barrier counts and bitmasks
     cudaMemset(h->xsync, 0, 16);
     cudaMemset(h->omask, 0, static_cast<size_t>((h->K + 31) / 32) * 8);
@@ -552,6 +606,13 @@ int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns) {
   if (!live(h)) return fail(INT8MM_ERR_INVALID_ARG, "invalid or freed weight handle");
   if (timeout_ns == 0) return fail(INT8MM_ERR_INVALID_ARG, "timeout must be positive");
   h->timeout_ns = timeout_ns;
+  return INT8MM_OK;
+}
+
+int8mm_status int8mm_set_split_k(int8mm_weight_t h, int split) {
+  if (!live(h)) return fail(INT8MM_ERR_INVALID_ARG, "invalid or freed weight handle");
+  if (split < 0 || split > kGemmMaxSplit) return fail(INT8MM_ERR_INVALID_ARG, "split %d outside 0..%d", split, kGemmMaxSplit);
+  h->split_override = split;
   return INT8MM_OK;
 }
 

@@ -45,6 +45,22 @@
 // its own TMEM and writes them; commits reach both CTAs' barriers.  Each SM
 // then streams 32 KB instead of 48 KB per 128x256x128 of MMA work, in a
 // 6-stage ring.  No TMA multicast is used.
+//
+// Split K (CTA pairs, when the tiles fill the pairs' rounds badly, e.g. 160
+// tiles of a K-heavy FFN contraction for 74 pairs): every tile is cut into S
+// equal ranges of k-blocks, and the S x tiles work units are dealt to the
+// pairs piece-major (all first pieces, then all second pieces, ...), so the
+// pairs of one round read the same k-slices and keep sharing them in L2.
+// The last piece owns the tile.  The other pieces store their exact int32
+// partial tiles in a workspace and count themselves on the tile's tickets
+// (one per CTA and 128-column half); the owner waits (bounded) for its
+// ticket to show the S-1 pieces, adds the partials to its accumulator before
+// dequantising, resets the ticket and finishes the tile as an unsplit one.
+// A pair deals with all its non-owner units before any owner unit, and
+// non-owner units wait on nothing, so every wait ends once all pairs are
+// resident (one pair per two SMs, as for the unsplit kernel; the wait is
+// bounded all the same).
+// Integer sums make the result independent of the split.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -112,6 +128,18 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// A named barrier over nthreads threads that also returns whether v holds
+// on all of them.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n bar.red.and.pred p, %2, %3, q;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ float dequant(uint32_t acc, float rx, float rw) {
   return __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(acc)), rx), rw);
 }
@@ -137,12 +165,29 @@ __device__ __forceinline__ void load_bias32(const __half* bias, int n, bool full
   }
 }
 
-// BIAS: the layer bias is added (a separate instantiation, so that the
-// common bias-free path carries none of its code).
-template <bool PAIR, bool BIAS>
+// One work unit: k-blocks [kb0, kb1) of a tile; piece S-1 finishes the tile.
+struct Unit {
+  int tile, piece, kb0, kb1;
+};
+
+template <bool SPLIT>
+__device__ __forceinline__ Unit unit_at(int u, int num_tiles, int num_kb, int split) {
+  if (!SPLIT) return Unit{u, 0, 0, num_kb};
+  Unit w;
+  w.piece = u / num_tiles;
+  w.tile = u - w.piece * num_tiles;
+  w.kb0 = w.piece * num_kb / split;
+  w.kb1 = (w.piece + 1) * num_kb / split;
+  return w;
+}
+
+// BIAS: the layer bias is added; SPLIT: split K (CTA pairs only).  Separate
+// instantiations, so that the common path carries none of their code.
+template <bool PAIR, bool BIAS, bool SPLIT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_decomp_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const GemmArgs a) {
+  static_assert(PAIR || !SPLIT, "split K is implemented for CTA pairs");
   using C = Cfg<PAIR>;
   constexpr int STAGES = C::STAGES;
   constexpr int STAGE_BYTES = C::STAGE_BYTES;
@@ -157,6 +202,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* tout = tdeq + 2;   // [2] outlier product added
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFFSET);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFFSET + 4);
+  volatile int* part_ok = reinterpret_cast<volatile int*>(smem + C::MISC_OFFSET + 8);  // [2] per half
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = a.M, N = a.N, K = a.K;
@@ -168,6 +214,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int num_n = (N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = (K + BK - 1) / BK;
+  const int S = SPLIT ? a.split : 1;  // pieces per tile
+  const int num_units = num_tiles * S;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -231,22 +279,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // The weight tiles of the first k-blocks do not depend on the
       // activation pass: issue them before waiting for it, then the
       // matching activation tiles (all stages start empty).
-      const int first = tile0;
-      const int pre = first < num_tiles ? min(STAGES, num_kb) : 0;
-      for (int kb = 0; kb < pre; ++kb) {
-        expect(kb);
-        load_b(kb, kb, first / num_m);
+      const Unit first = unit_at<SPLIT>(tile0, num_tiles, num_kb, S);
+      const int pre = tile0 < num_units ? min(STAGES, first.kb1 - first.kb0) : 0;
+      for (int i = 0; i < pre; ++i) {
+        expect(i);
+        load_b(i, first.kb0 + i, first.tile / num_m);
       }
       pdl_wait();
-      for (int kb = 0; kb < pre; ++kb) {
-        load_a(kb, kb, first % num_m);
-        issued_mask |= 1u << kb;
+      for (int i = 0; i < pre; ++i) {
+        load_a(i, first.kb0 + i, first.tile % num_m);
+        issued_mask |= 1u << i;
       }
       stage = pre % STAGES;
       phase = pre == STAGES ? 1u : 0u;
-      for (int tile = tile0; tile < num_tiles && ok; tile += tstride) {
-        const int m_blk = tile % num_m, n_blk = tile / num_m;
-        for (int kb = tile == first ? pre : 0; kb < num_kb; ++kb) {
+      for (int u = tile0; u < num_units && ok; u += tstride) {
+        const Unit w = unit_at<SPLIT>(u, num_tiles, num_kb, S);
+        const int m_blk = w.tile % num_m, n_blk = w.tile / num_m;
+        for (int kb = w.kb0 + (u == tile0 ? pre : 0); kb < w.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
             ok = false;
             break;
@@ -291,6 +340,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int cnt = PAIR ? *a.count : 0;
       const int nk = cnt > 0 ? (min(cnt, kOutMma) + 15) / 16 : 0;
       uint32_t pend_use = 0;
+      // with split K, tdeq/tout complete only for units that finish a tile:
+      // their phases count those uses of each buffer
+      uint32_t fin_uses[2] = {0u, 0u};
       int pend = -1;  // accumulator buffer whose outlier product is due
       auto issue_outl = [&]() -> bool {
         if (!mbar_wait(&tdeq[pend], pend_use & 1u, tmo, abort_flag)) return false;
@@ -305,7 +357,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         pend = -1;
         return true;
       };
-      for (int tile = tile0; tile < num_tiles && ok; tile += tstride, ++lt) {
+      for (int u = tile0; u < num_units && ok; u += tstride, ++lt) {
+        const Unit w = unit_at<SPLIT>(u, num_tiles, num_kb, S);
         const int buf = lt & 1;
         const uint32_t use = static_cast<uint32_t>(lt >> 1);
         if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, tmo, abort_flag)) {
@@ -323,7 +376,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
             // advance 32 bytes along K inside the 128-byte swizzled row
-            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            const uint32_t acc = (kb != w.kb0 || kk != 0) ? 1u : 0u;
             if (PAIR)
               mma_i8_pair(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2),
                           C::IDESC, acc);
@@ -339,17 +392,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           return true;
         };
-        const int ksplit = pend >= 0 ? min(num_kb, OUT_ISSUE_KB) : num_kb;
-        for (int kb = 0; kb < ksplit && ok; ++kb) ok = kblock(kb);
+        const int ksplit = pend >= 0 ? min(w.kb1, w.kb0 + OUT_ISSUE_KB) : w.kb1;
+        for (int kb = w.kb0; kb < ksplit && ok; ++kb) ok = kblock(kb);
         if (ok && pend >= 0) ok = issue_outl();
-        for (int kb = ksplit; kb < num_kb && ok; ++kb) ok = kblock(kb);
+        for (int kb = ksplit; kb < w.kb1 && ok; ++kb) ok = kblock(kb);
         if (ok) {
           if (PAIR) mma_commit_pair(&tfull[buf], 0x3);
           else mma_commit(&tfull[buf]);
         }
-        if (nk > 0) {
+        if (nk > 0 && w.piece == S - 1) {  // the tile is complete: its outlier product is due
           pend = buf;
-          pend_use = use;
+          pend_use = SPLIT ? fin_uses[buf]++ : use;
         }
       }
       if (ok && pend >= 0) ok = issue_outl();
@@ -381,10 +434,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const bool y32 = (reinterpret_cast<uintptr_t>(a.Y) & 31u) == 0;
     bool alive = true;
     int lt = 0;
-    for (int tile = tile0; tile < num_tiles; tile += tstride, ++lt) {
+    uint32_t fin_uses[2] = {0u, 0u};  // units that finished a tile, per accumulator buffer
+    for (int u = tile0; u < num_units; u += tstride, ++lt) {
+      const Unit w = unit_at<SPLIT>(u, num_tiles, num_kb, S);
+      const int tile = w.tile;
       const int m_blk = tile % num_m, n_blk = tile / num_m;
+      // a unit that finishes its tile (always, without split K); the others
+      // only hand their partial sums on
+      const bool fin = !SPLIT || w.piece == S - 1;
+      const bool outl_u = outl && fin;
       const int buf = lt & 1;
       const uint32_t use = static_cast<uint32_t>(lt >> 1);
+      uint32_t fuse = use;  // phase of this buffer's tout barrier
+      if (SPLIT && fin) fuse = fin_uses[buf]++;
       const int nh = n_blk * BN + h * HALF_N;  // first column of this half
       const int m = m_blk * C::TILE_M + static_cast<int>(rank) * BM + row_t;
       const bool row_ok = m < M;
@@ -392,7 +454,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // (1) stage this tile's scales and outlier weight rows; this runs
       //     while the tensor cores still accumulate the tile.
       named_bar_sync(bar_id, 128);  // readers of the previous tile are done
-      if (tl < HALF_N / 4) {
+      if (fin && tl < HALF_N / 4) {
         const int n = nh + tl * 4;
         const float4 f = n < N ? __ldg(reinterpret_cast<const float4*>(a.inv_cw + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
         reinterpret_cast<float4*>(rws)[tl] = f;
@@ -413,7 +475,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int o = 0; o < OUT_CAP; ++o)
         xo[o] = (o < cs && row_ok) ? __half2float(a.X_OT[static_cast<size_t>(o) * M + m]) : 0.0f;
-      if (outl) {
+      if (outl_u) {
         // this tile's outlier-product operand blocks, as fp16 rows of the
         // 128-byte-swizzled K-major layout (16-byte chunk c of row r stored at
         // chunk c ^ (r % 8), groups of 8 rows 1024 bytes apart): half 0 writes
@@ -448,6 +510,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float c = a.c_x[m];
         rx = c == 0.0f ? 0.0f : __frcp_rn(c);
       }
+      if (SPLIT && fin && h == 0 && tl == 0) {
+        // the other pieces' partial tiles (normally stored long before): pull
+        // them into L2 while the tensor cores finish this piece
+        for (int p = 0; p < S - 1; ++p)
+          bulk_prefetch_l2(a.sk_ws + ((static_cast<size_t>(p) * num_tiles + tile) * 2 + rank) * (BM * BN),
+                           BM * BN * 4);
+      }
       named_bar_sync(bar_id, 128);  // staging visible to the half's 4 warps
 
       // (2) wait for the accumulator (all lanes; the vote keeps the warp
@@ -457,11 +526,86 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         alive = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], use & 1u, tmo, abort_flag));
         if (!alive && lane == 0) fail(a, abort_flag);
       }
+      // with split K more named barriers follow: the half's warps decide together
+      if (SPLIT) alive = named_bar_and(bar_id, 128, alive);
       if (!alive) continue;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(buf * BN + h * HALF_N);
-      if (outl) {
+      // piece p's partial sums of this thread's 32-column chunk ch, as 8
+      // int4: the workspace holds [piece][tile][CTA rank][half][chunk][int4
+      // t4][row] so that a warp's access is 512 contiguous bytes
+      auto part_at = [&](int p, int ch) {
+        return reinterpret_cast<int4*>(a.sk_ws + ((static_cast<size_t>(p) * num_tiles + tile) * 2 + rank) * (BM * BN)) +
+               (h * (HALF_N / 32) + ch) * 8 * BM + row_t;
+      };
+      uint32_t* ticket = SPLIT ? a.sk_ticket + (static_cast<size_t>(tile) * 2 + rank) * 2 + h : nullptr;
+      if (SPLIT && !fin) {
+        // a piece that does not finish the tile: store the partial sums,
+        // then count this half on the owner's ticket
+#pragma unroll 1
+        for (int ch = 0; ch < HALF_N / 32; ++ch) {
+          const int cl = ch * 32;
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(cl), r);
+          tmem_wait_ld();
+          if (ch == HALF_N / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+          }
+          int4* pp = part_at(w.piece, ch);
+#pragma unroll
+          for (int t4 = 0; t4 < 8; ++t4)
+            pp[t4 * BM] = make_int4(static_cast<int>(r[4 * t4]), static_cast<int>(r[4 * t4 + 1]),
+                                    static_cast<int>(r[4 * t4 + 2]), static_cast<int>(r[4 * t4 + 3]));
+        }
+        __threadfence();
+        named_bar_sync(bar_id, 128);
+        if (tl == 0) red_release_add_gpu(ticket, 1u);
+        continue;
+      }
+      if (SPLIT) {
+        // the owner: wait until the other S-1 pieces of this half are stored
+        if (tl == 0) {
+          const uint32_t need = static_cast<uint32_t>(S - 1);
+          int got = 1;
+          if (ld_acquire_gpu_u32(ticket) != need) {
+            const uint64_t t0 = global_timer_ns();
+            for (uint32_t it = 1; ld_acquire_gpu_u32(ticket) != need; ++it) {
+              if ((it & 15u) == 0 && (*abort_flag || global_timer_ns() - t0 > tmo)) {
+                got = 0;
+                break;
+              }
+            }
+          }
+          if (got) *ticket = 0u;  // ready for the next launch
+          else fail(a, abort_flag);
+          part_ok[h] = got;
+        }
+        named_bar_sync(bar_id, 128);
+        if (!part_ok[h]) {  // the next unit's first barrier orders the reuse of part_ok
+          alive = false;
+          continue;
+        }
+      }
+      // adds the other pieces' partial sums to the 32 accumulator columns of chunk ch
+      auto add_parts = [&](uint32_t(&r)[32], int ch) {
+        for (int p = 0; p < S - 1; ++p) {
+          const int4* pp = part_at(p, ch);
+          int4 v[8];
+#pragma unroll
+          for (int t4 = 0; t4 < 8; ++t4) v[t4] = __ldcg(pp + t4 * BM);
+#pragma unroll
+          for (int t4 = 0; t4 < 8; ++t4) {
+            r[4 * t4 + 0] += static_cast<uint32_t>(v[t4].x);
+            r[4 * t4 + 1] += static_cast<uint32_t>(v[t4].y);
+            r[4 * t4 + 2] += static_cast<uint32_t>(v[t4].z);
+            r[4 * t4 + 3] += static_cast<uint32_t>(v[t4].w);
+          }
+        }
+      };
+      if (outl_u) {
         // (3) dequantise in place (int32 -> fp32 in TMEM), hand the tile to
         //     the MMA warp for the outlier product, and wait for it
 #pragma unroll 1
@@ -470,6 +614,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(cl), r);
           tmem_wait_ld();
+          if (SPLIT) add_parts(r, ch);
           const int n = nh + cl;
           if (a.acc_dump != nullptr && row_ok && n < N) {
             uint4* ap = reinterpret_cast<uint4*>(a.acc_dump + static_cast<size_t>(m) * N + n);
@@ -505,7 +650,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tdeq[buf]), 0));  // the leader's barrier
-        alive = __all_sync(0xffffffffu, mbar_wait(&tout[buf], use & 1u, tmo, abort_flag));
+        alive = __all_sync(0xffffffffu, mbar_wait(&tout[buf], fuse & 1u, tmo, abort_flag));
         if (!alive) {
           if (lane == 0) fail(a, abort_flag);
           continue;
@@ -528,9 +673,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const int n = nh + cl;
         if (n >= N) continue;  // warp-uniform
+        if (SPLIT && !outl_u) add_parts(r, ch);
         const bool full32 = n + 32 <= N;
         float v[32];
-        if (outl) {  // already dequantised, outlier product included
+        if (outl_u) {  // already dequantised, outlier product included
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
         } else {
@@ -603,7 +749,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               yp[3] = out[3];
             }
           }
-          if (a.acc_dump != nullptr && !outl) {
+          if (a.acc_dump != nullptr && !outl_u) {
             uint4* ap = reinterpret_cast<uint4*>(a.acc_dump + static_cast<size_t>(m) * N + n);
 #pragma unroll
             for (int t4 = 0; t4 < 8; ++t4)
@@ -624,28 +770,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <bool PAIR, bool BIAS>
+template <bool PAIR, bool BIAS, bool SPLIT>
 cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms, bool pdl,
                      cudaStream_t stream) {
   using C = Cfg<PAIR>;
+  auto kern = gemm_i8_decomp_kernel<PAIR, BIAS, SPLIT>;
   static unsigned long long attr_set = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   const unsigned long long bit = 1ull << (dev & 63);
-  if (!(attr_set & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_i8_decomp_kernel<PAIR, BIAS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set |= bit;
-  }
-  const int num_tiles = ((a.M + C::TILE_M - 1) / C::TILE_M) * ((a.N + BN - 1) / BN);
-  const int units = PAIR ? num_sms / 2 : num_sms;
-  const int grid = std::max(1, std::min(num_tiles, units)) * (PAIR ? 2 : 1);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = stream;
   cudaLaunchAttribute attrs[2];
   int n = 0;
   if (PAIR) {
@@ -655,27 +789,64 @@ cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmA
     attrs[n].val.clusterDim.z = 1;
     ++n;
   }
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attrs;
+  cfg.numAttrs = n;
+  if (!(attr_set & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set |= bit;
+  }
+  const int num_tiles = ((a.M + C::TILE_M - 1) / C::TILE_M) * ((a.N + BN - 1) / BN);
+  const int units_of_work = num_tiles * (SPLIT ? a.split : 1);
+  // one CTA (pair) per SM (pair of SMs), all resident at once: owners of
+  // split tiles wait on other pairs' pieces
+  const int slots = PAIR ? num_sms / 2 : num_sms;
+  cfg.gridDim = dim3(std::max(1, std::min(units_of_work, slots)) * (PAIR ? 2 : 1));
   if (pdl) {
     attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attrs[n].val.programmaticStreamSerializationAllowed = 1;
     ++n;
   }
-  cfg.attrs = attrs;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, gemm_i8_decomp_kernel<PAIR, BIAS>, tmA, tmB, a);
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
 }
 
 }  // namespace
+
+int gemm_split_for(int64_t M, int64_t N, int64_t K, int num_sms) {
+  if (M <= BM) return 1;  // single CTAs: not split
+  const int64_t tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + BN - 1) / BN);
+  const int64_t pairs = std::max(1, num_sms / 2);
+  const int64_t num_kb = (K + BK - 1) / BK;
+  // time of the slowest pair, in k-blocks: rounds of units x (k-blocks per
+  // unit + a fixed cost per unit of about 16 k-blocks, as measured on a
+  // 2048 x 20480 x 5120 contraction: the pipeline turn-around and the
+  // owner's pass over the partial tiles)
+  auto cost = [&](int64_t s) {
+    const int64_t rounds = (tiles * s + pairs - 1) / pairs;
+    return rounds * ((num_kb + s - 1) / s + 16);
+  };
+  int best = 1;
+  for (int s = 2; s <= kGemmMaxSplit && num_kb / s >= 8; ++s)
+    if (cost(s) < cost(best)) best = s;
+  return best;
+}
 
 cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB256, const CUtensorMap& tmB128,
                                const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
   // one 128-row tile height: single CTAs; taller problems: CTA pairs
   const bool bias = a.bias != nullptr;
   if (a.M <= BM)
-    return bias ? launch_t<false, true>(tmA, tmB256, a, num_sms, pdl, stream)
-                : launch_t<false, false>(tmA, tmB256, a, num_sms, pdl, stream);
-  return bias ? launch_t<true, true>(tmA, tmB128, a, num_sms, pdl, stream)
-              : launch_t<true, false>(tmA, tmB128, a, num_sms, pdl, stream);
+    return bias ? launch_t<false, true, false>(tmA, tmB256, a, num_sms, pdl, stream)
+                : launch_t<false, false, false>(tmA, tmB256, a, num_sms, pdl, stream);
+  if (a.split > 1)
+    return bias ? launch_t<true, true, true>(tmA, tmB128, a, num_sms, pdl, stream)
+                : launch_t<true, false, true>(tmA, tmB128, a, num_sms, pdl, stream);
+  return bias ? launch_t<true, true, false>(tmA, tmB128, a, num_sms, pdl, stream)
+              : launch_t<true, false, false>(tmA, tmB128, a, num_sms, pdl, stream);
 }
 
 }  // namespace i8mm

@@ -72,6 +72,9 @@ struct GemmArgs {
   __half* Y;               // [M,N] fp16 output
   const __half* bias;      // [N] fp16 layer bias added before the rounding, or nullptr
   int32_t* acc_dump;       // [M,N] int32 accumulators, or nullptr
+  int split;               // pieces per tile along K (CTA pairs): 1, or 2 .. kGemmMaxSplit
+  int32_t* sk_ws;          // split > 1: [split-1][tiles][2][128][256] int32 partial tiles
+  uint32_t* sk_ticket;     // split > 1: [tiles][2][2] counters, zero between launches
   int* status;             // device status word
   unsigned long long timeout_ns;
 };
@@ -83,6 +86,11 @@ struct GemmArgs {
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 128;
+constexpr int kGemmMaxSplit = 4;
+// Pieces along K per 256x256 tile of the CTA-pair GEMM for an M x N x K
+// problem (1 for single-CTA tiles): the split that best fills the pairs'
+// rounds of work.
+int gemm_split_for(int64_t M, int64_t N, int64_t K, int num_sms);
 // tmB256 / tmB128 map the weight with 256- and 128-row boxes (the second is
 // used by the CTA-pair mode, for M > 128).  With `pdl`, launched as a
 // programmatic dependent of the activation pass: its prologue and the first

@@ -195,6 +195,56 @@ def test_forward_with_bias(M, K, N, n_out, alpha):
     assert torch.equal(y1, y0)
 
 
+SPLIT_SHAPES = [
+    # M, K, N, planted outliers, alpha, forced pieces along K
+    (300, 1040, 784, 5, 6.0, 2),        # ragged M and N; the owner runs the tensor-core outlier product
+    (257, 2048, 512, 3, math.inf, 3),   # no outliers: the partials join the direct epilogue
+    (513, 4096, 1040, 7, 6.0, 4),       # several tiles per pair, owners waiting on other pairs
+    (130, 384, 256, 2, 6.0, 4),         # three k-blocks: the split is capped at 3
+    (513, 2048, 512, 80, 6.0, 2),       # more than 64 outliers: FMA tail on the owner
+    (1000, 2048, 256, 4, 0.0, 3),       # alpha = 0: the int8 partials are all zero
+]
+
+
+@pytest.mark.parametrize("M,K,N,n_out,alpha,split", SPLIT_SHAPES)
+def test_split_k(M, K, N, n_out, alpha, split):
+    # K split into pieces whose int32 partial tiles the owner adds: the same
+    # accumulators and Y as the unsplit GEMM, bit for bit, over repeats
+    p = workloads.small(M, K, N, n_out, seed=M + 5 * K + N + split, alpha=alpha)
+    w = m.int8mm_prepare_weight(torch.from_numpy(p.W).to(dev()))
+    m.int8mm_set_split_k(w, split)
+    out = check(p, w=w)
+    X = torch.from_numpy(p.X).to(dev())
+    ys = [m.int8mm_forward(w, X, alpha) for _ in range(3)]
+    m.int8mm_set_split_k(w, 1)
+    d1 = m.int8mm_forward_debug(w, X, alpha)
+    torch.cuda.synchronize()
+    assert m.int8mm_get_status(w) == m.INT8MM_OK
+    assert torch.equal(d1["acc"], out["d"]["acc"])
+    for y in [out["d"]["Y"]] + ys:
+        assert torch.equal(y, d1["Y"])
+    m.int8mm_free(w)
+
+
+def test_split_k_with_bias():
+    M, K, N = 300, 2064, 784
+    p = workloads.small(M, K, N, 5, seed=17)
+    b = (np.random.default_rng(5).standard_normal(N) * 0.5).astype(np.float16)
+    w = m.int8mm_prepare_weight(torch.from_numpy(p.W).to(dev()))
+    X, B = torch.from_numpy(p.X).to(dev()), torch.from_numpy(b).to(dev())
+    y1 = m.int8mm_forward_bias(w, X, 6.0, B)
+    m.int8mm_set_split_k(w, 3)
+    y3 = m.int8mm_forward_bias(w, X, 6.0, B)
+    torch.cuda.synchronize()
+    assert m.int8mm_get_status(w) == m.INT8MM_OK
+    r = oracle.decomp_matmul(p.X, p.W, 6.0, bias=b)
+    assert_y_close(y3.cpu().numpy(), r["Y"], p.X, p.W, r["idx"])
+    assert torch.equal(y1, y3)
+    with pytest.raises(RuntimeError):
+        m.int8mm_set_split_k(w, 5)
+    m.int8mm_free(w)
+
+
 def test_linear8bitlt_module():
     torch.manual_seed(0)
     K, N = 1040, 784
