@@ -55,7 +55,9 @@ typedef enum {
   INT8MM_ERR_ALIGNMENT = 3,         /* a pointer not 16-byte aligned */
   INT8MM_ERR_OOM = 4,               /* device allocation failed */
   INT8MM_ERR_CUDA = 5,              /* a CUDA runtime/driver call failed */
-  INT8MM_ERR_TIMEOUT = 6            /* a device wait ran out of time (see get_status) */
+  INT8MM_ERR_TIMEOUT = 6,           /* a device wait ran out of time (see get_status) */
+  INT8MM_ERR_OUTLIER_CAP = 7        /* a forward found more outlier columns than a static
+                                       weight holds (see get_status) */
 } int8mm_status;
 
 /* Shape limits: 16 <= K <= 65536 with K % 16 == 0 (K <= 133144 keeps the
@@ -76,6 +78,36 @@ typedef enum {
  */
 int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N, void* stream,
                                     int8mm_weight_t* out);
+
+/*
+ * Memory-saving variant of int8mm_prepare_weight.  The outlier dimensions are
+ * systematic, a few fixed input dimensions in every layer, and only they need
+ * the fp16 path ("LLM.int8() — 大模型激活值里藏着几个超大异常通道": the
+ * outliers sit in fixed feature dimensions; 方法2: those dimensions go
+ * through fp16, a small fraction of the weight).
+ *
+ * Prepares the int8 codes and scales from W exactly as int8mm_prepare_weight
+ * does, and copies the fp16 rows W[rows[i], :], i < n_rows, into the handle.
+ * `rows` is a host array of distinct input dimensions in [0, K); n_rows may
+ * be 0.  W is NOT borrowed: the call synchronises `stream` before it returns,
+ * after which W may be freed.
+ *
+ * Each forward gathers the weight rows of the outlier columns it found
+ * (one more kernel per forward).  A stored dimension uses its fp16 row.  For
+ * any other outlier column the row is rebuilt from its int8 codes as
+ * fp16(q * (1/c_w)) in fp32; the pages leave this case open.  The fp16
+ * outlier product then uses that quantised row.
+ *
+ * At most `max_outliers` (1..K) outlier columns per forward.  The handle
+ * holds max_outliers x N fp16 for their rows.  A forward that finds more
+ * leaves the product of the columns past that count out of Y, and
+ * int8mm_get_status returns INT8MM_ERR_OUTLIER_CAP.
+ *
+ * Errors: as int8mm_prepare_weight, plus INT8MM_ERR_INVALID_ARG for bad
+ * rows, n_rows or max_outliers.
+ */
+int8mm_status int8mm_prepare_weight_static(const void* W_fp16_dev, int64_t K, int64_t N, const int32_t* rows,
+                                           int64_t n_rows, int max_outliers, void* stream, int8mm_weight_t* out);
 
 /*
  * Pre-size the per-forward workspace for up to M_max rows, so that later
@@ -99,7 +131,8 @@ int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream);
  * fused int8 GEMM, a programmatic dependent launch that starts while the
  * activation pass finishes.  The activation pass is one kernel when X fits
  * in the GPU's shared memory (rows split evenly over one block per SM, K <=
- * 32768) or M <= 64, else two (detection, then quantisation); see
+ * 32768) or M <= 64, else two (detection, then quantisation); a static
+ * weight adds the gather of the outlier rows; see
  * int8mm_launches_per_forward.  The outlier count never leaves the device,
  * so the call does not synchronise.  Grows the workspace when M exceeds every
  * earlier M (stream-ordered allocation).
@@ -160,10 +193,12 @@ int8mm_status int8mm_forward_debug(int8mm_weight_t h, const void* X_fp16_dev, in
                                    void* Y_fp16_dev, void* stream, const int8mm_debug_bufs* dbg);
 
 /*
- * Device status word of the handle: INT8MM_OK, or INT8MM_ERR_TIMEOUT if a
+ * Device status word of the handle: INT8MM_OK, INT8MM_ERR_TIMEOUT if a
  * kernel of an earlier forward gave up on a wait (the outputs of that
- * forward are then incomplete).  SYNCHRONISES the device, then clears the
- * word.  Also returns INT8MM_ERR_CUDA if the device reports an error.
+ * forward are then incomplete), or INT8MM_ERR_OUTLIER_CAP if a forward with
+ * a static weight found more outlier columns than it holds.  SYNCHRONISES
+ * the device, then clears the word.  Also returns INT8MM_ERR_CUDA if the
+ * device reports an error.
  */
 int8mm_status int8mm_get_status(int8mm_weight_t h);
 
@@ -190,7 +225,8 @@ int8mm_status int8mm_set_split_k(int8mm_weight_t h, int split);
 int8mm_status int8mm_weight_bytes(int8mm_weight_t h, size_t* bytes);
 
 /* Number of kernels a forward of M rows launches with this handle (0 for
- * M == 0, else 2 or 3).  Host-side only; nothing is enqueued. */
+ * M == 0, else 2 or 3, one more for a static weight).  Host-side only;
+ * nothing is enqueued. */
 int8mm_status int8mm_launches_per_forward(int8mm_weight_t h, int64_t M, int* count);
 
 /*

@@ -26,8 +26,9 @@ INT8MM_ERR_ALIGNMENT = 3
 INT8MM_ERR_OOM = 4
 INT8MM_ERR_CUDA = 5
 INT8MM_ERR_TIMEOUT = 6
+INT8MM_ERR_OUTLIER_CAP = 7
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_SHAPE", 3: "ALIGNMENT", 4: "OOM",
-                5: "CUDA", 6: "TIMEOUT"}
+                5: "CUDA", 6: "TIMEOUT", 7: "OUTLIER_CAP"}
 MAX_K = 65536
 
 # Symbols of include/int8mm.h and their ctypes signatures.
@@ -45,6 +46,7 @@ SIGNATURES = {
     "int8mm_get_status": (_ST, [_P]),
     "int8mm_set_wait_limit": (_ST, [_P, ctypes.c_uint64]),
     "int8mm_set_split_k": (_ST, [_P, ctypes.c_int]),
+    "int8mm_prepare_weight_static": (_ST, [_P, _I64, _I64, _P, _I64, ctypes.c_int, _P, ctypes.POINTER(_P)]),
     "int8mm_weight_bytes": (_ST, [_P, ctypes.POINTER(ctypes.c_size_t)]),
     "int8mm_launches_per_forward": (_ST, [_P, _I64, ctypes.POINTER(ctypes.c_int)]),
     "int8mm_free": (None, [_P]),
@@ -108,12 +110,13 @@ def _dev_f16_2d(t: torch.Tensor, name: str) -> torch.Tensor:
 
 class Weight:
     """A prepared weight (the library-owned handle).  Keeps a reference to
-    the borrowed fp16 weight so that it outlives the handle."""
+    the borrowed fp16 weight so that it outlives the handle (None for a
+    static weight, which keeps what it needs itself)."""
 
-    def __init__(self, handle: int, W: torch.Tensor):
+    def __init__(self, handle: int, W: torch.Tensor | None, K: int | None = None, N: int | None = None):
         self.handle = handle
         self.W = W
-        self.K, self.N = W.shape
+        self.K, self.N = W.shape if W is not None else (K, N)
 
     def __del__(self):
         h, self.handle = getattr(self, "handle", None), None
@@ -127,6 +130,20 @@ def int8mm_prepare_weight(W: torch.Tensor, stream=None) -> Weight:
     out = _P()
     _check(lib().int8mm_prepare_weight(W.data_ptr(), K, N, _stream(stream), ctypes.byref(out)))
     return Weight(out.value, W)
+
+
+def int8mm_prepare_weight_static(W: torch.Tensor, rows, max_outliers: int = 256, stream=None) -> Weight:
+    """Memory-saving prepared weight: keeps the fp16 rows W[rows, :] of the
+    calibrated outlier dimensions (any other outlier row is rebuilt from the
+    int8 codes) and at most max_outliers (capped at K) outlier columns per
+    forward.  W is not kept: it may be freed after this call."""
+    _dev_f16_2d(W, "W")
+    K, N = W.shape
+    r = (ctypes.c_int32 * max(len(rows), 1))(*[int(x) for x in rows])
+    out = _P()
+    _check(lib().int8mm_prepare_weight_static(W.data_ptr(), K, N, ctypes.cast(r, _P), len(rows),
+                                              int(min(max_outliers, K)), _stream(stream), ctypes.byref(out)))
+    return Weight(out.value, None, K, N)
 
 
 def int8mm_reserve(w: Weight, M_max: int, stream=None) -> None:

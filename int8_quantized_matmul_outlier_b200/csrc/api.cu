@@ -3,6 +3,7 @@
 // sequence of the decomposed int8 matmul.
 #include "int8mm.h"
 #include "kernels.cuh"
+#include "wstatic.cuh"
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -16,6 +17,7 @@
 #include <mutex>
 #include <string>
 #include <unordered_set>
+#include <vector>
 
 using namespace i8mm;
 
@@ -23,7 +25,7 @@ struct int8mm_weight {
   int device = 0;
   int num_sms = 148;
   int64_t K = 0, N = 0;
-  const __half* W = nullptr;  // borrowed fp16 weight [K, N]
+  const __half* W = nullptr;  // borrowed fp16 weight [K, N] (nullptr for a static weight)
   int64_t N_pad = 0;          // N rounded up to kWeightRowPad
   int8_t* Wb = nullptr;       // [K/128][N_pad][128] int8 codes, K-blocked
   float* c_w = nullptr;       // [N]
@@ -68,6 +70,17 @@ struct int8mm_weight {
   int64_t io_rows = 0;
   __half* dX = nullptr;
   __half* dY = nullptr;
+  // memory-saving weight (int8mm_prepare_weight_static): the stored fp16
+  // rows, the row map, and per forward the gathered outlier rows, which the
+  // GEMMs read as W with idx = 0, 1, 2, ...
+  bool wstatic = false;
+  int64_t w_rows = 0;
+  int out_cap = 0;
+  __half* Wc = nullptr;        // [w_rows][N]
+  int32_t* wmap = nullptr;     // [K] slot in Wc, or -1
+  int32_t* iota = nullptr;     // [out_cap] 0, 1, 2, ...
+  __half* WO = nullptr;        // [out_cap][N]
+  int32_t* count_w = nullptr;  // [1] min(|O|, out_cap)
   unsigned long long timeout_ns = 2000000000ull;
   size_t bytes = 0;
 };
@@ -177,6 +190,11 @@ void free_all(int8mm_weight* h) {
   release(&h->count);
   release(&h->colmax);
   release(&h->status);
+  release(&h->Wc);
+  release(&h->wmap);
+  release(&h->iota);
+  release(&h->WO);
+  release(&h->count_w);
 }
 
 size_t ws_bytes(const int8mm_weight* h, int64_t rows) {
@@ -308,10 +326,22 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     if ((e = launch_row_quant(Xh, M, h->K, sc, h->Xq, h->c_x, h->X_OT, /*pdl=*/true, s)) != cudaSuccess)
       return cuda_fail(e, "row quantisation launch");
   }
+  if (h->wstatic) {
+    // this forward's outlier weight rows, in the order of idx
+    GatherArgs ga{h->idx, h->count, h->wmap, h->Wc, h->Wb, h->inv_cw, static_cast<int>(h->N),
+                  static_cast<int>(h->N_pad), h->out_cap, h->WO, h->count_w, h->status};
+    if ((e = launch_gather_outlier_rows(ga, h->num_sms, /*pdl=*/true, s)) != cudaSuccess)
+      return cuda_fail(e, "outlier row gather launch");
+  }
   rec(1);
   // Without events between them, the GEMM is a programmatic dependent of the
   // row pass; an event record in between makes it an ordinary launch.
   const bool pdl = !(events && events[1]);
+  // the GEMMs read the outlier product's weight rows as W[idx[o]]: the
+  // borrowed W and the outlier columns, or the gathered rows and 0, 1, 2, ...
+  const __half* Wrows = h->wstatic ? h->WO : h->W;
+  const int32_t* widx = h->wstatic ? h->iota : h->idx;
+  const int32_t* wcount = h->wstatic ? h->count_w : h->count;
   if (decode) {
     DecodeArgs d;
     d.M = static_cast<int>(M);
@@ -320,10 +350,10 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     d.N_pad = static_cast<int>(h->N_pad);
     d.c_x = h->c_x;
     d.inv_cw = h->inv_cw;
-    d.W = h->W;
+    d.W = Wrows;
     d.X_OT = h->X_OT;
-    d.idx = h->idx;
-    d.count = h->count;
+    d.idx = widx;
+    d.count = wcount;
     d.Y = static_cast<__half*>(Y);
     d.bias = static_cast<const __half*>(bias);
     d.acc_dump = dbg ? dbg->acc : nullptr;
@@ -382,10 +412,10 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     a.N_pad = static_cast<int>(h->N_pad);
     a.c_x = h->c_x;
     a.inv_cw = h->inv_cw;
-    a.W = h->W;
+    a.W = Wrows;
     a.X_OT = h->X_OT;
-    a.idx = h->idx;
-    a.count = h->count;
+    a.idx = widx;
+    a.count = wcount;
     a.Y = static_cast<__half*>(Y);
     a.bias = static_cast<const __half*>(bias);
     a.acc_dump = dbg ? dbg->acc : nullptr;
@@ -429,10 +459,12 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
 
 void i8mm::set_last_error(const std::string& message) { g_last_error = message; }
 
-extern "C" {
+namespace {
 
-int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N, void* stream,
-                                    int8mm_weight_t* out) {
+// Shared by both prepare entry points; with `wstatic`, the memory-saving
+// weight keeping W[rows[i], :] for i < n_rows (validated by the caller).
+int8mm_status prepare_impl(const void* W_fp16_dev, int64_t K, int64_t N, void* stream, int8mm_weight_t* out,
+                           bool wstatic, const int32_t* rows, int64_t n_rows, int max_outliers) {
   if (out == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if (W_fp16_dev == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "W is NULL");
@@ -493,6 +525,31 @@ int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N
   const uint64_t wb_rows = kblocks * static_cast<uint64_t>(h->N_pad);
   int8mm_status st = make_tmap_i8(&h->tmB, h->Wb, 128, wb_rows, kGemmBK, kGemmBN);
   if (st == INT8MM_OK) st = make_tmap_i8(&h->tmW128, h->Wb, 128, wb_rows, kGemmBK, 128);
+  if (st == INT8MM_OK && wstatic) {
+    // the stored rows and the row map; W is not kept
+    std::vector<int32_t> wmap(Kz, -1), iota(static_cast<size_t>(max_outliers));
+    for (int64_t i = 0; i < n_rows; ++i) wmap[static_cast<size_t>(rows[i])] = static_cast<int32_t>(i);
+    for (int i = 0; i < max_outliers; ++i) iota[static_cast<size_t>(i)] = i;
+    const size_t R = static_cast<size_t>(n_rows), cap = static_cast<size_t>(max_outliers);
+    h->wstatic = true;
+    h->w_rows = n_rows;
+    h->out_cap = max_outliers;
+    if ((e = alloc(&h->Wc, R * Nz, s, tot)) != cudaSuccess || (e = alloc(&h->wmap, Kz, s, tot)) != cudaSuccess ||
+        (e = alloc(&h->iota, cap, s, tot)) != cudaSuccess || (e = alloc(&h->WO, cap * Nz, s, tot)) != cudaSuccess ||
+        (e = alloc(&h->count_w, 1, s, tot)) != cudaSuccess) {
+      st = cuda_fail(e, "static weight allocation");
+    } else {
+      for (size_t i = 0; i < R && e == cudaSuccess; ++i)
+        e = cudaMemcpyAsync(h->Wc + i * Nz, h->W + static_cast<size_t>(rows[i]) * Nz, Nz * 2,
+                            cudaMemcpyDeviceToDevice, s);
+      if (e == cudaSuccess) e = cudaMemcpyAsync(h->wmap, wmap.data(), Kz * 4, cudaMemcpyHostToDevice, s);
+      if (e == cudaSuccess) e = cudaMemcpyAsync(h->iota, iota.data(), cap * 4, cudaMemcpyHostToDevice, s);
+      // the host vectors and the caller's W must outlive the copies
+      if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+      if (e != cudaSuccess) st = cuda_fail(e, "static weight rows");
+    }
+    h->W = nullptr;
+  }
   if (st != INT8MM_OK) {
     cudaStreamSynchronize(s);
     free_all(h);
@@ -505,6 +562,35 @@ int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N
   }
   *out = h;
   return INT8MM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int8mm_status int8mm_prepare_weight(const void* W_fp16_dev, int64_t K, int64_t N, void* stream,
+                                    int8mm_weight_t* out) {
+  return prepare_impl(W_fp16_dev, K, N, stream, out, false, nullptr, 0, 0);
+}
+
+int8mm_status int8mm_prepare_weight_static(const void* W_fp16_dev, int64_t K, int64_t N, const int32_t* rows,
+                                           int64_t n_rows, int max_outliers, void* stream, int8mm_weight_t* out) {
+  if (out == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (K < 16 || K > INT8MM_MAX_K)  // the shape error, from the common checks
+    return prepare_impl(W_fp16_dev, K, N, stream, out, true, rows, 0, 1);
+  if (n_rows < 0 || n_rows > K || (n_rows > 0 && rows == nullptr))
+    return fail(INT8MM_ERR_INVALID_ARG, "n_rows=%lld: need 0 <= n_rows <= K and rows given", (long long)n_rows);
+  if (max_outliers < 1 || max_outliers > K)
+    return fail(INT8MM_ERR_INVALID_ARG, "max_outliers=%d: need 1 <= max_outliers <= K", max_outliers);
+  std::vector<char> seen(static_cast<size_t>(K), 0);
+  for (int64_t i = 0; i < n_rows; ++i) {
+    if (rows[i] < 0 || rows[i] >= K || seen[static_cast<size_t>(rows[i])])
+      return fail(INT8MM_ERR_INVALID_ARG, "rows[%lld]=%d: need distinct input dimensions in [0, K)", (long long)i,
+                  rows[i]);
+    seen[static_cast<size_t>(rows[i])] = 1;
+  }
+  return prepare_impl(W_fp16_dev, K, N, stream, out, true, rows, n_rows, max_outliers);
 }
 
 int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream) {
@@ -599,6 +685,9 @@ int8mm_status int8mm_get_status(int8mm_weight_t h) {
     cudaDeviceSynchronize();
     return fail(INT8MM_ERR_TIMEOUT, "a device wait ran out of time");
   }
+  if (word & kStatusOutlierCap)
+    return fail(INT8MM_ERR_OUTLIER_CAP, "a forward found more than the static weight's %d outlier columns",
+                h->out_cap);
   return INT8MM_OK;
 }
 
@@ -628,6 +717,7 @@ int8mm_status int8mm_launches_per_forward(int8mm_weight_t h, int64_t M, int* cou
   if (M == 0) *count = 0;
   else if (M <= kDecodeMaxM) *count = small_act_fits(M, h->K) ? 2 : 3;
   else *count = row_act_fits(M, h->K, h->num_sms) ? 2 : 3;
+  if (M > 0 && h->wstatic) *count += 1;  // the outlier row gather
   return INT8MM_OK;
 }
 

@@ -58,6 +58,7 @@ def lib():
         L.orc_outlier_columns.argtypes = [P, I64, I64, ctypes.c_float, P, P]
         L.orc_outlier_columns.restype = I64
         L.orc_quantize_rows.argtypes = [P, I64, I64, P, I64, P, P]
+        L.orc_rebuild_weight_rows.argtypes = [P, P, I64, I64, P]
         L.orc_quantize_cols.argtypes = [P, I64, I64, P, P]
         L.orc_int8_matmul.argtypes = [P, P, I64, I64, I64, P]
         L.orc_int8_matmul.restype = ctypes.c_int
@@ -140,6 +141,27 @@ def quantize_cols(W: np.ndarray):
     c = np.empty(N, np.float32)
     lib().orc_quantize_cols(_p(W), K, N, _p(q), _p(c))
     return q, c
+
+
+def rebuild_weight_rows(qw: np.ndarray, c_w: np.ndarray) -> np.ndarray:
+    """W rebuilt from its codes, fp16(q * (1/c_w)) per element, [K, N]."""
+    qw = np.ascontiguousarray(qw, dtype=np.int8)
+    c_w = np.ascontiguousarray(c_w, dtype=np.float32)
+    K, N = qw.shape
+    out = np.empty((K, N), dtype=np.uint16)
+    lib().orc_rebuild_weight_rows(_p(qw), _p(c_w), K, N, _p(out))
+    return out.view(np.float16)
+
+
+def static_weight(W: np.ndarray, qw: np.ndarray, c_w: np.ndarray, rows) -> np.ndarray:
+    """The weight rows a memory-saving prepared weight uses in the outlier
+    product: W[k] for the stored dimensions k in `rows`, the rebuilt row for
+    every other k."""
+    Ws = rebuild_weight_rows(qw, c_w)
+    r = np.asarray(list(rows), dtype=np.int64)
+    if r.size:
+        Ws[r] = _f16(W)[r]
+    return Ws
 
 
 def int8_matmul(qx: np.ndarray, qw: np.ndarray) -> np.ndarray:

@@ -32,6 +32,11 @@
  *  - dequantisation is acc / (c_x[i] * c_w[j]) ([estelledc] 方法1), here in
  *    double; the fp16 outlier product is accumulated in double in ascending
  *    column order; the sum is rounded once to fp16, ties to even.
+ *  - memory-saving weight: the fp16 rows of W are kept for a fixed set of
+ *    input dimensions only ([estelledc]: the outliers sit in a few fixed
+ *    feature dimensions; 方法2: only those go through fp16).  The pages leave
+ *    open what an outlier column outside the set uses: here its row is
+ *    rebuilt from the codes, w = q * (1/c_w) in fp32, rounded to fp16.
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC.
  * Floating point is IEEE binary32/binary64 with SSE arithmetic (no x87
@@ -184,6 +189,22 @@ void orc_quantize_cols(const uint16_t *W, int64_t K, int64_t N, int8_t *q, float
             float w = (float)orc_half_to_double(W[k * N + j]);
             q[k * N + j] = orc_quantize_value(w, c[j]);
         }
+}
+
+/* Memory-saving weight, rows outside the stored set: the weight row rebuilt */
+/* from its codes (the reading in the header: the pages leave it open).     */
+/* out[k,j] = binary16(rne(float(q[k,j]) * (1/c_w[j]))), the reciprocal an */
+/* fp32 division rounded once, 0 for an all-zero column (c_w = 0).          */
+void orc_rebuild_weight_rows(const int8_t *q, const float *c, int64_t K, int64_t N, uint16_t *out)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k < K; ++k) {
+        for (int64_t j = 0; j < N; ++j) {
+            float inv = (c[j] == 0.0f) ? 0.0f : 1.0f / c[j];
+            float w = (float)q[k * N + j] * inv;
+            out[k * N + j] = orc_double_to_half((double)w);
+        }
+    }
 }
 
 /* Step 3 — int8 x int8 -> int32 contraction ([aliyun] Fig. 2: Out_i32).    */

@@ -44,6 +44,29 @@ def test_prepare_rejects_bad_arguments_on_the_host():
         m.INT8MM_ERR_ALIGNMENT
 
 
+def test_static_prepare_rejects_bad_rows_on_the_host():
+    L = m.lib()
+    out = ctypes.c_void_p(1234)
+    fake = ctypes.c_void_p(4096)  # never dereferenced: the row checks come first
+
+    def rows(*v):
+        return ctypes.cast((ctypes.c_int32 * len(v))(*v), ctypes.c_void_p)
+
+    cases = [(None, 1, 4),            # rows missing
+             (rows(1, 2), -1, 4),     # negative count
+             (rows(3, 3), 2, 4),      # repeated dimension
+             (rows(64), 1, 4),        # outside [0, K)
+             (rows(-1), 1, 4),
+             (rows(1), 1, 0),         # no room for outliers
+             (rows(1), 1, 65)]        # more room than K
+    for r, n, cap in cases:
+        st = L.int8mm_prepare_weight_static(fake, 64, 64, r, n, cap, None, ctypes.byref(out))
+        assert st == m.INT8MM_ERR_INVALID_ARG, (n, cap)
+        assert out.value is None
+    assert L.int8mm_prepare_weight_static(fake, 15, 64, None, 0, 4, None, ctypes.byref(out)) == \
+        m.INT8MM_ERR_UNSUPPORTED_SHAPE
+
+
 def test_calls_on_an_unknown_handle_are_rejected():
     L = m.lib()
     bogus = ctypes.c_void_p(0xdead0)

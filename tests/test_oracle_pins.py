@@ -344,3 +344,48 @@ def test_tensorwise_absmax_hand_example():
     # y = acc / (15.875 * 63.5) = acc / 1008.0625 -> [16.5078.., -7.0472..]
     acc = np.array([[16641, -7104], [-64 * 127 + 8 * 32, -64 * -64 + 8 * 64]], np.float64)
     assert (r["Y"].astype(np.float64) == (acc / (15.875 * 63.5)).astype(np.float16)).all()
+
+
+# --------------------------------------------------------------------------
+# memory-saving weight: rows outside the stored set rebuilt from the codes
+
+def test_rebuilt_weight_rows_exact_on_the_code_grid():
+    # columns whose entries lie on their own code grid (absmax / 127 apart)
+    # come back exactly: absmax 63.5 (c_w = 2), 127 (c_w = 1), 254 (c_w = 0.5).
+    # A scale applied the wrong way (q * c_w) or not at all fails the first
+    # and the last column.
+    rng = np.random.default_rng(3)
+    q = rng.integers(-127, 128, size=(40, 3))
+    q[0] = [127, -127, 127]  # every column reaches its absmax
+    W = (q * np.array([0.5, 1.0, 2.0])).astype(np.float16)
+    qw, c_w = oracle.quantize_cols(W)
+    assert c_w.tolist() == [2.0, 1.0, 0.5]
+    assert (qw == q).all()
+    assert (oracle.rebuild_weight_rows(qw, c_w) == W).all()
+
+
+def test_rebuilt_weight_rows_within_half_a_code_step():
+    # |w~ - w| <= absmax / 254 (half a code step, up to fp32 rounding of the
+    # product) + half an fp16 ulp of w~; an all-zero column rebuilds to zeros
+    rng = np.random.default_rng(4)
+    W = (rng.standard_normal((64, 9)) * 0.02).astype(np.float16)
+    W[:, 4] = 0
+    qw, c_w = oracle.quantize_cols(W)
+    Wr = oracle.rebuild_weight_rows(qw, c_w)
+    absmax = np.abs(W.astype(np.float64)).max(axis=0)
+    err = np.abs(Wr.astype(np.float64) - W.astype(np.float64))
+    bound = absmax / 254 * (1 + 1e-6) + np.spacing(np.abs(Wr)).astype(np.float64) / 2
+    assert (err <= bound).all()
+    assert (Wr[:, 4] == 0).all() and c_w[4] == 0
+    assert err.max() > 0  # the rebuilt rows are the quantised weight, not W
+
+
+def test_static_weight_keeps_the_stored_rows():
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((12, 7)) * 0.05).astype(np.float16)
+    qw, c_w = oracle.quantize_cols(W)
+    Ws = oracle.static_weight(W, qw, c_w, [1, 5])
+    Wr = oracle.rebuild_weight_rows(qw, c_w)
+    assert (Ws[[1, 5]] == W[[1, 5]]).all()
+    others = [k for k in range(12) if k not in (1, 5)]
+    assert (Ws[others] == Wr[others]).all()

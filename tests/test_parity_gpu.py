@@ -245,6 +245,72 @@ def test_split_k_with_bias():
     m.int8mm_free(w)
 
 
+# ------------------------------------------------- memory-saving weight
+
+def test_static_weight_with_the_outlier_dims_stored_equals_the_borrowed_weight():
+    # the stored rows are the rows of W: the same Y, bit for bit, as the
+    # handle that borrows all of W, on the prefill and the decode kernels;
+    # the static handle keeps no reference to W (overwritten after prepare)
+    p = workloads.small(300, 1040, 784, 5, seed=41)
+    X = torch.from_numpy(p.X).to(dev())
+    W = torch.from_numpy(p.W).to(dev())
+    wb = m.int8mm_prepare_weight(W)
+    Wtmp = W.clone()
+    ws = m.int8mm_prepare_weight_static(Wtmp, p.planted.tolist(), max_outliers=16)
+    Wtmp.fill_(7.0)
+    assert m.int8mm_launches_per_forward(ws, 300) == m.int8mm_launches_per_forward(wb, 300) + 1
+    for rows in (X, X[:8].contiguous(), X[:64].contiguous()):
+        yb = m.int8mm_forward(wb, rows, 6.0)
+        ys = m.int8mm_forward(ws, rows, 6.0)
+        torch.cuda.synchronize()
+        assert m.int8mm_get_status(ws) == m.INT8MM_OK
+        assert torch.equal(yb, ys)
+
+
+@pytest.mark.parametrize("M,stored", [(300, "none"), (300, "half"), (8, "half"), (2048, "half")])
+def test_static_weight_against_oracle(M, stored):
+    # outlier columns outside the stored set use the weight rows rebuilt from
+    # the codes; accumulators bit-exact, Y within tolerance of the oracle
+    p = workloads.small(M, 2048, 1040, 6, seed=M + 43)
+    _, idx = oracle.outlier_columns(p.X, p.alpha)
+    rows = [] if stored == "none" else idx[::2].tolist()
+    ws = m.int8mm_prepare_weight_static(torch.from_numpy(p.W).to(dev()), rows, max_outliers=32)
+    d = m.int8mm_forward_debug(ws, torch.from_numpy(p.X).to(dev()), p.alpha)
+    torch.cuda.synchronize()
+    assert m.int8mm_get_status(ws) == m.INT8MM_OK
+    qx, c_x = oracle.quantize_rows(p.X, idx)
+    qw, c_w = oracle.quantize_cols(p.W)
+    acc = oracle.int8_matmul(qx, qw)
+    assert (d["acc"].cpu().numpy() == acc).all()
+    Ws = oracle.static_weight(p.W, qw, c_w, rows)
+    y_o, _ = oracle.dequant_add_outliers(acc, c_x, c_w, p.X, Ws, idx)
+    assert_y_close(d["Y"].cpu().numpy(), y_o, p.X, Ws, idx)
+    m.int8mm_free(ws)
+
+
+def test_static_weight_outlier_cap():
+    # 7 outlier columns against room for 4: the first 4 (ascending) get their
+    # fp16 product, the rest none, and the status word says so
+    p = workloads.small(300, 1040, 784, 7, seed=47)
+    X = torch.from_numpy(p.X).to(dev())
+    ws = m.int8mm_prepare_weight_static(torch.from_numpy(p.W).to(dev()), [], max_outliers=4)
+    y = m.int8mm_forward(ws, X, 6.0)
+    torch.cuda.synchronize()
+    assert m.int8mm_get_status(ws) == m.INT8MM_ERR_OUTLIER_CAP
+    _, idx = oracle.outlier_columns(p.X, 6.0)
+    assert idx.size == 7
+    qx, c_x = oracle.quantize_rows(p.X, idx)
+    qw, c_w = oracle.quantize_cols(p.W)
+    Ws = oracle.static_weight(p.W, qw, c_w, [])
+    y_o, _ = oracle.dequant_add_outliers(oracle.int8_matmul(qx, qw), c_x, c_w, p.X, Ws, idx[:4])
+    assert_y_close(y.cpu().numpy(), y_o, p.X, Ws, idx[:4])
+    m.int8mm_forward(ws, X, math.inf)  # no outliers: within the cap again
+    torch.cuda.synchronize()
+    assert m.int8mm_get_status(ws) == m.INT8MM_OK
+    with pytest.raises(RuntimeError):
+        m.int8mm_prepare_weight_static(torch.from_numpy(p.W).to(dev()), [3, 3], max_outliers=4)
+
+
 def test_linear8bitlt_module():
     torch.manual_seed(0)
     K, N = 1040, 784
