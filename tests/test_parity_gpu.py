@@ -311,6 +311,32 @@ def test_static_weight_outlier_cap():
         m.int8mm_prepare_weight_static(torch.from_numpy(p.W).to(dev()), [3, 3], max_outliers=4)
 
 
+# ------------------------------------------------- column-parallel shards
+
+@pytest.mark.parametrize("M", [300, 8])
+def test_column_shards_reproduce_the_unsharded_forward(M):
+    # the N-split on one GPU, shard by shard (no collective): each rank's
+    # weight slice gives exactly its columns of the unsharded Y and acc
+    from int8_quantized_matmul_outlier_b200.nsplit import ColumnParallelInt8Matmul, column_ranges
+    p = workloads.small(M, 1040, 784, 5, seed=M + 53)
+    X = torch.from_numpy(p.X).to(dev())
+    W = torch.from_numpy(p.W).to(dev())
+    full = m.int8mm_prepare_weight(W)
+    d = m.int8mm_forward_debug(full, X, p.alpha)
+    for world in (2, 3):
+        ranges = column_ranges(784, world)
+        shards = [m.int8mm_prepare_weight(W[:, a:b].contiguous()) for a, b in ranges]
+        parts = [m.int8mm_forward_debug(w, X, p.alpha) for w in shards]
+        torch.cuda.synchronize()
+        assert torch.equal(torch.cat([q["acc"] for q in parts], 1), d["acc"])
+        assert torch.equal(torch.cat([q["Y"] for q in parts], 1), d["Y"])
+    # the module in one process (one rank), borrowed and static weights
+    y1 = ColumnParallelInt8Matmul(W)(X, p.alpha)
+    y2 = ColumnParallelInt8Matmul(W, static_rows=p.planted.tolist(), max_outliers=16)(X, p.alpha)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, d["Y"]) and torch.equal(y2, d["Y"])
+
+
 def test_linear8bitlt_module():
     torch.manual_seed(0)
     K, N = 1040, 784
