@@ -364,6 +364,13 @@ def test_linear8bitlt_module():
     assert torch.allclose(y0.float() + lin.bias.float(), y.float(), atol=2e-2, rtol=1e-2)
     with pytest.raises(TypeError):
         q(x.float())
+    # the memory-saving layer with the outlier dimensions stored: the same
+    # output, and no fp16 weight kept
+    qs = m.Linear8bitLt.from_linear(lin, threshold=6.0, static_rows=p.planted.tolist(), max_outliers=16)
+    assert qs.weight is None
+    ys = qs(x)
+    torch.cuda.synchronize()
+    assert torch.equal(ys, y)
 
 
 def test_zero_rows_and_columns():
