@@ -41,8 +41,12 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        build()
-        L = ctypes.CDLL(_LIB_PATH)
+        # INT8MM_ORACLE_LIB is set only by the oracle's own mutation test, to
+        # run the pins against a copy of oracle.c with one planted mistake
+        path = os.environ.get("INT8MM_ORACLE_LIB")
+        if not path:
+            path = build()
+        L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
         L.orc_half_to_double.argtypes = [ctypes.c_uint16]
