@@ -213,6 +213,18 @@ def cpu_rows_for(p, target_s: float, wq):
     return int(max(1, min(M, 16 * target_s / max(t, 1e-4))))
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo", encoding="utf-8", errors="replace") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(p: workloads.Problem, rows: int) -> dict:
     import oracle
     wq = oracle.quantize_cols(p.W)
@@ -233,7 +245,8 @@ def cpu_baseline(p: workloads.Problem, rows: int) -> dict:
             "sample": f"batch of the first {rows} of {M} rows, whole forward on it; "
                       f"weight codes prepared outside the timed region",
             "seconds": t,
-            "single_thread_tiny_forward_s": t1}
+            "single_thread_tiny_forward_s": t1,
+            "cpu_model": cpu_model(), "host_threads": os.cpu_count()}
 
 
 # --------------------------------------------------------------------------
@@ -417,6 +430,7 @@ def run_reference(args):
         "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": workload_config(p),
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+                         "cpu_model": cpu_model(),
                          "sample": f"each step: whole forward on a batch of the first {rows} of {M} rows; "
                                    f"weight codes prepared once, untimed"},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
