@@ -204,8 +204,12 @@ int8mm_status int8mm_get_status(int8mm_weight_t h);
 
 /*
  * Time limit, in nanoseconds, for each device-side wait of later forwards
- * (default 2e9, i.e. two seconds).  Diagnostic: a tiny limit makes waits
- * give up early and report INT8MM_ERR_TIMEOUT through int8mm_get_status.
+ * (default 2e9, i.e. two seconds), at least 1e6 (one millisecond).  A
+ * kernel whose wait gives up reports INT8MM_ERR_TIMEOUT through
+ * int8mm_get_status; before its blocks exit they wait, within the same
+ * limit, for the copies and tensor-core operations they have already issued,
+ * which take microseconds: the floor keeps that drain complete.
+ * INT8MM_ERR_INVALID_ARG below the floor.
  */
 int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns);
 

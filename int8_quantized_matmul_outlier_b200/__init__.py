@@ -268,6 +268,7 @@ def int8mm_get_status(w: Weight) -> int:
 
 
 def int8mm_set_wait_limit(w: Weight, timeout_ns: int) -> None:
+    """Limit of each device-side wait, in ns (at least 1e6)."""
     _check(lib().int8mm_set_wait_limit(w.handle, int(timeout_ns)))
 
 

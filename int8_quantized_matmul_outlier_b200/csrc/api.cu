@@ -693,7 +693,11 @@ int8mm_status int8mm_get_status(int8mm_weight_t h) {
 
 int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns) {
   if (!live(h)) return fail(INT8MM_ERR_INVALID_ARG, "invalid or freed weight handle");
-  if (timeout_ns == 0) return fail(INT8MM_ERR_INVALID_ARG, "timeout must be positive");
+  // a block that gives up still waits, within this limit, for the copies and
+  // MMAs it has issued (microseconds); the floor keeps that drain complete
+  if (timeout_ns < 1000000ull)
+    return fail(INT8MM_ERR_INVALID_ARG, "timeout %llu ns is below the 1 ms minimum",
+                static_cast<unsigned long long>(timeout_ns));
   h->timeout_ns = timeout_ns;
   return INT8MM_OK;
 }
