@@ -203,6 +203,16 @@ int8mm_status int8mm_forward_debug(int8mm_weight_t h, const void* X_fp16_dev, in
 int8mm_status int8mm_get_status(int8mm_weight_t h);
 
 /*
+ * Failure-detection self-test: enqueues on `stream` one single-thread kernel
+ * that waits, bounded by the handle's wait limit (int8mm_set_wait_limit), on
+ * a device flag that nothing sets, as the forward's kernels wait on tickets
+ * and barriers.  The wait runs out; the kernel records it in the handle's
+ * status word and returns, so int8mm_get_status then reports
+ * INT8MM_ERR_TIMEOUT and the handle and the CUDA context stay usable.
+ */
+int8mm_status int8mm_wait_selftest(int8mm_weight_t h, void* stream);
+
+/*
  * Time limit, in nanoseconds, for each device-side wait of later forwards
  * (default 2e9, i.e. two seconds), at least 1e6 (one millisecond).  A
  * kernel whose wait gives up reports INT8MM_ERR_TIMEOUT through

@@ -46,6 +46,7 @@ SIGNATURES = {
     "int8mm_get_status": (_ST, [_P]),
     "int8mm_set_wait_limit": (_ST, [_P, ctypes.c_uint64]),
     "int8mm_set_split_k": (_ST, [_P, ctypes.c_int]),
+    "int8mm_wait_selftest": (_ST, [_P, _P]),
     "int8mm_prepare_weight_static": (_ST, [_P, _I64, _I64, _P, _I64, ctypes.c_int, _P, ctypes.POINTER(_P)]),
     "int8mm_weight_bytes": (_ST, [_P, ctypes.POINTER(ctypes.c_size_t)]),
     "int8mm_launches_per_forward": (_ST, [_P, _I64, ctypes.POINTER(ctypes.c_int)]),
@@ -270,6 +271,13 @@ def int8mm_get_status(w: Weight) -> int:
 def int8mm_set_wait_limit(w: Weight, timeout_ns: int) -> None:
     """Limit of each device-side wait, in ns (at least 1e6)."""
     _check(lib().int8mm_set_wait_limit(w.handle, int(timeout_ns)))
+
+
+def int8mm_wait_selftest(w: Weight, stream=None) -> None:
+    """Enqueue the failure-detection self-test: a device wait that runs out
+    after the handle's wait limit and leaves INT8MM_ERR_TIMEOUT for
+    int8mm_get_status."""
+    _check(lib().int8mm_wait_selftest(w.handle, _stream(stream)))
 
 
 def int8mm_set_split_k(w: Weight, split: int) -> None:

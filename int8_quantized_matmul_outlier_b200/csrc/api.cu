@@ -3,6 +3,7 @@
 // sequence of the decomposed int8 matmul.
 #include "int8mm.h"
 #include "kernels.cuh"
+#include "selftest.cuh"
 #include "wstatic.cuh"
 
 #include <cuda.h>
@@ -81,6 +82,7 @@ struct int8mm_weight {
   int32_t* iota = nullptr;     // [out_cap] 0, 1, 2, ...
   __half* WO = nullptr;        // [out_cap][N]
   int32_t* count_w = nullptr;  // [1] min(|O|, out_cap)
+  uint32_t* never_set = nullptr;  // [1] zero: the flag of the wait self-test
   unsigned long long timeout_ns = 2000000000ull;
   size_t bytes = 0;
 };
@@ -195,6 +197,7 @@ void free_all(int8mm_weight* h) {
   release(&h->iota);
   release(&h->WO);
   release(&h->count_w);
+  release(&h->never_set);
 }
 
 size_t ws_bytes(const int8mm_weight* h, int64_t rows) {
@@ -699,6 +702,25 @@ int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns) {
     return fail(INT8MM_ERR_INVALID_ARG, "timeout %llu ns is below the 1 ms minimum",
                 static_cast<unsigned long long>(timeout_ns));
   h->timeout_ns = timeout_ns;
+  return INT8MM_OK;
+}
+
+int8mm_status int8mm_wait_selftest(int8mm_weight_t h, void* stream) {
+  if (!live(h)) return fail(INT8MM_ERR_INVALID_ARG, "invalid or freed weight handle");
+  int8mm_status st = set_device(h);
+  if (st != INT8MM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (h->never_set == nullptr) {
+    if ((e = alloc(&h->never_set, 1, s, &h->bytes)) != cudaSuccess ||
+        (e = cudaMemsetAsync(h->never_set, 0, 4, s)) != cudaSuccess) {
+      cudaStreamSynchronize(s);
+      release(&h->never_set);
+      return cuda_fail(e, "self-test flag allocation");
+    }
+  }
+  if ((e = launch_wait_selftest(h->never_set, h->status, h->timeout_ns, s)) != cudaSuccess)
+    return cuda_fail(e, "wait self-test launch");
   return INT8MM_OK;
 }
 

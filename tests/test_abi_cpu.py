@@ -78,6 +78,7 @@ def test_calls_on_an_unknown_handle_are_rejected():
     assert L.int8mm_reserve(bogus, 16, None) == m.INT8MM_ERR_INVALID_ARG
     assert L.int8mm_set_wait_limit(bogus, 1000) == m.INT8MM_ERR_INVALID_ARG
     assert L.int8mm_set_split_k(bogus, 2) == m.INT8MM_ERR_INVALID_ARG
+    assert L.int8mm_wait_selftest(bogus, None) == m.INT8MM_ERR_INVALID_ARG
     n = ctypes.c_size_t()
     assert L.int8mm_weight_bytes(bogus, ctypes.byref(n)) == m.INT8MM_ERR_INVALID_ARG
     L.int8mm_free(None)    # no-op
