@@ -112,7 +112,10 @@ int8mm_status int8mm_prepare_weight_static(const void* W_fp16_dev, int64_t K, in
 /*
  * Pre-size the per-forward workspace for up to M_max rows, so that later
  * forward calls with M <= M_max allocate nothing (needed before CUDA graph
- * capture of a forward).  Stream-ordered allocation on `stream`.
+ * capture of a forward): the activation workspace, the decode GEMM's scratch
+ * and the split-K workspace of the largest split any M <= M_max uses with
+ * the int8mm_set_split_k setting in effect (call it again after changing
+ * that setting).  Stream-ordered allocation on `stream`.
  */
 int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream);
 

@@ -237,6 +237,74 @@ int8mm_status ensure_workspace(int8mm_weight* h, int64_t M, cudaStream_t s) {
   return INT8MM_OK;
 }
 
+// Scratch of the decode GEMM (M <= kDecodeMaxM): int32 partial sums and
+// per-n-block tickets, zeroed; allocated once, in stream order.
+int8mm_status ensure_decode_scratch(int8mm_weight* h, cudaStream_t s) {
+  if (h->part != nullptr) return INT8MM_OK;
+  const size_t nb = static_cast<size_t>((h->N + 127) / 128);
+  cudaError_t ea;
+  if ((ea = alloc(&h->part, static_cast<size_t>(kDecodeMaxM) * h->N, s, &h->bytes)) != cudaSuccess ||
+      (ea = alloc(&h->dticket, nb, s, &h->bytes)) != cudaSuccess ||
+      (ea = cudaMemsetAsync(h->part, 0, static_cast<size_t>(kDecodeMaxM) * h->N * 4, s)) != cudaSuccess ||
+      (ea = cudaMemsetAsync(h->dticket, 0, nb * 4, s)) != cudaSuccess) {
+    cudaStreamSynchronize(s);
+    release(&h->part);
+    release(&h->dticket);
+    return cuda_fail(ea, "decode scratch allocation");
+  }
+  return INT8MM_OK;
+}
+
+// Pieces along K of the prefill GEMM for M rows (1 for single-CTA tiles).
+int split_for(const int8mm_weight* h, int64_t M) {
+  if (M <= kGemmBM) return 1;
+  const int64_t num_kb = (h->K + kGemmBK - 1) / kGemmBK;
+  return h->split_override > 0 ? static_cast<int>(std::min<int64_t>(h->split_override, num_kb))
+                               : gemm_split_for(M, h->N, h->K, h->num_sms);
+}
+
+// 256 x 256 tiles of the CTA-pair GEMM for M rows.
+size_t pair_tiles(const int8mm_weight* h, int64_t M) {
+  return static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM)) *
+         static_cast<size_t>((h->N + kGemmBN - 1) / kGemmBN);
+}
+
+// Grows the split-K partial-tile workspace to ws_elems int32 and the tickets
+// to n_tickets zeroed counters, in stream order (old buffers freed on s).
+int8mm_status ensure_split_scratch(int8mm_weight* h, size_t ws_elems, size_t n_tickets, cudaStream_t s) {
+  cudaError_t e;
+  if (ws_elems > h->sk_ws_elems) {
+    if (h->sk_ws) {
+      cudaFreeAsync(h->sk_ws, s);
+      h->bytes -= h->sk_ws_elems * 4;
+      h->sk_ws = nullptr;
+      h->sk_ws_elems = 0;
+    }
+    if ((e = alloc(&h->sk_ws, ws_elems, s, &h->bytes)) != cudaSuccess) {
+      cudaStreamSynchronize(s);
+      release(&h->sk_ws);
+      return cuda_fail(e, "split-K workspace allocation");
+    }
+    h->sk_ws_elems = ws_elems;
+  }
+  if (n_tickets > h->sk_ticket_n) {
+    if (h->sk_ticket) {
+      cudaFreeAsync(h->sk_ticket, s);
+      h->bytes -= h->sk_ticket_n * 4;
+      h->sk_ticket = nullptr;
+      h->sk_ticket_n = 0;
+    }
+    if ((e = alloc(&h->sk_ticket, n_tickets, s, &h->bytes)) != cudaSuccess ||
+        (e = cudaMemsetAsync(h->sk_ticket, 0, n_tickets * 4, s)) != cudaSuccess) {
+      cudaStreamSynchronize(s);
+      release(&h->sk_ticket);
+      return cuda_fail(e, "split-K ticket allocation");
+    }
+    h->sk_ticket_n = n_tickets;
+  }
+  return INT8MM_OK;
+}
+
 int8mm_status check_forward_args(const int8mm_weight* h, const void* X, int64_t M, float alpha, const void* Y) {
   if (!live(h)) return fail(INT8MM_ERR_INVALID_ARG, "invalid or freed weight handle");
   if (M < 0 || M >= (int64_t(1) << 31)) return fail(INT8MM_ERR_INVALID_ARG, "M=%lld out of range", (long long)M);
@@ -276,19 +344,7 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     h->tmA_rows = M;
     h->tmA_box = box_rows;
   }
-  if (decode && h->part == nullptr) {
-    const size_t nb = static_cast<size_t>((h->N + 127) / 128);
-    cudaError_t ea;
-    if ((ea = alloc(&h->part, static_cast<size_t>(kDecodeMaxM) * h->N, s, &h->bytes)) != cudaSuccess ||
-        (ea = alloc(&h->dticket, nb, s, &h->bytes)) != cudaSuccess ||
-        (ea = cudaMemsetAsync(h->part, 0, static_cast<size_t>(kDecodeMaxM) * h->N * 4, s)) != cudaSuccess ||
-        (ea = cudaMemsetAsync(h->dticket, 0, nb * 4, s)) != cudaSuccess) {
-      cudaStreamSynchronize(s);
-      release(&h->part);
-      release(&h->dticket);
-      return cuda_fail(ea, "decode scratch allocation");
-    }
-  }
+  if (decode && (st = ensure_decode_scratch(h, s)) != INT8MM_OK) return st;
   OutlierScratch sc{h->colkey, h->epoch, h->ticket, h->mask, h->pre, h->idx, h->count, h->colmax};
   const __half* Xh = static_cast<const __half*>(X);
   cudaError_t e;
@@ -368,45 +424,12 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
       return cuda_fail(e, "int8 decode GEMM launch");
   } else {
     // split K for the CTA-pair tiles; the scratch grows on demand
-    int split = 1;
-    if (M > kGemmBM) {
-      const int64_t num_kb = (h->K + kGemmBK - 1) / kGemmBK;
-      split = h->split_override > 0 ? static_cast<int>(std::min<int64_t>(h->split_override, num_kb))
-                                    : gemm_split_for(M, h->N, h->K, h->num_sms);
-    }
+    const int split = split_for(h, M);
     if (split > 1) {
-      const size_t tiles = static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM)) *
-                           static_cast<size_t>((h->N + kGemmBN - 1) / kGemmBN);
-      const size_t ws = static_cast<size_t>(split - 1) * tiles * 2 * kGemmBM * kGemmBN;
-      if (ws > h->sk_ws_elems) {
-        if (h->sk_ws) {
-          cudaFreeAsync(h->sk_ws, s);
-          h->bytes -= h->sk_ws_elems * 4;
-          h->sk_ws = nullptr;
-          h->sk_ws_elems = 0;
-        }
-        if ((e = alloc(&h->sk_ws, ws, s, &h->bytes)) != cudaSuccess) {
-          cudaStreamSynchronize(s);
-          release(&h->sk_ws);
-          return cuda_fail(e, "split-K workspace allocation");
-        }
-        h->sk_ws_elems = ws;
-      }
-      if (tiles * 4 > h->sk_ticket_n) {
-        if (h->sk_ticket) {
-          cudaFreeAsync(h->sk_ticket, s);
-          h->bytes -= h->sk_ticket_n * 4;
-          h->sk_ticket = nullptr;
-          h->sk_ticket_n = 0;
-        }
-        if ((e = alloc(&h->sk_ticket, tiles * 4, s, &h->bytes)) != cudaSuccess ||
-            (e = cudaMemsetAsync(h->sk_ticket, 0, tiles * 16, s)) != cudaSuccess) {
-          cudaStreamSynchronize(s);
-          release(&h->sk_ticket);
-          return cuda_fail(e, "split-K ticket allocation");
-        }
-        h->sk_ticket_n = tiles * 4;
-      }
+      const size_t tiles = pair_tiles(h, M);
+      if ((st = ensure_split_scratch(h, static_cast<size_t>(split - 1) * tiles * 2 * kGemmBM * kGemmBN, tiles * 4,
+                                     s)) != INT8MM_OK)
+        return st;
     }
     GemmArgs a;
     a.M = static_cast<int>(M);
@@ -601,7 +624,23 @@ int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream) {
   if (M_max < 0 || M_max >= (int64_t(1) << 31)) return fail(INT8MM_ERR_INVALID_ARG, "M_max out of range");
   int8mm_status st = set_device(h);
   if (st != INT8MM_OK) return st;
-  return ensure_workspace(h, M_max, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = ensure_workspace(h, M_max, s)) != INT8MM_OK) return st;
+  if (M_max >= 1 && (st = ensure_decode_scratch(h, s)) != INT8MM_OK) return st;
+  // the largest split-K scratch of any M <= M_max (the split depends on M
+  // only through its number of 256-row tiles)
+  size_t ws_max = 0, tickets_max = 0;
+  for (int64_t mt = 1; (mt - 1) * 2 * kGemmBM < M_max; ++mt) {
+    const int64_t M = std::min<int64_t>(M_max, mt * 2 * kGemmBM);
+    const int split = split_for(h, M);
+    if (split > 1) {
+      const size_t tiles = pair_tiles(h, M);
+      ws_max = std::max(ws_max, static_cast<size_t>(split - 1) * tiles * 2 * kGemmBM * kGemmBN);
+      tickets_max = std::max(tickets_max, tiles * 4);
+    }
+  }
+  if (ws_max > 0) return ensure_split_scratch(h, ws_max, tickets_max, s);
+  return INT8MM_OK;
 }
 
 int8mm_status int8mm_forward(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha, void* Y_fp16_dev,
