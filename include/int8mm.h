@@ -197,11 +197,16 @@ int8mm_status int8mm_forward_debug(int8mm_weight_t h, const void* X_fp16_dev, in
 
 /*
  * Device status word of the handle: INT8MM_OK, INT8MM_ERR_TIMEOUT if a
- * kernel of an earlier forward gave up on a wait (the outputs of that
- * forward are then incomplete), or INT8MM_ERR_OUTLIER_CAP if a forward with
- * a static weight found more outlier columns than it holds.  SYNCHRONISES
- * the device, then clears the word.  Also returns INT8MM_ERR_CUDA if the
- * device reports an error.
+ * kernel of an earlier forward gave up on a wait, or INT8MM_ERR_OUTLIER_CAP
+ * if a forward with a static weight found more outlier columns than it
+ * holds.  SYNCHRONISES the device, then clears the word.  Also returns
+ * INT8MM_ERR_CUDA if the device reports an error.
+ *
+ * After a timeout, the forward that timed out AND every later forward on the
+ * handle are invalid until this call has returned INT8MM_ERR_TIMEOUT: an
+ * aborted kernel can leave counters (split-K and decode tickets, the
+ * activation pass's grid barrier) that a later forward would misread, and
+ * this call is what resets them.
  */
 int8mm_status int8mm_get_status(int8mm_weight_t h);
 
@@ -254,11 +259,13 @@ int8mm_status int8mm_launches_per_forward(int8mm_weight_t h, int64_t M, int* cou
  * warm-up, or a process whose caching allocator already holds nearly all of
  * the device memory.
  *
- * X_fp16_dev: [M, K] fp16 row-major, 16-byte aligned (M >= 0).
+ * X_fp16_dev: [M, K] fp16 row-major, 16-byte aligned (0 <= M < 2^31; may
+ *             be NULL when M == 0).
  * idx_dev:    [K] int32, written with the ascending outlier columns; the
  *             first *count_dev entries are valid.
  * count_dev:  [1] int32, written with |O|.
- * colmax_dev: [K] fp32 max_i |X[i,j]|, or NULL to skip it.
+ * colmax_dev: [K] fp32 max_i |X[i,j]| (all 0 when M == 0), or NULL to skip
+ *             it.
  * All three outputs are device memory owned by the caller.  Same results as
  * the outlier_idx / outlier_count / colmax of int8mm_forward_debug.
  *
@@ -267,9 +274,11 @@ int8mm_status int8mm_launches_per_forward(int8mm_weight_t h, int64_t M, int* cou
  * exits; the call itself makes no cudaMalloc, cudaFree or other allocation.
  * Limit: 16 <= K <= INT8MM_MAX_K, K % 16 == 0 (larger K is rejected with
  * INT8MM_ERR_UNSUPPORTED_SHAPE).  The first call on a device looks up the
- * array's device address; make that first call before any CUDA stream
- * capture.  All calls share the array and each call clears what must start
- * at zero; calls whose kernels overlap on the GPU (unordered streams) race.
+ * array's device address in the current context (again after the context
+ * is re-created, e.g. by cudaDeviceReset); make that first call before any
+ * CUDA stream capture.  All calls share the array and each call clears what
+ * must start at zero; calls whose kernels overlap on the GPU (unordered
+ * streams) race.
  */
 #define INT8MM_NOALLOC_SCRATCH_BYTES (1u << 20)
 int8mm_status int8mm_outlier_columns_noalloc(const void* X_fp16_dev, int64_t M, int64_t K, float alpha,

@@ -18,6 +18,7 @@
 #include "int8mm.h"
 #include "kernels.cuh"
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -43,6 +44,11 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
+// Per device: the context the address was looked up in, and the address.
+// A context that is destroyed and re-created (cudaDeviceReset, or a primary
+// context released and retained again) reloads the library's device image,
+// so the array may move: the address is looked up again for a new context.
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 void* g_scratch_ptr[kMaxDevices] = {};
 
 int8mm_status setup_error(int8mm_status s, const std::string& msg) {
@@ -50,16 +56,46 @@ int8mm_status setup_error(int8mm_status s, const std::string& msg) {
   return s;
 }
 
-// Once per device, with that device current: the device address of the
-// static scratch array (its host-side name is only a stand-in).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if there is none or
+// the driver cannot say); ids are never reused within a process.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Once per device and context, with that device current: the device address
+// of the static scratch array (its host-side name is only a stand-in).
 int8mm_status device_scratch(int dev, void** ptr) {
   std::lock_guard<std::mutex> g(g_setup_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_scratch_ptr[dev] == nullptr || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess)
       return setup_error(INT8MM_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
     g_scratch_ptr[dev] = p;
+    // the lookup makes the device's primary context current if none was
+    g_scratch_ctx[dev] = ctx != 0 ? ctx : current_context_id();
   }
   *ptr = g_scratch_ptr[dev];
   return INT8MM_OK;
@@ -72,8 +108,8 @@ extern "C" {
 int8mm_status int8mm_outlier_columns_noalloc(const void* X_fp16_dev, int64_t M, int64_t K, float alpha,
                                              int32_t* idx_dev, int32_t* count_dev, float* colmax_dev,
                                              void* stream) {
-  if (X_fp16_dev == nullptr || idx_dev == nullptr || count_dev == nullptr)
-    return setup_error(INT8MM_ERR_INVALID_ARG, "X, idx and count must not be NULL");
+  if (idx_dev == nullptr || count_dev == nullptr || (M > 0 && X_fp16_dev == nullptr))
+    return setup_error(INT8MM_ERR_INVALID_ARG, "idx and count, and X when M > 0, must not be NULL");
   if (std::isnan(alpha)) return setup_error(INT8MM_ERR_INVALID_ARG, "alpha is NaN");
   if (M < 0 || M >= (int64_t(1) << 31))
     return setup_error(INT8MM_ERR_INVALID_ARG, "M must be in [0, 2^31)");
@@ -94,9 +130,11 @@ int8mm_status int8mm_outlier_columns_noalloc(const void* X_fp16_dev, int64_t M, 
   if (st != INT8MM_OK) return st;
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (M == 0) {  // no rows: no outlier columns
-    if ((e = cudaMemsetAsync(count_dev, 0, sizeof(int32_t), cs)) != cudaSuccess)
-      return setup_error(INT8MM_ERR_CUDA, std::string("count reset: ") + cudaGetErrorString(e));
+  if (M == 0) {  // no rows: no outlier columns, and every column maximum is 0
+    if ((e = cudaMemsetAsync(count_dev, 0, sizeof(int32_t), cs)) != cudaSuccess ||
+        (colmax_dev != nullptr &&
+         (e = cudaMemsetAsync(colmax_dev, 0, static_cast<size_t>(K) * sizeof(float), cs)) != cudaSuccess))
+      return setup_error(INT8MM_ERR_CUDA, std::string("output reset: ") + cudaGetErrorString(e));
     return INT8MM_OK;
   }
   unsigned char* s = static_cast<unsigned char*>(base);
