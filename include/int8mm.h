@@ -232,6 +232,28 @@ int8mm_status int8mm_wait_selftest(int8mm_weight_t h, void* stream);
 int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns);
 
 /*
+ * Failure-detection tests of the forward's own waits (test use only).  Each
+ * bit makes later forwards on the handle leave out one kind of arrival that
+ * another part of the GPU waits for, and changes nothing else (no address,
+ * load or store): the bounded wait then runs out as it would if that
+ * arrival were lost, the kernels drain what they have in flight and exit,
+ * and int8mm_get_status reports INT8MM_ERR_TIMEOUT and resets the counters.
+ * The outputs of such forwards are invalid.  0 (the default) turns them off.
+ *   INT8MM_TEST_SKIP_SPLITK_TICKET    split-K pieces of the prefill GEMM do
+ *                                     not count themselves on the ticket the
+ *                                     tile's owner waits for;
+ *   INT8MM_TEST_SKIP_DECODE_TICKET    split n blocks of the decode GEMM (M <=
+ *                                     64) likewise;
+ *   INT8MM_TEST_SKIP_BARRIER_ARRIVAL  block 0 of the single-launch activation
+ *                                     pass does not arrive at its grid barrier.
+ * INT8MM_ERR_INVALID_ARG for other bits.
+ */
+#define INT8MM_TEST_SKIP_SPLITK_TICKET 1
+#define INT8MM_TEST_SKIP_DECODE_TICKET 2
+#define INT8MM_TEST_SKIP_BARRIER_ARRIVAL 4
+int8mm_status int8mm_set_test_skip(int8mm_weight_t h, int bits);
+
+/*
  * Split of the prefill GEMM along K (forwards with M > 128, whose 256 x 256
  * output tiles are computed by pairs of SMs).  0 (the default) lets the
  * library choose: it cuts each tile's K range into the S in 1..4 pieces that

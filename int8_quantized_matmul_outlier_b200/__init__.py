@@ -47,6 +47,7 @@ SIGNATURES = {
     "int8mm_set_wait_limit": (_ST, [_P, ctypes.c_uint64]),
     "int8mm_set_split_k": (_ST, [_P, ctypes.c_int]),
     "int8mm_wait_selftest": (_ST, [_P, _P]),
+    "int8mm_set_test_skip": (_ST, [_P, ctypes.c_int]),
     "int8mm_prepare_weight_static": (_ST, [_P, _I64, _I64, _P, _I64, ctypes.c_int, _P, ctypes.POINTER(_P)]),
     "int8mm_weight_bytes": (_ST, [_P, ctypes.POINTER(ctypes.c_size_t)]),
     "int8mm_launches_per_forward": (_ST, [_P, _I64, ctypes.POINTER(ctypes.c_int)]),
@@ -278,6 +279,17 @@ def int8mm_wait_selftest(w: Weight, stream=None) -> None:
     after the handle's wait limit and leaves INT8MM_ERR_TIMEOUT for
     int8mm_get_status."""
     _check(lib().int8mm_wait_selftest(w.handle, _stream(stream)))
+
+
+INT8MM_TEST_SKIP_SPLITK_TICKET = 1
+INT8MM_TEST_SKIP_DECODE_TICKET = 2
+INT8MM_TEST_SKIP_BARRIER_ARRIVAL = 4
+
+
+def int8mm_set_test_skip(w: Weight, bits: int) -> None:
+    """Failure-detection tests only: later forwards leave out the arrivals
+    named by `bits` (INT8MM_TEST_SKIP_*), so a device wait runs out."""
+    _check(lib().int8mm_set_test_skip(w.handle, int(bits)))
 
 
 def int8mm_set_split_k(w: Weight, split: int) -> None:

@@ -32,8 +32,7 @@ struct int8mm_weight {
   float* c_w = nullptr;       // [N]
   float* inv_cw = nullptr;    // [N]
   uint32_t* colmax_bits = nullptr;  // [N] prep scratch
-  CUtensorMap tmB;     // Wb, 256-row boxes (prefill GEMM operand B)
-  CUtensorMap tmW128;  // Wb, 128-row boxes (decode GEMM operand A)
+  CUtensorMap tmW128;  // Wb, 128-row boxes (operand B of the prefill GEMM, A of the decode GEMM)
   // decode (M <= 64) scratch: int32 partial sums and per-n-block tickets
   int32_t* part = nullptr;
   unsigned* dticket = nullptr;
@@ -84,6 +83,7 @@ struct int8mm_weight {
   int32_t* count_w = nullptr;  // [1] min(|O|, out_cap)
   uint32_t* never_set = nullptr;  // [1] zero: the flag of the wait self-test
   unsigned long long timeout_ns = 2000000000ull;
+  int test_skip = 0;  // INT8MM_TEST_SKIP_* bits (failure-detection tests only)
   size_t bytes = 0;
 };
 
@@ -200,10 +200,14 @@ void free_all(int8mm_weight* h) {
   release(&h->never_set);
 }
 
+// Row stride of X_OT for M rows: a multiple of 8, so that the GEMM reads
+// 8 rows of an outlier column with one 16-byte load.
+int64_t xot_stride(int64_t M) { return (M + 7) / 8 * 8; }
+
 size_t ws_bytes(const int8mm_weight* h, int64_t rows) {
-  return static_cast<size_t>(rows) * h->K                  // Xq
-         + static_cast<size_t>(rows) * 4                   // c_x
-         + static_cast<size_t>(rows) * h->K * 2;           // X_OT
+  return static_cast<size_t>(rows) * h->K                       // Xq
+         + static_cast<size_t>(rows) * 4                        // c_x
+         + static_cast<size_t>(xot_stride(rows)) * h->K * 2;    // X_OT
 }
 
 int8mm_status ensure_workspace(int8mm_weight* h, int64_t M, cudaStream_t s) {
@@ -225,7 +229,7 @@ int8mm_status ensure_workspace(int8mm_weight* h, int64_t M, cudaStream_t s) {
   cudaError_t e;
   if ((e = alloc(&h->Xq, static_cast<size_t>(rows) * h->K, s, nullptr)) != cudaSuccess ||
       (e = alloc(&h->c_x, static_cast<size_t>(rows), s, nullptr)) != cudaSuccess ||
-      (e = alloc(&h->X_OT, static_cast<size_t>(rows) * h->K, s, nullptr)) != cudaSuccess) {
+      (e = alloc(&h->X_OT, static_cast<size_t>(xot_stride(rows)) * h->K, s, nullptr)) != cudaSuccess) {
     cudaStreamSynchronize(s);
     free_workspace(h);
     return cuda_fail(e, "workspace allocation");
@@ -255,9 +259,8 @@ int8mm_status ensure_decode_scratch(int8mm_weight* h, cudaStream_t s) {
   return INT8MM_OK;
 }
 
-// Pieces along K of the prefill GEMM for M rows (1 for single-CTA tiles).
+// Pieces along K of the prefill GEMM for M rows.
 int split_for(const int8mm_weight* h, int64_t M) {
-  if (M <= kGemmBM) return 1;
   const int64_t num_kb = (h->K + kGemmBK - 1) / kGemmBK;
   return h->split_override > 0 ? static_cast<int>(std::min<int64_t>(h->split_override, num_kb))
                                : gemm_split_for(M, h->N, h->K, h->num_sms);
@@ -337,6 +340,7 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
   if ((st = set_device(h)) != INT8MM_OK) return st;
   if ((st = ensure_workspace(h, M, s)) != INT8MM_OK) return st;
   const bool decode = M <= kDecodeMaxM;
+  const int64_t ld_xo = xot_stride(M);
   const int box_rows = decode ? decode_padded_tokens(M) : kGemmBM;
   if (h->tmA_ptr != h->Xq || h->tmA_rows != M || h->tmA_box != box_rows) {
     if ((st = make_tmap_i8(&h->tmA, h->Xq, h->K, M, kGemmBK, box_rows)) != INT8MM_OK) return st;
@@ -353,8 +357,8 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
   };
   rec(0);
   if (decode && small_act_fits(M, h->K)) {
-    SmallActArgs sa{Xh, static_cast<int>(M), static_cast<int>(h->K), alpha, h->Xq, h->c_x, h->X_OT,
-                    h->colmax, h->idx, h->count};
+    SmallActArgs sa{Xh,    static_cast<int>(M), static_cast<int>(h->K), alpha,  h->Xq,   h->c_x,
+                    h->X_OT, static_cast<int>(ld_xo), h->colmax, h->idx, h->count};
     if ((e = launch_small_act(sa, s)) != cudaSuccess) return cuda_fail(e, "activation pass launch");
   } else if (!decode && row_act_fits(M, h->K, h->num_sms)) {
     RowActArgs ra;
@@ -369,6 +373,7 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     ra.Xq = h->Xq;
     ra.c_x = h->c_x;
     ra.X_OT = h->X_OT;
+    ra.ld_xo = static_cast<int>(ld_xo);
     ra.idx = h->idx;
     ra.count = h->count;
     ra.omask = h->omask;
@@ -378,11 +383,12 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     ra.colmax = h->colmax;
     ra.status = h->status;
     ra.timeout_ns = h->timeout_ns;
+    ra.skip_arrival = (h->test_skip & INT8MM_TEST_SKIP_BARRIER_ARRIVAL) != 0;
     if ((e = launch_row_act(ra, h->num_sms, s)) != cudaSuccess) return cuda_fail(e, "activation pass launch");
   } else {
     if ((e = launch_outlier_detect(Xh, M, h->K, alpha, sc, s)) != cudaSuccess)
       return cuda_fail(e, "outlier detection launch");
-    if ((e = launch_row_quant(Xh, M, h->K, sc, h->Xq, h->c_x, h->X_OT, /*pdl=*/true, s)) != cudaSuccess)
+    if ((e = launch_row_quant(Xh, M, h->K, sc, h->Xq, h->c_x, h->X_OT, ld_xo, /*pdl=*/true, s)) != cudaSuccess)
       return cuda_fail(e, "row quantisation launch");
   }
   if (h->wstatic) {
@@ -407,10 +413,12 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     d.N = static_cast<int>(h->N);
     d.K = static_cast<int>(h->K);
     d.N_pad = static_cast<int>(h->N_pad);
+    d.Wb = h->Wb;
     d.c_x = h->c_x;
     d.inv_cw = h->inv_cw;
     d.W = Wrows;
     d.X_OT = h->X_OT;
+    d.ld_xo = static_cast<int>(ld_xo);
     d.idx = widx;
     d.count = wcount;
     d.Y = static_cast<__half*>(Y);
@@ -420,6 +428,7 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     d.ticket = h->dticket;
     d.status = h->status;
     d.timeout_ns = h->timeout_ns;
+    d.skip_arrival = (h->test_skip & INT8MM_TEST_SKIP_DECODE_TICKET) != 0;
     if ((e = launch_gemm_decode(h->tmW128, h->tmA, d, h->num_sms, pdl, s)) != cudaSuccess)
       return cuda_fail(e, "int8 decode GEMM launch");
   } else {
@@ -440,6 +449,7 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     a.inv_cw = h->inv_cw;
     a.W = Wrows;
     a.X_OT = h->X_OT;
+    a.ld_xo = static_cast<int>(ld_xo);
     a.idx = widx;
     a.count = wcount;
     a.Y = static_cast<__half*>(Y);
@@ -450,7 +460,8 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     a.sk_ticket = h->sk_ticket;
     a.status = h->status;
     a.timeout_ns = h->timeout_ns;
-    if ((e = launch_gemm_decomp(h->tmA, h->tmB, h->tmW128, a, h->num_sms, pdl, s)) != cudaSuccess)
+    a.skip_arrival = (h->test_skip & INT8MM_TEST_SKIP_SPLITK_TICKET) != 0;
+    if ((e = launch_gemm_decomp(h->tmA, h->tmW128, a, h->num_sms, pdl, s)) != cudaSuccess)
       return cuda_fail(e, "int8 GEMM launch");
   }
   rec(2);
@@ -549,8 +560,7 @@ int8mm_status prepare_impl(const void* W_fp16_dev, int64_t K, int64_t N, void* s
     return cuda_fail(e, "weight preparation");
   }
   const uint64_t wb_rows = kblocks * static_cast<uint64_t>(h->N_pad);
-  int8mm_status st = make_tmap_i8(&h->tmB, h->Wb, 128, wb_rows, kGemmBK, kGemmBN);
-  if (st == INT8MM_OK) st = make_tmap_i8(&h->tmW128, h->Wb, 128, wb_rows, kGemmBK, 128);
+  int8mm_status st = make_tmap_i8(&h->tmW128, h->Wb, 128, wb_rows, kGemmBK, 128);
   if (st == INT8MM_OK && wstatic) {
     // the stored rows and the row map; W is not kept
     std::vector<int32_t> wmap(Kz, -1), iota(static_cast<size_t>(max_outliers));
@@ -632,6 +642,7 @@ int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream) {
   size_t ws_max = 0, tickets_max = 0;
   for (int64_t mt = 1; (mt - 1) * 2 * kGemmBM < M_max; ++mt) {
     const int64_t M = std::min<int64_t>(M_max, mt * 2 * kGemmBM);
+    if (M <= kDecodeMaxM) continue;  // the decode GEMM: no split
     const int split = split_for(h, M);
     if (split > 1) {
       const size_t tiles = pair_tiles(h, M);
@@ -760,6 +771,14 @@ int8mm_status int8mm_wait_selftest(int8mm_weight_t h, void* stream) {
   }
   if ((e = launch_wait_selftest(h->never_set, h->status, h->timeout_ns, s)) != cudaSuccess)
     return cuda_fail(e, "wait self-test launch");
+  return INT8MM_OK;
+}
+
+int8mm_status int8mm_set_test_skip(int8mm_weight_t h, int bits) {
+  if (!live(h)) return fail(INT8MM_ERR_INVALID_ARG, "invalid or freed weight handle");
+  const int all = INT8MM_TEST_SKIP_SPLITK_TICKET | INT8MM_TEST_SKIP_DECODE_TICKET | INT8MM_TEST_SKIP_BARRIER_ARRIVAL;
+  if ((bits & ~all) != 0) return fail(INT8MM_ERR_INVALID_ARG, "unknown test bits 0x%x", bits);
+  h->test_skip = bits;
   return INT8MM_OK;
 }
 

@@ -12,45 +12,46 @@
 // int8 cuBLAS GEMM followed by a separate fp16 GEMM; here both, and the
 // dequantisation, run in one persistent kernel.
 //
-// Structure (one CTA per SM, 10 warps):
-//   warp 0      TMA producer: 128x128 A tiles (Xq) and B tiles (Wq, K-blocked),
-//               128-byte swizzled, into a STAGES-deep shared-memory ring;
-//   warp 1      allocates 512 TMEM columns; one thread issues
+// Structure: clusters of two CTAs on neighbouring SMs (a CTA pair), one CTA
+// per SM, 10 warps each.  A pair computes a 256x256 output tile with
+// tcgen05.mma.cta_group::2 (256x256x32 int8) issued by the leader (rank 0);
+// each CTA loads its own 128 rows of A and 128 rows of B (TMA completing on
+// the leader's barrier), keeps its 128 accumulator rows in its own TMEM and
+// writes them; commits reach both CTAs' barriers.  Each SM streams 32 KB per
+// 128x256x128 of MMA work through a 6-stage ring.  No TMA multicast is used.
+//   warp 0      TMA producer: 128x128 A tiles (Xq) and B tiles (Wq,
+//               K-blocked), 128-byte swizzled;
+//   warp 1      allocates 512 TMEM columns; in the leader one thread issues
 //               tcgen05.mma.kind::i8 into a double-buffered int32
 //               accumulator (2 x 256 columns);
 //   warps 2-9   epilogue, two warps per TMEM lane quarter (warp w reads lanes
 //               32*(w%4)..+31, one output row per thread), each covering one
 //               128-column half of the tile: tcgen05.ld of the accumulator,
-//               scale by 1/c_x and 1/c_w, add the fp16 outlier product, write
-//               fp16.
+//               scale by 1/c_x and 1/c_w, write fp16.
 // The epilogue of tile t overlaps the main loop of tile t+1.  Every wait is
 // bounded; a timeout sets the status word and the CTA drains and exits.
+// Problems of at most 128 rows use the same tiles: the peer's 128 rows lie
+// past M, where TMA fills zeros and nothing is stored.
 //
-// The outlier product X[:,O] W[O,:] (CTA pairs, the first kOutMma outliers)
-// runs on the tensor cores too.  While a tile accumulates, the epilogue warps
-// write its operand blocks into shared memory in the 128-byte-swizzled
-// K-major layout the int8 tiles use: X_O (this CTA's 128 rows x the outliers,
-// from X_OT) and W_O (its 128 columns x the outliers, from the rows W[O,:]).
-// Once the tile is done they write the dequantised tile back into TMEM as
-// fp32; the MMA warp adds X_O W_O^T onto it with tcgen05.mma.kind::f16
-// (K = 16 per step), between the int8 k-blocks of the next tile; the
-// epilogue reads the sums.  Single CTAs (M <= 128) and outliers past
-// kOutMma use CUDA-core FMAs in the epilogue (W rows staged in shared memory).
+// The outlier product X[:,O] W[O,:] runs on the tensor cores too, kOutMma
+// outliers at a time.  While a tile accumulates, the epilogue warps write the
+// first chunk of its operand blocks into shared memory in the
+// 128-byte-swizzled K-major layout the int8 tiles use: X_O (this CTA's 128
+// rows x the chunk's outliers, from X_OT) and W_O (its 128 columns x those
+// outliers, from the rows W[O,:]); both sources are o-major, so each thread
+// reads an 8 x 8 block with eight 16-byte loads and transposes it in
+// registers.  Once the tile is done they write the dequantised tile back
+// into TMEM as fp32; the MMA warp adds X_O W_O^T onto it with
+// tcgen05.mma.kind::f16 (K = 16 per step), between the int8 k-blocks of the
+// next tile.  With more than kOutMma outliers the epilogue stages the next
+// chunk as soon as the tensor cores are done with the blocks, and the MMA
+// warp picks it up after its next k-block.  The epilogue then reads the sums.
 //
-// Two modes.  Single CTA (M <= 128): 128x256 tiles, B tiles of 256 rows,
-// 4 stages.  CTA pair (M > 128): a cluster of two CTAs on neighbouring SMs
-// computes a 256x256 tile with tcgen05.mma.cta_group::2 (256x256x32) issued
-// by the leader; each CTA loads its own 128 rows of A and 128 rows of B
-// (TMA completing on the leader's barrier), keeps its 128 accumulator rows in
-// its own TMEM and writes them; commits reach both CTAs' barriers.  Each SM
-// then streams 32 KB instead of 48 KB per 128x256x128 of MMA work, in a
-// 6-stage ring.  No TMA multicast is used.
-//
-// Split K (CTA pairs, when the tiles fill the pairs' rounds badly, e.g. 160
-// tiles of a K-heavy FFN contraction for 74 pairs): every tile is cut into S
-// equal ranges of k-blocks, and the S x tiles work units are dealt to the
-// pairs piece-major (all first pieces, then all second pieces, ...), so the
-// pairs of one round read the same k-slices and keep sharing them in L2.
+// Split K (when the tiles fill the pairs' rounds badly, e.g. 160 tiles of a
+// K-heavy FFN contraction for 74 pairs): every tile is cut into S equal
+// ranges of k-blocks, and the S x tiles work units are dealt to the pairs
+// piece-major (all first pieces, then all second pieces, ...), so the pairs
+// of one round read the same k-slices and keep sharing them in L2.
 // The last piece owns the tile.  The other pieces store their exact int32
 // partial tiles in a workspace and count themselves on the tile's tickets
 // (one per CTA and 128-column half); the owner waits (bounded) for its
@@ -58,8 +59,7 @@
 // dequantising, resets the ticket and finishes the tile as an unsplit one.
 // A pair deals with all its non-owner units before any owner unit, and
 // non-owner units wait on nothing, so every wait ends once all pairs are
-// resident (one pair per two SMs, as for the unsplit kernel; the wait is
-// bounded all the same).
+// resident (one pair per two SMs; the wait is bounded all the same).
 // Integer sums make the result independent of the split.
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -70,50 +70,41 @@ namespace i8mm {
 namespace {
 
 constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK;
-constexpr int A_BYTES = BM * BK;  // 16 KB: 128 rows of A per CTA
-// Epilogue staging: per 128-column half of the tile, the first OUT_CAP
-// outlier rows W[idx[o], cols] and 1/c_w[cols] as fp32.
+constexpr int A_BYTES = BM * BK;   // 16 KB: 128 rows of A per CTA
+constexpr int B_ROWS = BN / 2;     // rows of B per CTA
+constexpr int B_BYTES = B_ROWS * BK;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int STAGES = 6;
+constexpr int TILE_M = 2 * BM;     // rows per tile
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int HALF_N = BN / 2;
-constexpr int OUT_CAP = 16;
 // The outlier product of tile t is issued after this many int8 k-blocks of
 // tile t+1 (by then the epilogue has written tile t back to TMEM), splitting
 // the k-block loop in two tight loops.
 constexpr int OUT_ISSUE_KB = 16;
-constexpr int WO_BYTES = 2 * OUT_CAP * HALF_N * 4;
-constexpr int RW_BYTES = 2 * HALF_N * 4;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 static_assert(TMEM_COLS == 512, "two 128x256 int32 accumulators fill TMEM");
 
-// Single CTA: 128x256 tile, 4 stages of A (16 KB) + B (32 KB).  CTA pair:
-// 256x256 tile, each CTA holding 128 rows of A and 128 rows of B, 6 stages
-// of 32 KB: a third less operand traffic per SM for the same MMA work.
-template <bool PAIR>
-struct Cfg {
-  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // rows of B per CTA
-  static constexpr int B_BYTES = B_ROWS * BK;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = PAIR ? 6 : 4;
-  static constexpr int TILE_M = PAIR ? 2 * BM : BM;  // rows per tile
-  static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
-  // full, empty, tmem_full[2], tmem_empty[2], drain, and for the outlier
-  // product: tile dequantised (operands staged)[2], product done[2]
-  static constexpr int NUM_BARS = 2 * STAGES + 5 + 4;
-  static constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
-  // pairs: the outlier product's operand blocks (128 rows of 128 bytes each:
-  // up to 64 fp16 outliers for 128 rows of X_O, and for 128 columns of W_O);
-  // single CTAs: the staged outlier weight rows
-  static constexpr int OA_OFFSET = (MISC_OFFSET + 16 + 1023) & ~1023;
-  static constexpr int OB_OFFSET = OA_OFFSET + (PAIR ? A_BYTES : 0);
-  static constexpr int WO_OFFSET = OB_OFFSET + (PAIR ? A_BYTES : 0);
-  static constexpr int RW_OFFSET = WO_OFFSET + (PAIR ? 0 : WO_BYTES);
-  static constexpr int SMEM_BYTES = RW_OFFSET + RW_BYTES + 1024;  // + slack to align the base to 1024
-  static constexpr uint32_t IDESC_F16 = idesc_f16_f32(TILE_M, BN);
-  static constexpr uint32_t IDESC = idesc_i8(TILE_M, BN);
-  static_assert(SMEM_BYTES <= 232448, "fits the 227 KB of shared memory per block");
-  static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-byte aligned for the 128B swizzle");
-};
+// Shared memory: the ring of 6 stages (A 16 KB + B 16 KB), the barriers:
+// full, empty, tmem_full[2], tmem_empty[2], drain, and for the outlier
+// product: tile dequantised (operands staged)[2], product done[2]; then the
+// outlier product's operand blocks (128 rows of 128 bytes each: up to 64
+// fp16 outliers for 128 rows of X_O, and for 128 columns of W_O) and 1/c_w of
+// the tile's columns.
+constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
+constexpr int NUM_BARS = 2 * STAGES + 5 + 4;
+constexpr int MISC_OFFSET = BAR_OFFSET + NUM_BARS * 8;
+constexpr int OA_OFFSET = (MISC_OFFSET + 16 + 1023) & ~1023;
+constexpr int OB_OFFSET = OA_OFFSET + A_BYTES;
+constexpr int RW_OFFSET = OB_OFFSET + A_BYTES;
+constexpr int RW_BYTES = 2 * HALF_N * 4;
+constexpr int SMEM_BYTES = RW_OFFSET + RW_BYTES + 1024;  // + slack to align the base to 1024
+constexpr uint32_t IDESC_F16 = idesc_f16_f32(TILE_M, BN);
+constexpr uint32_t IDESC = idesc_i8(TILE_M, BN);
+static_assert(SMEM_BYTES <= 232448, "fits the 227 KB of shared memory per block");
+static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-byte aligned for the 128B swizzle");
+static_assert(kOutMma == 64, "a chunk of outliers fills one 128-byte operand row");
 
 __device__ __forceinline__ void fail(const GemmArgs& a, volatile int* abort_flag) {
   *abort_flag = 1;
@@ -165,6 +156,23 @@ __device__ __forceinline__ void load_bias32(const __half* bias, int n, bool full
   }
 }
 
+// 8 x 8 transpose of 16-bit values: v[r] holds row r (8 values, two per
+// word); on return t[c] holds column c, i.e. element r of row c is value c of
+// v[r].
+__device__ __forceinline__ void transpose8x8_b16(const uint4 (&v)[8], uint4 (&t)[8]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t sel = (c & 1) ? 0x7632u : 0x5410u;  // high or low halves of the two words
+    uint32_t w[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const uint32_t a = (&v[2 * p].x)[c >> 1], b = (&v[2 * p + 1].x)[c >> 1];
+      w[p] = __byte_perm(a, b, sel);
+    }
+    t[c] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 // One work unit: k-blocks [kb0, kb1) of a tile; piece S-1 finishes the tile.
 struct Unit {
   int tile, piece, kb0, kb1;
@@ -181,36 +189,32 @@ __device__ __forceinline__ Unit unit_at(int u, int num_tiles, int num_kb, int sp
   return w;
 }
 
-// BIAS: the layer bias is added; SPLIT: split K (CTA pairs only).  Separate
-// instantiations, so that the common path carries none of their code.
-template <bool PAIR, bool BIAS, bool SPLIT>
+// BIAS: the layer bias is added; SPLIT: split K.  Separate instantiations,
+// so that the common path carries none of their code.
+template <bool BIAS, bool SPLIT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_i8_decomp_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const GemmArgs a) {
-  static_assert(PAIR || !SPLIT, "split K is implemented for CTA pairs");
-  using C = Cfg<PAIR>;
-  constexpr int STAGES = C::STAGES;
-  constexpr int STAGE_BYTES = C::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFFSET);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFFSET);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* tdeq = drain + 1;  // [2] operands staged and tile dequantised into TMEM (leader)
   uint64_t* tout = tdeq + 2;   // [2] outlier product added
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFFSET);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFFSET + 4);
-  volatile int* part_ok = reinterpret_cast<volatile int*>(smem + C::MISC_OFFSET + 8);  // [2] per half
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFFSET);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + MISC_OFFSET + 4);
+  volatile int* part_ok = reinterpret_cast<volatile int*>(smem + MISC_OFFSET + 8);  // [2] per half
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = a.M, N = a.N, K = a.K;
   // a pair of CTAs (a cluster of 2) shares each tile; rank 0 issues the MMAs
-  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
-  const int tile0 = PAIR ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
-  const int tstride = PAIR ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
-  const int num_m = (M + C::TILE_M - 1) / C::TILE_M;
+  const uint32_t rank = cluster_ctarank();
+  const int tile0 = static_cast<int>(blockIdx.x) / 2;
+  const int tstride = static_cast<int>(gridDim.x) / 2;
+  const int num_m = (M + TILE_M - 1) / TILE_M;
   const int num_n = (N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = (K + BK - 1) / BK;
@@ -224,31 +228,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], NUM_EPI_WARPS * (PAIR ? 2 : 1));
+      mbar_init(&tempty[b], NUM_EPI_WARPS * 2);
     }
     mbar_init(drain, 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&tdeq[b], NUM_EPI_WARPS * (PAIR ? 2 : 1));
+      mbar_init(&tdeq[b], NUM_EPI_WARPS * 2);
       mbar_init(&tout[b], 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-
   }
   if (warp == 1) {
-    if (PAIR) {
-      tmem_alloc_pair(tmem_slot, TMEM_COLS);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(tmem_slot, TMEM_COLS);
-      tmem_relinquish();
-    }
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  if (PAIR) cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
-  else __syncthreads();
+  cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const unsigned long long tmo = a.timeout_ns;
@@ -260,21 +257,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_phase = 0;
       bool ok = true;
-      // In a pair both CTAs' loads complete on the leader's full barrier, and
-      // the leader alone announces the pair's bytes.
+      // Both CTAs' loads complete on the leader's full barrier, and the
+      // leader alone announces the pair's bytes.
       auto full_of = [&](int st) { return mapa_shared(smem_u32(&full[st]), 0); };
       auto expect = [&](int st) {
-        if (!PAIR || rank == 0) mbar_arrive_expect_tx(&full[st], (PAIR ? 2 : 1) * STAGE_BYTES);
+        if (rank == 0) mbar_arrive_expect_tx(&full[st], 2 * STAGE_BYTES);
       };
       auto load_a = [&](int st, int kb, int m_blk) {
-        const int row = m_blk * C::TILE_M + static_cast<int>(rank) * BM;
-        if (PAIR) tma_load_2d_pair(smem + st * STAGE_BYTES, &tmA, full_of(st), kb * BK, row);
-        else tma_load_2d(smem + st * STAGE_BYTES, &tmA, &full[st], kb * BK, row);
+        const int row = m_blk * TILE_M + static_cast<int>(rank) * BM;
+        tma_load_2d_pair(smem + st * STAGE_BYTES, &tmA, full_of(st), kb * BK, row);
       };
       auto load_b = [&](int st, int kb, int n_blk) {
-        const int row = kb * a.N_pad + n_blk * BN + static_cast<int>(rank) * C::B_ROWS;
-        if (PAIR) tma_load_2d_pair(smem + st * STAGE_BYTES + A_BYTES, &tmB, full_of(st), 0, row);
-        else tma_load_2d(smem + st * STAGE_BYTES + A_BYTES, &tmB, &full[st], 0, row);
+        const int row = kb * a.N_pad + n_blk * BN + static_cast<int>(rank) * B_ROWS;
+        tma_load_2d_pair(smem + st * STAGE_BYTES + A_BYTES, &tmB, full_of(st), 0, row);
       };
       // The weight tiles of the first k-blocks do not depend on the
       // activation pass: issue them before waiting for it, then the
@@ -313,9 +308,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok) {
         fail(a, abort_flag);
-        // Let every load already issued land before the CTA can exit (a
-        // pair's peer cannot watch the leader's barriers: it waits a while).
-        if (!PAIR || rank == 0) {
+        // Let every load already issued land before the CTA can exit (the
+        // peer cannot watch the leader's barriers: it waits a while).
+        if (rank == 0) {
           for (int s = 0; s < STAGES; ++s)
             if (issued_mask & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, tmo, nullptr);
         } else {
@@ -326,36 +321,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && (!PAIR || rank == 0)) {
+    if (lane == 0 && rank == 0) {
       // -------------------------------------------------------- MMA issuer
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int lt = 0;
-      // Outlier product of a finished tile (pairs with |O| > 0): once the
-      // epilogue has staged the operand blocks and written the dequantised
-      // tile back to TMEM, D += X_O W_O^T in min(|O|, 64)/16 steps of K = 16,
-      // issued after OUT_ISSUE_KB int8 k-blocks of the next tile.
+      // Outlier product of a finished tile: once the epilogue has staged a
+      // chunk of operand blocks (and, for the first, written the dequantised
+      // tile back to TMEM), D += X_O W_O^T in up to 64/16 steps of K = 16;
+      // the first chunk after OUT_ISSUE_KB int8 k-blocks of the next tile.
       pdl_wait();
-      const int cnt = PAIR ? *a.count : 0;
-      const int nk = cnt > 0 ? (min(cnt, kOutMma) + 15) / 16 : 0;
-      uint32_t pend_use = 0;
-      // with split K, tdeq/tout complete only for units that finish a tile:
-      // their phases count those uses of each buffer
-      uint32_t fin_uses[2] = {0u, 0u};
-      int pend = -1;  // accumulator buffer whose outlier product is due
-      auto issue_outl = [&]() -> bool {
-        if (!mbar_wait(&tdeq[pend], pend_use & 1u, tmo, abort_flag)) return false;
+      const int cnt = *a.count;
+      const int nchunks = (cnt + kOutMma - 1) / kOutMma;
+      // tdeq/tout phases used so far per accumulator buffer: one per chunk of
+      // every tile whose product ran there (with split K only units that
+      // finish a tile have one)
+      uint32_t chunk_ph[2] = {0u, 0u};
+      int pend = -1;        // accumulator buffer whose outlier product is due
+      int pend_chunk = 0;   // its next chunk
+      uint32_t pend_base = 0;
+      // Issues the next chunk of the pending product once the epilogue has
+      // staged it.  `block`: wait for that (bounded); otherwise only look.
+      // Returns 1 when issued, 0 when not ready yet, -1 after a timeout.
+      auto issue_chunk = [&](bool block) -> int {
+        const uint32_t par = (pend_base + static_cast<uint32_t>(pend_chunk)) & 1u;
+        if (block) {
+          if (!mbar_wait(&tdeq[pend], par, tmo, abort_flag)) return -1;
+        } else if (!mbar_try_wait(&tdeq[pend], par)) {
+          return 0;
+        }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(pend * BN);
-        const uint64_t adesc = smem_desc_k_sw128(smem_u32(smem + C::OA_OFFSET));
-        const uint64_t bdesc = smem_desc_k_sw128(smem_u32(smem + C::OB_OFFSET));
+        const uint64_t adesc = smem_desc_k_sw128(smem_u32(smem + OA_OFFSET));
+        const uint64_t bdesc = smem_desc_k_sw128(smem_u32(smem + OB_OFFSET));
+        const int nk = (min(cnt - pend_chunk * kOutMma, kOutMma) + 15) / 16;
         for (int kk = 0; kk < nk; ++kk)  // 32 bytes (16 fp16) along K per step
           mma_f16_pair(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2),
-                       C::IDESC_F16, 1u);
+                       IDESC_F16, 1u);
         mma_commit_pair(&tout[pend], 0x3);
-        pend = -1;
-        return true;
+        if (++pend_chunk == nchunks) pend = -1;
+        return 1;
       };
       for (int u = tile0; u < num_units && ok; u += tstride, ++lt) {
         const Unit w = unit_at<SPLIT>(u, num_tiles, num_kb, S);
@@ -374,18 +380,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t adesc = smem_desc_k_sw128(sa);
           const uint64_t bdesc = smem_desc_k_sw128(sa + A_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 32; ++kk) {
-            // advance 32 bytes along K inside the 128-byte swizzled row
-            const uint32_t acc = (kb != w.kb0 || kk != 0) ? 1u : 0u;
-            if (PAIR)
-              mma_i8_pair(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2),
-                          C::IDESC, acc);
-            else
-              mma_i8(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), C::IDESC,
-                     acc);
-          }
-          if (PAIR) mma_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
-          else mma_commit(&empty[stage]);
+          for (int kk = 0; kk < BK / 32; ++kk)  // advance 32 bytes along K inside the 128-byte swizzled row
+            mma_i8_pair(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), IDESC,
+                        (kb != w.kb0 || kk != 0) ? 1u : 0u);
+          mma_commit_pair(&empty[stage], 0x3);  // frees the stage in both CTAs
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -393,23 +391,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           return true;
         };
         const int ksplit = pend >= 0 ? min(w.kb1, w.kb0 + OUT_ISSUE_KB) : w.kb1;
-        for (int kb = w.kb0; kb < ksplit && ok; ++kb) ok = kblock(kb);
-        if (ok && pend >= 0) ok = issue_outl();
-        for (int kb = ksplit; kb < w.kb1 && ok; ++kb) ok = kblock(kb);
-        if (ok) {
-          if (PAIR) mma_commit_pair(&tfull[buf], 0x3);
-          else mma_commit(&tfull[buf]);
+        int kb = w.kb0;
+        for (; kb < ksplit && ok; ++kb) ok = kblock(kb);
+        if (ok && pend >= 0) ok = issue_chunk(true) > 0;
+        // more than kOutMma outliers: the later chunks go in as soon as the
+        // epilogue has staged them, looked for after every k-block
+        for (; kb < w.kb1 && ok && pend >= 0; ++kb) {
+          ok = kblock(kb);
+          if (ok) ok = issue_chunk(false) >= 0;
         }
-        if (nk > 0 && w.piece == S - 1) {  // the tile is complete: its outlier product is due
+        for (; kb < w.kb1 && ok; ++kb) ok = kblock(kb);
+        if (ok) mma_commit_pair(&tfull[buf], 0x3);
+        // the previous tile's product is complete before this one's is due
+        while (ok && pend >= 0) ok = issue_chunk(true) > 0;
+        if (nchunks > 0 && w.piece == S - 1) {  // the tile is complete: its outlier product is due
           pend = buf;
-          pend_use = SPLIT ? fin_uses[buf]++ : use;
+          pend_chunk = 0;
+          pend_base = chunk_ph[buf];
+          chunk_ph[buf] += static_cast<uint32_t>(nchunks);
         }
       }
-      if (ok && pend >= 0) ok = issue_outl();
+      while (ok && pend >= 0) ok = issue_chunk(true) > 0;
       if (!ok) {
         fail(a, abort_flag);
-        if (PAIR) mma_commit_pair(drain, 0x1);
-        else mma_commit(drain);
+        mma_commit_pair(drain, 0x1);
         mbar_wait(drain, 0, tmo, nullptr);
       }
     }
@@ -422,19 +427,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row_t = q * 32 + lane;
     pdl_wait();  // count, idx, X_OT and c_x come from the activation pass
     const int cnt = *a.count;
-    // pairs: the first kOutMma outliers are added on the tensor cores; single
-    // CTAs: the first OUT_CAP outliers from staged weight rows; both: any
-    // further outliers from global memory
-    const bool outl = PAIR && cnt > 0;
-    const int cs = PAIR ? 0 : min(cnt, OUT_CAP);  // outliers staged in shared memory
-    const int o_tail = PAIR ? kOutMma : OUT_CAP;
-    float* wo = reinterpret_cast<float*>(smem + C::WO_OFFSET) + h * OUT_CAP * HALF_N;  // [OUT_CAP][HALF_N]
-    float* rws = reinterpret_cast<float*>(smem + C::RW_OFFSET) + h * HALF_N;           // [HALF_N]
+    const int nchunks = (cnt + kOutMma - 1) / kOutMma;
+    float* rws = reinterpret_cast<float*>(smem + RW_OFFSET) + h * HALF_N;  // [HALF_N]
     const uint32_t bar_id = 1 + h;
     const bool y32 = (reinterpret_cast<uintptr_t>(a.Y) & 31u) == 0;
     bool alive = true;
     int lt = 0;
-    uint32_t fin_uses[2] = {0u, 0u};  // units that finished a tile, per accumulator buffer
+    uint32_t chunk_ph[2] = {0u, 0u};  // tdeq/tout phases used per accumulator buffer (one per chunk)
+    // Stages this thread's share of the operand blocks for outliers
+    // [64 c, 64 c + 64) of tile (m_blk, n_blk): half 0 writes X_O (rows m of
+    // this CTA x outliers, from X_OT[o][m]), half 1 W_O (columns n x
+    // outliers, from W[O_o][n]).  Thread tl takes the 8 x 8 block of rows
+    // 8 (tl >> 3) .. +7 and outliers 8 (tl & 7) .. +7: eight 16-byte loads
+    // along the rows, transposed in registers into eight 16-byte pieces of
+    // the 128-byte-swizzled K-major layout (piece j of row r stored at piece
+    // j ^ (r % 8), groups of 8 rows 1024 bytes apart).  Only the outliers the
+    // product reads (whole K = 16 steps) are written; zero past |O| and
+    // past M or N.
+    auto stage_chunk = [&](int c, int m_blk, int n_blk) {
+      const int o0 = c * kOutMma;
+      const int no = min(cnt - o0, kOutMma);
+      const int og = tl & 7, rg = tl >> 3;  // outlier group, row group
+      if (og >= 2 * ((no + 15) / 16)) return;  // not read by the product
+      const int r0 = (h == 0 ? m_blk * TILE_M + static_cast<int>(rank) * BM
+                             : n_blk * BN + static_cast<int>(rank) * B_ROWS) + 8 * rg;
+      const int lim = h == 0 ? M : N;
+      uint4 v[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int o = 8 * og + r;
+        v[r] = make_uint4(0u, 0u, 0u, 0u);
+        if (o < no && r0 < lim) {
+          const __half* src = h == 0 ? a.X_OT + static_cast<size_t>(o0 + o) * a.ld_xo + r0
+                                     : a.W + static_cast<size_t>(__ldg(a.idx + o0 + o)) * N + r0;
+          v[r] = __ldg(reinterpret_cast<const uint4*>(src));
+        }
+      }
+      if (r0 + 8 > lim) {  // rows past M in the last group of X_O: zero them
+        const int keep = max(0, lim - r0);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          uint32_t* wv = &v[r].x;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (2 * e >= keep) wv[e] = 0u;
+            else if (2 * e + 1 >= keep) wv[e] &= 0xffffu;
+          }
+        }
+      }
+      uint4 t[8];
+      transpose8x8_b16(v, t);
+      uint8_t* blk = smem + (h == 0 ? OA_OFFSET : OB_OFFSET) + rg * 1024;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)  // row 8 rg + i of the block, outliers 8 og ..
+        *reinterpret_cast<uint4*>(blk + i * 128 + ((og ^ i) << 4)) = t[i];
+    };
+    // makes this warp's staged pieces visible to the tensor cores and
+    // counts it on the leader's tdeq barrier
+    auto hand_over = [&](int buf) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tdeq[buf]), 0));
+    };
     for (int u = tile0; u < num_units; u += tstride, ++lt) {
       const Unit w = unit_at<SPLIT>(u, num_tiles, num_kb, S);
       const int tile = w.tile;
@@ -442,69 +496,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // a unit that finishes its tile (always, without split K); the others
       // only hand their partial sums on
       const bool fin = !SPLIT || w.piece == S - 1;
-      const bool outl_u = outl && fin;
+      const bool outl_u = cnt > 0 && fin;
       const int buf = lt & 1;
       const uint32_t use = static_cast<uint32_t>(lt >> 1);
-      uint32_t fuse = use;  // phase of this buffer's tout barrier
-      if (SPLIT && fin) fuse = fin_uses[buf]++;
+      const uint32_t cbase = chunk_ph[buf];  // phase of this tile's first chunk
+      if (outl_u) chunk_ph[buf] += static_cast<uint32_t>(nchunks);
       const int nh = n_blk * BN + h * HALF_N;  // first column of this half
-      const int m = m_blk * C::TILE_M + static_cast<int>(rank) * BM + row_t;
+      const int m = m_blk * TILE_M + static_cast<int>(rank) * BM + row_t;
       const bool row_ok = m < M;
 
-      // (1) stage this tile's scales and outlier weight rows; this runs
-      //     while the tensor cores still accumulate the tile.
+      // (1) stage this tile's column scales and the first chunk of its
+      //     outlier-product operands while the tensor cores still accumulate
+      //     the tile (the previous tile's product has completed, waited for
+      //     below, so the blocks are free)
       named_bar_sync(bar_id, 128);  // readers of the previous tile are done
       if (fin && tl < HALF_N / 4) {
         const int n = nh + tl * 4;
         const float4 f = n < N ? __ldg(reinterpret_cast<const float4*>(a.inv_cw + n)) : make_float4(0.f, 0.f, 0.f, 0.f);
         reinterpret_cast<float4*>(rws)[tl] = f;
       }
-      for (int e = tl; e < cs * (HALF_N / 8); e += 128) {
-        const int o = e / (HALF_N / 8), part = e % (HALF_N / 8);
-        const int n = nh + part * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (n < N) v = __ldg(reinterpret_cast<const uint4*>(a.W + static_cast<size_t>(__ldg(a.idx + o)) * N + n));
-        const __half2* hv = reinterpret_cast<const __half2*>(&v);
-        const float2 f0 = __half22float2(hv[0]), f1 = __half22float2(hv[1]);
-        const float2 f2 = __half22float2(hv[2]), f3 = __half22float2(hv[3]);
-        float4* dst = reinterpret_cast<float4*>(wo + o * HALF_N + part * 8);
-        dst[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
-        dst[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
-      }
-      float xo[OUT_CAP];
-#pragma unroll
-      for (int o = 0; o < OUT_CAP; ++o)
-        xo[o] = (o < cs && row_ok) ? __half2float(a.X_OT[static_cast<size_t>(o) * M + m]) : 0.0f;
-      if (outl_u) {
-        // this tile's outlier-product operand blocks, as fp16 rows of the
-        // 128-byte-swizzled K-major layout (16-byte chunk c of row r stored at
-        // chunk c ^ (r % 8), groups of 8 rows 1024 bytes apart): half 0 writes
-        // row tl of X_O (X[m, O_o]), half 1 row tl of W_O (W[O_o, n]); only
-        // the chunks the product reads, zero past |O|.  The previous tile's
-        // product has completed (waited for below), so the blocks are free.
-        const int no = min(cnt, kOutMma), nch = 2 * ((no + 15) / 16);
-        uint8_t* rowp = smem + (h == 0 ? C::OA_OFFSET : C::OB_OFFSET) + (tl >> 3) * 1024 + (tl & 7) * 128;
-        const int mrow = m_blk * C::TILE_M + static_cast<int>(rank) * BM + tl;
-        const int ncol = n_blk * BN + static_cast<int>(rank) * C::B_ROWS + tl;
-        const bool ok_rc = h == 0 ? mrow < M : ncol < N;
-        const uint16_t* src = h == 0 ? reinterpret_cast<const uint16_t*>(a.X_OT) + mrow
-                                     : reinterpret_cast<const uint16_t*>(a.W) + ncol;
-        for (int c = 0; c < nch; ++c) {
-          uint32_t w2[4];
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            const int o = 8 * c + 2 * p;
-            uint32_t lo = 0u, hi = 0u;
-            if (ok_rc && o < no)
-              lo = __ldg(src + (h == 0 ? static_cast<size_t>(o) * M : static_cast<size_t>(__ldg(a.idx + o)) * N));
-            if (ok_rc && o + 1 < no)
-              hi = __ldg(src + (h == 0 ? static_cast<size_t>(o + 1) * M : static_cast<size_t>(__ldg(a.idx + o + 1)) * N));
-            w2[p] = lo | (hi << 16);
-          }
-          *reinterpret_cast<uint4*>(rowp + ((c ^ (tl & 7)) << 4)) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
-      }
+      if (outl_u) stage_chunk(0, m_blk, n_blk);
       float rx = 0.0f;
       if (row_ok) {
         const float c = a.c_x[m];
@@ -562,7 +573,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         __threadfence();
         named_bar_sync(bar_id, 128);
-        if (tl == 0) red_release_add_gpu(ticket, 1u);
+        if (tl == 0 && !a.skip_arrival) red_release_add_gpu(ticket, 1u);
         continue;
       }
       if (SPLIT) {
@@ -607,7 +618,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       if (outl_u) {
         // (3) dequantise in place (int32 -> fp32 in TMEM), hand the tile to
-        //     the MMA warp for the outlier product, and wait for it
+        //     the MMA warp for the outlier product, chunk by chunk, and wait
+        //     for it
 #pragma unroll 1
         for (int ch = 0; ch < HALF_N / 32; ++ch) {
           const int cl = ch * 32;
@@ -648,9 +660,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tdeq[buf]), 0));  // the leader's barrier
-        alive = __all_sync(0xffffffffu, mbar_wait(&tout[buf], fuse & 1u, tmo, abort_flag));
+        hand_over(buf);
+        // the other chunks: once the tensor cores are done with a chunk's
+        // operand blocks, stage the next one there and hand it over
+        for (int c = 1; c < nchunks && alive; ++c) {
+          alive = __all_sync(0xffffffffu, mbar_wait(&tout[buf], (cbase + c - 1) & 1u, tmo, abort_flag));
+          if (!alive) break;
+          stage_chunk(c, m_blk, n_blk);
+          hand_over(buf);
+        }
+        if (alive) alive = __all_sync(0xffffffffu, mbar_wait(&tout[buf], (cbase + nchunks - 1) & 1u, tmo, abort_flag));
         if (!alive) {
           if (lane == 0) fail(a, abort_flag);
           continue;
@@ -663,13 +682,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(cl), r);
         tmem_wait_ld();
-        if (ch == HALF_N / 32 - 1) {  // accumulator buffer no longer read: release it
+        if (ch == HALF_N / 32 - 1) {  // accumulator buffer no longer read: release it (the leader's barrier)
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));  // the leader's barrier
-            else mbar_arrive(&tempty[buf]);
-          }
+          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
         }
         const int n = nh + cl;
         if (n >= N) continue;  // warp-uniform
@@ -694,39 +710,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             load_bias32(a.bias, n, full32, bb);
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __fadd_rn(v[i], bb[i]);
-          }
-        }
-        // fp16 outlier product X[m, O] . W[O, n..n+31] with fp32 accumulation,
-        // in ascending order of O: staged rows first, then any beyond OUT_CAP.
-#pragma unroll
-        for (int o = 0; o < OUT_CAP; ++o) {
-          if (o < cs) {
-            const float4* w4 = reinterpret_cast<const float4*>(wo + o * HALF_N + cl);
-#pragma unroll
-            for (int t4 = 0; t4 < 8; ++t4) {
-              const float4 w = w4[t4];
-              v[4 * t4 + 0] = __fmaf_rn(xo[o], w.x, v[4 * t4 + 0]);
-              v[4 * t4 + 1] = __fmaf_rn(xo[o], w.y, v[4 * t4 + 1]);
-              v[4 * t4 + 2] = __fmaf_rn(xo[o], w.z, v[4 * t4 + 2]);
-              v[4 * t4 + 3] = __fmaf_rn(xo[o], w.w, v[4 * t4 + 3]);
-            }
-          }
-        }
-        for (int o = o_tail; o < cnt; ++o) {
-          const int j = __ldg(a.idx + o);
-          const float x1 = row_ok ? __half2float(a.X_OT[static_cast<size_t>(o) * M + m]) : 0.0f;
-          const uint4* wr = reinterpret_cast<const uint4*>(a.W + static_cast<size_t>(j) * N + n);
-          uint4 wv[4];
-          wv[0] = __ldg(wr);
-          wv[1] = __ldg(wr + 1);
-          wv[2] = full32 ? __ldg(wr + 2) : make_uint4(0, 0, 0, 0);
-          wv[3] = full32 ? __ldg(wr + 3) : make_uint4(0, 0, 0, 0);
-          const __half2* wh = reinterpret_cast<const __half2*>(wv);
-#pragma unroll
-          for (int p = 0; p < 16; ++p) {
-            const float2 f = __half22float2(wh[p]);
-            v[2 * p] = __fmaf_rn(x1, f.x, v[2 * p]);
-            v[2 * p + 1] = __fmaf_rn(x1, f.y, v[2 * p + 1]);
           }
         }
         if (row_ok) {
@@ -762,54 +745,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (PAIR) cluster_sync_all();  // no CTA leaves while its peer may still signal it
+  cluster_sync_all();  // no CTA leaves while its peer may still signal it
   if (warp == 1) {
     tc_fence_after();
-    if (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
-    else tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
-template <bool PAIR, bool BIAS, bool SPLIT>
+template <bool BIAS, bool SPLIT>
 cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms, bool pdl,
                      cudaStream_t stream) {
-  using C = Cfg<PAIR>;
-  auto kern = gemm_i8_decomp_kernel<PAIR, BIAS, SPLIT>;
+  auto kern = gemm_i8_decomp_kernel<BIAS, SPLIT>;
   static unsigned long long attr_set = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   const unsigned long long bit = 1ull << (dev & 63);
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attrs[2];
-  int n = 0;
-  if (PAIR) {
-    attrs[n].id = cudaLaunchAttributeClusterDimension;
-    attrs[n].val.clusterDim.x = 2;
-    attrs[n].val.clusterDim.y = 1;
-    attrs[n].val.clusterDim.z = 1;
-    ++n;
-  }
-  cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = stream;
-  cfg.attrs = attrs;
-  cfg.numAttrs = n;
   if (!(attr_set & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set |= bit;
   }
-  const int num_tiles = ((a.M + C::TILE_M - 1) / C::TILE_M) * ((a.N + BN - 1) / BN);
-  const int units_of_work = num_tiles * (SPLIT ? a.split : 1);
-  // one CTA (pair) per SM (pair of SMs), all resident at once: owners of
-  // split tiles wait on other pairs' pieces
-  const int slots = PAIR ? num_sms / 2 : num_sms;
-  cfg.gridDim = dim3(std::max(1, std::min(units_of_work, slots)) * (PAIR ? 2 : 1));
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attrs[2];
+  int n = 0;
+  attrs[n].id = cudaLaunchAttributeClusterDimension;
+  attrs[n].val.clusterDim.x = 2;
+  attrs[n].val.clusterDim.y = 1;
+  attrs[n].val.clusterDim.z = 1;
+  ++n;
   if (pdl) {
     attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attrs[n].val.programmaticStreamSerializationAllowed = 1;
     ++n;
   }
+  const int num_tiles = ((a.M + TILE_M - 1) / TILE_M) * ((a.N + BN - 1) / BN);
+  const int units_of_work = num_tiles * (SPLIT ? a.split : 1);
+  // one CTA pair per pair of SMs, all resident at once: owners of split
+  // tiles wait on other pairs' pieces
+  const int slots = num_sms / 2;
+  cfg.gridDim = dim3(std::max(1, std::min(units_of_work, slots)) * 2);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attrs;
   cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, a);
 }
@@ -817,8 +795,7 @@ cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmA
 }  // namespace
 
 int gemm_split_for(int64_t M, int64_t N, int64_t K, int num_sms) {
-  if (M <= BM) return 1;  // single CTAs: not split
-  const int64_t tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + BN - 1) / BN);
+  const int64_t tiles = ((M + TILE_M - 1) / TILE_M) * ((N + BN - 1) / BN);
   const int64_t pairs = std::max(1, num_sms / 2);
   const int64_t num_kb = (K + BK - 1) / BK;
   // time of the slowest pair, in k-blocks: rounds of units x (k-blocks per
@@ -835,18 +812,14 @@ int gemm_split_for(int64_t M, int64_t N, int64_t K, int num_sms) {
   return best;
 }
 
-cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB256, const CUtensorMap& tmB128,
-                               const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
-  // one 128-row tile height: single CTAs; taller problems: CTA pairs
+cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
+                               bool pdl, cudaStream_t stream) {
   const bool bias = a.bias != nullptr;
-  if (a.M <= BM)
-    return bias ? launch_t<false, true, false>(tmA, tmB256, a, num_sms, pdl, stream)
-                : launch_t<false, false, false>(tmA, tmB256, a, num_sms, pdl, stream);
   if (a.split > 1)
-    return bias ? launch_t<true, true, true>(tmA, tmB128, a, num_sms, pdl, stream)
-                : launch_t<true, false, true>(tmA, tmB128, a, num_sms, pdl, stream);
-  return bias ? launch_t<true, true, false>(tmA, tmB128, a, num_sms, pdl, stream)
-              : launch_t<true, false, false>(tmA, tmB128, a, num_sms, pdl, stream);
+    return bias ? launch_t<true, true>(tmA, tmB, a, num_sms, pdl, stream)
+                : launch_t<false, true>(tmA, tmB, a, num_sms, pdl, stream);
+  return bias ? launch_t<true, false>(tmA, tmB, a, num_sms, pdl, stream)
+              : launch_t<false, false>(tmA, tmB, a, num_sms, pdl, stream);
 }
 
 }  // namespace i8mm

@@ -42,7 +42,11 @@ constexpr int DBK = 128;  // K bytes per stage
 // Six stages of weight tiles in flight per SM measured faster than deeper
 // rings (4: slower, 11: 12% slower): more outstanding reads only congest HBM.
 constexpr int D_STAGES = 6;
-constexpr int D_OUT_STAGE = 64;  // outliers whose activations are staged in smem
+// Weight tiles past the ring that each CTA asks L2 to fetch while the
+// activation pass is still running (512 KB per CTA, 76 MB over 148 SMs):
+// the weight does not depend on it, so HBM keeps streaming meanwhile.
+constexpr int D_L2_PREFETCH = 32;
+constexpr int D_OUT_STAGE = 128;  // outliers whose activations (and indices) are staged in smem
 constexpr int D_EPI = 256;  // epilogue threads: eight warps
 constexpr int D_THREADS = 64 + D_EPI;
 
@@ -161,6 +165,13 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         mbar_arrive_expect_tx(&full[i], C::STAGE);
         tma_load_2d_hint(smem + i * C::STAGE, &tmW, &full[i], 0, kb * a.N_pad + nb * DBM, wpol);
       }
+      // the next tiles into L2 (each one contiguous 16 KB block of the K-blocked layout)
+      const long long pf_end = min(u_end, u_begin + pre + D_L2_PREFETCH);
+      for (long long uu = u_begin + pre; uu < pf_end; ++uu) {
+        const int nb = static_cast<int>(uu / num_kb), kb = static_cast<int>(uu % num_kb);
+        bulk_prefetch_l2(a.Wb + (static_cast<size_t>(kb) * a.N_pad + static_cast<size_t>(nb) * DBM) * DBK,
+                         C::W_BYTES);
+      }
       dpdl_wait();
       for (int i = 0; i < pre; ++i) {
         const int kb = static_cast<int>((u_begin + i) % num_kb);
@@ -251,7 +262,7 @@ __global__ void __launch_bounds__(D_THREADS, 1)
     const int cs = min(cnt, D_OUT_STAGE);
     for (int e = et; e < cs * M; e += D_EPI) {
       const int o = e / M, m = e % M;
-      xo_s[o * 64 + m] = a.X_OT[static_cast<size_t>(o) * M + m];
+      xo_s[o * 64 + m] = a.X_OT[static_cast<size_t>(o) * a.ld_xo + m];
     }
     for (int o = et; o < cs; o += D_EPI) idx_s[o] = a.idx[o];
     if (et < M) {
@@ -305,7 +316,7 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         }
         __threadfence();
         dbar_sync(1, D_EPI);
-        if (et == 0) atomicAdd(a.ticket + sg.nb, static_cast<unsigned>(sg.kb1 - sg.kb0));
+        if (et == 0 && !a.skip_arrival) atomicAdd(a.ticket + sg.nb, static_cast<unsigned>(sg.kb1 - sg.kb0));
         continue;
       }
       if (sg.kb1 != num_kb) {
@@ -362,15 +373,31 @@ __global__ void __launch_bounds__(D_THREADS, 1)
           for (int j = 0; j < HM; ++j)
             if (m0 + j < M) y[j] = __fmaf_rn(__half2float(xo_s[o * 64 + m0 + j]), wo[o], y[j]);
         }
-      for (int o = C::WCAP; o < cnt; ++o) {
-        const float w1 = __half2float(a.W[static_cast<size_t>(__ldg(a.idx + o)) * N + n]);
+      // outliers past WCAP: their weight values in batches (eight, four
+      // with 64 tokens, where registers are scarcer), the loads of a batch
+      // all in flight before its FMAs (still in ascending o)
+      constexpr int OB = MP >= 64 ? 4 : 8;
+      for (int o0 = C::WCAP; o0 < cnt; o0 += OB) {
+        float w8[OB];
 #pragma unroll
-        for (int j = 0; j < HM; ++j)
-          if (m0 + j < M) {
-            const float xo = o < cs ? __half2float(xo_s[o * 64 + m0 + j])
-                                    : __half2float(a.X_OT[static_cast<size_t>(o) * M + m0 + j]);
-            y[j] = __fmaf_rn(xo, w1, y[j]);
+        for (int u = 0; u < OB; ++u) {
+          const int o = o0 + u;
+          w8[u] = o < cnt ? __half2float(a.W[static_cast<size_t>(o < cs ? idx_s[o] : __ldg(a.idx + o)) * N + n])
+                          : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < OB; ++u) {
+          const int o = o0 + u;
+          if (o < cnt) {
+#pragma unroll
+            for (int j = 0; j < HM; ++j)
+              if (m0 + j < M) {
+                const float xo = o < cs ? __half2float(xo_s[o * 64 + m0 + j])
+                                        : __half2float(a.X_OT[static_cast<size_t>(o) * a.ld_xo + m0 + j]);
+                y[j] = __fmaf_rn(xo, w8[u], y[j]);
+              }
           }
+        }
       }
 #pragma unroll
       for (int j = 0; j < HM; ++j)

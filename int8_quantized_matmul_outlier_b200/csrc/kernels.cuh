@@ -13,9 +13,9 @@ namespace i8mm {
 // Status bits in the device status word.
 constexpr int kStatusTimeout = 1;
 
-// Outliers whose fp16 product the prefill GEMM (CTA pairs) computes on the
-// tensor cores (kind::f16, K = 16 per step, operand rows of 128 bytes); its
-// epilogue adds any further outliers with FMAs.
+// Outliers per chunk of the fp16 product that the prefill GEMM (CTA pairs)
+// computes on the tensor cores (kind::f16, K = 16 per step, operand rows of
+// 128 bytes); more outliers take more chunks.
 constexpr int kOutMma = 64;
 
 // Sets the message returned by int8mm_last_error() on this host thread.
@@ -53,11 +53,11 @@ cudaError_t launch_outlier_detect(const __half* X, int64_t M, int64_t K, float a
 
 // Pass 2: per row, absmax over non-outlier columns, c_x = 127/absmax, int8
 // codes (outlier columns 0), and the fp16 outlier values scattered as
-// X_OT[o][i] = X[i, idx[o]] (o-major, M entries per o).  With `pdl`,
-// launched as a programmatic dependent of pass 1: it loads its row of X
-// while that pass finishes.
+// X_OT[o][i] = X[i, idx[o]] (o-major, rows ld_xo entries apart).  With
+// `pdl`, launched as a programmatic dependent of pass 1: it loads its row of
+// X while that pass finishes.
 cudaError_t launch_row_quant(const __half* X, int64_t M, int64_t K, const OutlierScratch& s,
-                             int8_t* Xq, float* c_x, __half* X_OT, bool pdl, cudaStream_t stream);
+                             int8_t* Xq, float* c_x, __half* X_OT, int64_t ld_xo, bool pdl, cudaStream_t stream);
 
 // ---- fused tcgen05 GEMM ---------------------------------------------------
 struct GemmArgs {
@@ -66,7 +66,8 @@ struct GemmArgs {
   const float* c_x;        // [M]
   const float* inv_cw;     // [N] 1/c_w (0 where c_w == 0)
   const __half* W;         // [K,N] fp16, rows of the outlier set are read
-  const __half* X_OT;      // [|O|][M] gathered fp16 outlier activations
+  const __half* X_OT;      // [|O|][ld_xo] gathered fp16 outlier activations (o-major)
+  int ld_xo;               // row stride of X_OT: M rounded up to a multiple of 8
   const int32_t* idx;      // [K] ascending outlier columns
   const int32_t* count;    // [1] |O|
   __half* Y;               // [M,N] fp16 output
@@ -77,26 +78,26 @@ struct GemmArgs {
   uint32_t* sk_ticket;     // split > 1: [tiles][2][2] counters, zero between launches
   int* status;             // device status word
   unsigned long long timeout_ns;
+  int skip_arrival;        // failure-detection test only: split-K pieces do not count
+                           // themselves on the owner's ticket, so its wait runs out
 };
 
-// Y = (Xq Wq^T) / (c_x c_w^T) + X[:,O] W[O,:].  tmA maps Xq [M,K] int8 with
-// 128x128-byte swizzled boxes; tmB maps the K-blocked weight Wb as a 2-D
-// array of (K/128 * N_pad) rows of 128 bytes with kGemmBN-row boxes (the box
-// of n block j at k block kb starts at row kb * N_pad + j * kGemmBN).
+// Y = (Xq Wq^T) / (c_x c_w^T) + X[:,O] W[O,:], computed by pairs of CTAs on
+// 256 x 256 tiles.  tmA maps Xq [M,K] int8 with 128x128-byte swizzled boxes;
+// tmB maps the K-blocked weight Wb as a 2-D array of (K/128 * N_pad) rows of
+// 128 bytes with 128-row boxes (the rows of n block j at k block kb start at
+// row kb * N_pad + j * kGemmBN).
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 128;
 constexpr int kGemmMaxSplit = 4;
 // Pieces along K per 256x256 tile of the CTA-pair GEMM for an M x N x K
-// problem (1 for single-CTA tiles): the split that best fills the pairs'
-// rounds of work.
+// problem: the split that best fills the pairs' rounds of work.
 int gemm_split_for(int64_t M, int64_t N, int64_t K, int num_sms);
-// tmB256 / tmB128 map the weight with 256- and 128-row boxes (the second is
-// used by the CTA-pair mode, for M > 128).  With `pdl`, launched as a
-// programmatic dependent of the activation pass: its prologue and the first
-// weight-tile loads overlap that pass.
-cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB256, const CUtensorMap& tmB128,
-                               const GemmArgs& a, int num_sms, bool pdl, cudaStream_t stream);
+// With `pdl`, launched as a programmatic dependent of the activation pass:
+// its prologue and the first weight-tile loads overlap that pass.
+cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
+                               bool pdl, cudaStream_t stream);
 
 // Largest K any kernel here accepts (the row kernels keep a row in registers).
 constexpr int64_t kMaxK = 65536;
@@ -114,7 +115,8 @@ struct SmallActArgs {
   float alpha;
   int8_t* Xq;       // [M, K]
   float* c_x;       // [M]
-  __half* X_OT;     // [|O|][M]
+  __half* X_OT;     // [|O|][ld_xo]
+  int ld_xo;        // row stride of X_OT (M rounded up to a multiple of 8)
   float* colmax;    // [K]
   int32_t* idx;     // [K]
   int32_t* count;   // [1]
@@ -140,7 +142,8 @@ struct RowActArgs {
   int thr;             // half_magnitude_threshold(alpha)
   int8_t* Xq;          // [M, K]
   float* c_x;          // [M]
-  __half* X_OT;        // [|O|][M]
+  __half* X_OT;        // [|O|][ld_xo]
+  int ld_xo;           // row stride of X_OT (M rounded up to a multiple of 8)
   int32_t* idx;        // [K]
   int32_t* count;      // [1]
   uint32_t* omask;     // [2][ceil(K/32)] bitmasks; the one of the current generation is zero
@@ -150,6 +153,8 @@ struct RowActArgs {
   float* colmax;               // [K]
   int* status;
   unsigned long long timeout_ns;
+  int skip_arrival;            // failure-detection test only: block 0 does not arrive at the
+                               // grid barrier, so every block's wait there runs out
 };
 constexpr int64_t kRowActMaxK = 32768;
 constexpr int64_t kRowActMaxRows = 256;
@@ -164,10 +169,12 @@ cudaError_t launch_row_act(const RowActArgs& a, int num_sms, cudaStream_t stream
 struct DecodeArgs {
   int M, N, K;
   int N_pad;               // rows per k block in the weight layout
+  const int8_t* Wb;        // the K-blocked weight codes that tmW maps (for L2 prefetches)
   const float* c_x;        // [M]
   const float* inv_cw;     // [N]
   const __half* W;         // [K,N] fp16 (outlier rows are read)
-  const __half* X_OT;      // [|O|][M]
+  const __half* X_OT;      // [|O|][ld_xo]
+  int ld_xo;               // row stride of X_OT (M rounded up to a multiple of 8)
   const int32_t* idx;      // [K]
   const int32_t* count;    // [1]
   __half* Y;               // [M,N]
@@ -177,6 +184,8 @@ struct DecodeArgs {
   unsigned* ticket;        // [ceil(N/128)] k-steps done per n block, zero between launches
   int* status;
   unsigned long long timeout_ns;
+  int skip_arrival;        // failure-detection test only: split pieces do not count their
+                           // k steps on the owner's ticket, so its wait runs out
 };
 // Tokens padded to the MMA N of the decode kernel: 16, 32 or 64.
 int decode_padded_tokens(int64_t M);

@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(NT) row_quant_kernel(const __half* __restrict_
                                                        const uint32_t* __restrict__ mask,
                                                        const int32_t* __restrict__ pre,
                                                        int8_t* __restrict__ Xq, float* __restrict__ c_x,
-                                                       __half* __restrict__ X_OT) {
+                                                       __half* __restrict__ X_OT, int ld_xo) {
   const int row = blockIdx.x, tid = threadIdx.x;
   const int nvec = K / 8;
   const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<size_t>(row) * K);
@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(NT) row_quant_kernel(const __half* __restrict_
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           if ((fl[i] >> e) & 1u) {
-            X_OT[static_cast<size_t>(o) * M + row] = __ushort_as_half(hs[e]);
+            X_OT[static_cast<size_t>(o) * ld_xo + row] = __ushort_as_half(hs[e]);
             ++o;
           }
       }
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(NT) row_quant_kernel(const __half* __restrict_
 
 template <int VPT, int NT>
 cudaError_t launch_row_quant_t(const __half* X, int64_t M, int64_t K, const OutlierScratch& s, int8_t* Xq,
-                               float* c_x, __half* X_OT, bool pdl, cudaStream_t stream) {
+                               float* c_x, __half* X_OT, int64_t ld_xo, bool pdl, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(M));
   cfg.blockDim = dim3(NT);
@@ -326,7 +326,7 @@ cudaError_t launch_row_quant_t(const __half* X, int64_t M, int64_t K, const Outl
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, row_quant_kernel<VPT, NT>, X, static_cast<int>(M), static_cast<int>(K),
                             static_cast<const uint32_t*>(s.mask), static_cast<const int32_t*>(s.pre), Xq, c_x,
-                            X_OT);
+                            X_OT, static_cast<int>(ld_xo));
 }
 
 }  // namespace
@@ -360,12 +360,12 @@ cudaError_t launch_outlier_detect(const __half* X, int64_t M, int64_t K, float a
 }
 
 cudaError_t launch_row_quant(const __half* X, int64_t M, int64_t K, const OutlierScratch& s, int8_t* Xq,
-                             float* c_x, __half* X_OT, bool pdl, cudaStream_t stream) {
+                             float* c_x, __half* X_OT, int64_t ld_xo, bool pdl, cudaStream_t stream) {
   // 128 threads per row up to K = 16384, then 256 and 512; each thread
   // keeps VPT vectors of 8 halves of its row in registers.
   const int64_t nvec = K / 8;
 #define I8MM_ROWQ(V, T) \
-  if (nvec <= int64_t(V) * (T)) return launch_row_quant_t<V, T>(X, M, K, s, Xq, c_x, X_OT, pdl, stream)
+  if (nvec <= int64_t(V) * (T)) return launch_row_quant_t<V, T>(X, M, K, s, Xq, c_x, X_OT, ld_xo, pdl, stream)
   I8MM_ROWQ(1, 128);
   I8MM_ROWQ(2, 128);
   I8MM_ROWQ(3, 128);

@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) xact_rows_kernel(RowActArgs a)
   __syncthreads();
   if (tid == 0) {
     uint32_t* arrivals = a.sync + (gen & 1u);
-    red_release_add_gpu(arrivals, 1u);
+    if (!(a.skip_arrival && blockIdx.x == 0)) red_release_add_gpu(arrivals, 1u);
     int bar_ok = 1;
     if (ld_acquire_gpu_u32(arrivals) < gridDim.x) {
       const uint64_t t0 = global_timer_ns();
@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) xact_rows_kernel(RowActArgs a)
             int o = __shfl_sync(0xffffffffu, slot[i2], src);
             for (int e = 0; e < 8; ++e) {
               if ((f >> e) & 1u) {
-                __half* dst = a.X_OT + static_cast<size_t>(o) * M + r0 + rb;
+                __half* dst = a.X_OT + static_cast<size_t>(o) * a.ld_xo + r0 + rb;
                 for (int i = lane; i < rc; i += 32)
                   dst[i] = xh[static_cast<size_t>(slot_of(c, i)) * K + col0 + e];
                 ++o;

@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(NT) xact_small_kernel(SmallActArgs a) {
 #pragma unroll
       for (int e = 0; e < 8; ++e)
         if ((fl >> e) & 1u) {
-          a.X_OT[static_cast<size_t>(o) * M + r] = __ushort_as_half(hs[e]);
+          a.X_OT[static_cast<size_t>(o) * a.ld_xo + r] = __ushort_as_half(hs[e]);
           ++o;
         }
     }
