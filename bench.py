@@ -60,7 +60,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=["175b", "opt13b"], default="175b")
+    ap.add_argument("--config", default="175b",
+                    help="175b or opt13b (the headline workload); with --profile-forwards also "
+                         "ffn2 (OPT-13B FFN contraction), decode:M (M tokens against the 175B-scale "
+                         "weight) or sweep:M:O (K=N=8192, O planted outlier columns)")
     ap.add_argument("--sections", default="all",
                     help="comma-separated extra sections: opt13b,ffn_contraction,static_weight,decode,"
                          "sweep (or all, or none)")
@@ -76,6 +79,13 @@ def parse_args():
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
+    headline = a.config in ("175b", "opt13b")
+    if not headline and (a.profile_forwards <= 0 or a.impl != "ours"):
+        ap.error("--config other than 175b/opt13b only with --profile-forwards")
+    try:
+        make_problem(a.config, 0, check_only=True)
+    except ValueError as e:
+        ap.error(str(e))
     known = {"opt13b", "ffn_contraction", "static_weight", "decode", "sweep"}
     if a.sections == "all":
         a.sections = set(known)
@@ -88,10 +98,31 @@ def parse_args():
     return a
 
 
-def make_problem(config: str, rank: int) -> workloads.Problem:
-    if config == "opt13b":
-        return workloads.opt13b_prefill(repeat=rank)
-    return workloads.gpt175b_prefill(repeat=rank)
+def make_problem(config: str, rank: int, check_only: bool = False):
+    """The workload named by --config (see parse_args)."""
+    parts = config.split(":")
+    try:
+        if parts == ["opt13b"]:
+            return None if check_only else workloads.opt13b_prefill(repeat=rank)
+        if parts == ["175b"]:
+            return None if check_only else workloads.gpt175b_prefill(repeat=rank)
+        if parts == ["ffn2"]:
+            return None if check_only else workloads.opt13b_contraction(repeat=rank)
+        if parts[0] == "decode" and len(parts) == 2 and int(parts[1]) in DECODE_MS:
+            if check_only:
+                return None
+            p = workloads.decode(int(parts[1]), repeat=rank, with_weight=False)
+            p.W = workloads.weight(DECODE_K, DECODE_N, 3 * 1000 + 500_000 + rank)
+            return p
+        if parts[0] == "sweep" and len(parts) == 3 and int(parts[1]) in SWEEP_MS and int(parts[2]) in SWEEP_OUTLIERS:
+            if check_only:
+                return None
+            p = workloads.sweep(int(parts[1]), int(parts[2]), repeat=rank, with_weight=False)
+            p.W = workloads.weight(SWEEP_K, SWEEP_N, 4 * 1000 + 500_000 + rank)
+            return p
+    except ValueError:
+        pass
+    raise ValueError(f"unknown --config {config!r}")
 
 
 def workload_config(p: workloads.Problem) -> dict:

@@ -132,10 +132,9 @@ int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream);
  * M == 0 is a no-op.  Two or three kernels run on `stream`: the activation
  * pass (outlier detection, row quantisation and the outlier gather) and the
  * fused int8 GEMM, a programmatic dependent launch that starts while the
- * activation pass finishes.  The activation pass is one kernel when X fits
- * in the GPU's shared memory (rows split evenly over one block per SM, K <=
- * 32768) or M <= 64, else two (detection, then quantisation); a static
- * weight adds the gather of the outlier rows; see
+ * activation pass finishes.  The activation pass is one kernel for up to
+ * 256 rows per SM (37888 on a 148-SM B200), else two (detection, then
+ * quantisation); a static weight adds the gather of the outlier rows; see
  * int8mm_launches_per_forward.  The outlier count never leaves the device,
  * so the call does not synchronise.  Grows the workspace when M exceeds every
  * earlier M (stream-ordered allocation).

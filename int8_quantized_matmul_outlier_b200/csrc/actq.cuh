@@ -56,11 +56,12 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, float c) {
 }
 
 // The same codes without conversion instructions (which issue at a fraction
-// of the FMA rate): y = fl(x c) as above, then fl(y + 1.5 2^23), whose ulp is
-// 1 for |y| <= 2^22, rounds y to the nearest integer, ties to even, and the
-// sum's low mantissa byte is that integer in two's complement.  For |y| <= 127
-// (every non-outlier entry) the byte is the code; other entries are masked by
-// the caller.
+// of the FMA rate), by the textbook "magic number" rounding of a float to an
+// integer: y = fl(x c) as above, then fl(y + 1.5 2^23), whose ulp is 1 for
+// |y| <= 2^22, rounds y to the nearest integer, ties to even (the FPU's
+// rounding of the addition), and the sum's low mantissa byte is that integer
+// in two's complement.  For |y| <= 127 (every non-outlier entry) the byte is
+// the code; other entries are masked or overwritten by the caller.
 __device__ __forceinline__ uint32_t rne_low_byte(float x, float c) {
   return __float_as_uint(__fadd_rn(__fmul_rn(x, c), 12582912.0f));
 }

@@ -356,19 +356,13 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     if (events && events[i]) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
   };
   rec(0);
-  if (decode && small_act_fits(M, h->K)) {
-    SmallActArgs sa{Xh,    static_cast<int>(M), static_cast<int>(h->K), alpha,  h->Xq,   h->c_x,
-                    h->X_OT, static_cast<int>(ld_xo), h->colmax, h->idx, h->count};
-    if ((e = launch_small_act(sa, s)) != cudaSuccess) return cuda_fail(e, "activation pass launch");
-  } else if (!decode && row_act_fits(M, h->K, h->num_sms)) {
+  if (row_act_fits(M, h->K, h->num_sms)) {
     RowActArgs ra;
     ra.X = Xh;
     ra.M = static_cast<int>(M);
     ra.K = static_cast<int>(h->K);
     ra.rows_per_block = 0;
-    ra.chunk_rows = 0;
-    ra.slots = 0;
-    ra.col_threads = 0;
+    ra.groups = 0;
     ra.thr = half_magnitude_threshold(alpha);
     ra.Xq = h->Xq;
     ra.c_x = h->c_x;
@@ -378,12 +372,12 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     ra.count = h->count;
     ra.omask = h->omask;
     ra.sync = h->xsync;
-    ra.epoch = h->epoch;
-    ra.colkey = dbg ? h->colkey : nullptr;  // column maxima only for the debug dump
-    ra.colmax = h->colmax;
     ra.status = h->status;
     ra.timeout_ns = h->timeout_ns;
     ra.skip_arrival = (h->test_skip & INT8MM_TEST_SKIP_BARRIER_ARRIVAL) != 0;
+    // the debug dump's column maxima come from the detection kernel
+    if (dbg && (e = launch_outlier_detect(Xh, M, h->K, alpha, sc, s)) != cudaSuccess)
+      return cuda_fail(e, "outlier detection launch");
     if ((e = launch_row_act(ra, h->num_sms, s)) != cudaSuccess) return cuda_fail(e, "activation pass launch");
   } else {
     if ((e = launch_outlier_detect(Xh, M, h->K, alpha, sc, s)) != cudaSuccess)
@@ -413,7 +407,6 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     d.N = static_cast<int>(h->N);
     d.K = static_cast<int>(h->K);
     d.N_pad = static_cast<int>(h->N_pad);
-    d.Wb = h->Wb;
     d.c_x = h->c_x;
     d.inv_cw = h->inv_cw;
     d.W = Wrows;
@@ -799,7 +792,6 @@ int8mm_status int8mm_launches_per_forward(int8mm_weight_t h, int64_t M, int* cou
   if (!live(h) || count == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "invalid handle or NULL output");
   if (M < 0) return fail(INT8MM_ERR_INVALID_ARG, "M=%lld is negative", (long long)M);
   if (M == 0) *count = 0;
-  else if (M <= kDecodeMaxM) *count = small_act_fits(M, h->K) ? 2 : 3;
   else *count = row_act_fits(M, h->K, h->num_sms) ? 2 : 3;
   if (M > 0 && h->wstatic) *count += 1;  // the outlier row gather
   return INT8MM_OK;

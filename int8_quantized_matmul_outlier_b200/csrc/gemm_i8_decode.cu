@@ -42,10 +42,6 @@ constexpr int DBK = 128;  // K bytes per stage
 // Six stages of weight tiles in flight per SM measured faster than deeper
 // rings (4: slower, 11: 12% slower): more outstanding reads only congest HBM.
 constexpr int D_STAGES = 6;
-// Weight tiles past the ring that each CTA asks L2 to fetch while the
-// activation pass is still running (512 KB per CTA, 76 MB over 148 SMs):
-// the weight does not depend on it, so HBM keeps streaming meanwhile.
-constexpr int D_L2_PREFETCH = 32;
 constexpr int D_OUT_STAGE = 128;  // outliers whose activations (and indices) are staged in smem
 constexpr int D_EPI = 256;  // epilogue threads: eight warps
 constexpr int D_THREADS = 64 + D_EPI;
@@ -164,13 +160,6 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         const int nb = static_cast<int>(uu / num_kb), kb = static_cast<int>(uu % num_kb);
         mbar_arrive_expect_tx(&full[i], C::STAGE);
         tma_load_2d_hint(smem + i * C::STAGE, &tmW, &full[i], 0, kb * a.N_pad + nb * DBM, wpol);
-      }
-      // the next tiles into L2 (each one contiguous 16 KB block of the K-blocked layout)
-      const long long pf_end = min(u_end, u_begin + pre + D_L2_PREFETCH);
-      for (long long uu = u_begin + pre; uu < pf_end; ++uu) {
-        const int nb = static_cast<int>(uu / num_kb), kb = static_cast<int>(uu % num_kb);
-        bulk_prefetch_l2(a.Wb + (static_cast<size_t>(kb) * a.N_pad + static_cast<size_t>(nb) * DBM) * DBK,
-                         C::W_BYTES);
       }
       dpdl_wait();
       for (int i = 0; i < pre; ++i) {

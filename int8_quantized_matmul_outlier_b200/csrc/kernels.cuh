@@ -101,44 +101,21 @@ cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, c
 
 // Largest K any kernel here accepts (the row kernels keep a row in registers).
 constexpr int64_t kMaxK = 65536;
-// Forwards with at most this many rows take the few-token path.
+// Forwards with at most this many rows take the decode GEMM.
 constexpr int kDecodeMaxM = 64;
-
-// ---- activation pass for few tokens (M <= kDecodeMaxM) ---------------------
-// One thread-block cluster does detection, quantisation and the outlier
-// gather in one launch (csrc/xact_small.cu); it writes colmax, idx, count,
-// Xq, c_x and X_OT (not mask/pre).  It lets a programmatic dependent launch
-// (the decode GEMM) start at once.
-struct SmallActArgs {
-  const __half* X;  // [M, K]
-  int M, K;
-  float alpha;
-  int8_t* Xq;       // [M, K]
-  float* c_x;       // [M]
-  __half* X_OT;     // [|O|][ld_xo]
-  int ld_xo;        // row stride of X_OT (M rounded up to a multiple of 8)
-  float* colmax;    // [K]
-  int32_t* idx;     // [K]
-  int32_t* count;   // [1]
-};
-constexpr size_t kSmallActSmemMax = 200 * 1024;
-// Whether an M x K activation takes the single-cluster kernel.
-bool small_act_fits(int64_t M, int64_t K);
-cudaError_t launch_small_act(const SmallActArgs& a, cudaStream_t stream);
 
 // ---- activation pass in one launch --------------------------------------
 // Detection, quantisation and the outlier gather (csrc/xact_rows.cu) for K <=
-// kRowActMaxK: the rows, split into equal runs across one block per SM, are
-// held in shared memory when they fit, else streamed through it twice (in
-// chunks, double-buffered).  A cooperative launch with one grid barrier;
-// writes idx, count, Xq, c_x and X_OT (and colmax when colkey is given).
+// kRowActMaxK and at most kRowActMaxRows rows per SM (any M from 1 to 256
+// times the SM count; prefill and decode alike): the rows, split into
+// equal runs across one block per SM, stream through one shared-memory slot
+// per warp and are quantised as they land; a cooperative launch with one
+// grid barrier.  Writes idx, count, Xq, c_x and X_OT (not colmax).
 struct RowActArgs {
   const __half* X;     // [M, K]
   int M, K;
   int rows_per_block;  // set by the launcher
-  int chunk_rows;      // set by the launcher: rows per chunk (= rows_per_block when all fit)
-  int slots;           // set by the launcher: row slots in shared memory
-  int col_threads;     // set by the launcher: threads per row group
+  int groups;          // set by the launcher: row groups (row slots) per block
   int thr;             // half_magnitude_threshold(alpha)
   int8_t* Xq;          // [M, K]
   float* c_x;          // [M]
@@ -148,15 +125,12 @@ struct RowActArgs {
   int32_t* count;      // [1]
   uint32_t* omask;     // [2][ceil(K/32)] bitmasks; the one of the current generation is zero
   uint32_t* sync;      // [3] arrivals for generation parity 0 and 1, generation
-  unsigned long long* epoch;   // epoch of the colkey tags, advanced by every launch
-  unsigned long long* colkey;  // [K] or nullptr; with it, colmax is written too
-  float* colmax;               // [K]
   int* status;
   unsigned long long timeout_ns;
-  int skip_arrival;            // failure-detection test only: block 0 does not arrive at the
-                               // grid barrier, so every block's wait there runs out
+  int skip_arrival;    // failure-detection test only: block 0 does not arrive at the
+                       // grid barrier, so every block's wait there runs out
 };
-constexpr int64_t kRowActMaxK = 32768;
+constexpr int64_t kRowActMaxK = 65536;
 constexpr int64_t kRowActMaxRows = 256;
 constexpr size_t kRowActSmemMax = 220 * 1024;
 // Largest binary16 magnitude pattern (0 .. 0x7c00) whose value is <= alpha,
@@ -169,7 +143,6 @@ cudaError_t launch_row_act(const RowActArgs& a, int num_sms, cudaStream_t stream
 struct DecodeArgs {
   int M, N, K;
   int N_pad;               // rows per k block in the weight layout
-  const int8_t* Wb;        // the K-blocked weight codes that tmW maps (for L2 prefetches)
   const float* c_x;        // [M]
   const float* inv_cw;     // [N]
   const __half* W;         // [K,N] fp16 (outlier rows are read)

@@ -1,6 +1,5 @@
 // Activation pass for many rows in one launch: outlier-column detection,
-// vector-wise row quantisation and the fp16 outlier gather, for activations
-// that fit in the shared memory of the GPU's SMs.
+// vector-wise row quantisation and the fp16 outlier gather.
 //
 //   O      = { j : max_i |X[i,j]| > alpha }                        (ascending)
 //   c_x[i] = 127 / max_{j not in O} |X[i,j]|,  Xq = rne(X c_x), 0 on O
@@ -11,27 +10,39 @@
 // of the AI 十大核心论文解读 article (split, then scale).
 //
 // X is read from HBM once.  G co-resident blocks (cooperative launch, one per
-// SM); block b owns the R consecutive rows [b R, b R + R) and copies them into
-// its shared memory with bulk copies, one mbarrier per row.  Each thread owns
-// a fixed set of 8-column vectors (for all of its rows, or of one row group).
-// Then:
-//   1. per 8-column vector, the max |x| over the block's rows; a column with
-//      an entry above alpha sets its bit in the block's bitmask, and the
-//      non-zero words are OR-ed into a global bitmask.  Since every entry of a
-//      column not in O is at most alpha, "some entry above alpha" is exactly
-//      "column maximum above alpha".
-//   2. grid barrier: each block adds 1 (release) to the arrival counter of the
-//      current generation's parity and waits (acquire) until it reaches G.
-//      Block 0 then zeroes the other parity's counter and advances the
-//      generation; no block reads either again in this launch.
-//   3. every block reads the global bitmask and forms the prefix of its word
-//      popcounts (the slot of an outlier column); block 0 writes the
-//      ascending index list and the count.  From shared memory: per row the
-//      absmax over the non-outlier columns and c_x; then the codes and the
-//      outlier entries.
-// The global bitmask is double-buffered by the parity of the generation:
-// block 0 clears the buffer of the next generation, so no launch needs a
-// clearing pass and all state stays on the device.
+// SM); block b owns the R consecutive rows [b R, b R + R).  Each of its NW
+// warps takes the rows w, w + NW, ... and streams them through a shared-memory
+// slot of its own (one bulk copy and one mbarrier per row), so the warps need
+// no block-wide synchronisation while X lands.
+//
+// A row can be quantised before O is known.  A column is in O exactly when
+// one of its entries exceeds alpha, so every entry of a column outside O is
+// at most alpha.  The block keeps a bitmask of the columns it has seen an
+// entry above alpha in (a subset of O).  Per row, once it has landed, the
+// group
+//   1. flags the columns of the row's entries above alpha;
+//   2. takes S_i = max |X[i,j]| over the columns j not flagged so far (all
+//      of these entries are at most alpha); S_i is at least the absmax over
+//      the columns outside O, and equal to it unless S_i is reached in an
+//      outlier column not flagged yet;
+//   3. writes c_x[i] = 127 / S_i and the codes of every column with it.
+// Every group flags its first row before any row is quantised, so in the
+// pages' activations (a few outlier columns, large in most rows) the block's
+// bitmask already holds the outlier columns when the rows are quantised.
+// Then the block ORs its bitmask into a global one and meets the other
+// blocks at a grid barrier (a release add on an arrival counter, acquire
+// polling, bounded by %globaltimer).  After it, with the global bitmask:
+//   4. for every outlier column j of slot o and every row i of the block:
+//      X_OT[o][i] = X[i,j] and the code of (i, j) is set to 0; a row with an
+//      outlier-column entry <= alpha equal to S_i is marked;
+//   5. a marked row (S_i may come from an outlier column) is quantised
+//      again with the exact absmax over the columns outside O.
+// Step 5 is rare, and the work after the barrier is a few scattered
+// accesses per outlier column and row.
+//
+// Counters and bitmasks are double-buffered by a generation word that block
+// 0 advances after the barrier, so no launch clears anything and the state
+// stays on the device (CUDA-graph replay stays valid).
 #include "actq.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -42,160 +53,161 @@
 namespace i8mm {
 namespace {
 
-constexpr int kMaxThreads = 1024;
+constexpr int kMaxWarps = 32;
+constexpr int kMaxGroups = 15;  // named barriers 1..15, one per row group
 
-// Thread (g, t), g = tid / CT, t = tid % CT, owns the 8-column vectors
-// v = t + i CT (i < VPT) of the rows j = g, g + RG, .. of its block (RG row
-// groups of CT threads, CT a multiple of 32).  Everything a thread needs about
-// its columns (outlier flags, code masks, outlier slots) is fixed for all rows.
-template <int VPT>
-__global__ void __launch_bounds__(kMaxThreads, 1) xact_rows_kernel(RowActArgs a) {
+// Shared memory of a block: one row slot of 2K bytes and one mbarrier per
+// row group, the per-warp partial maxima, the bitmask and its word prefix
+// (KW words each), S_i and the mark of step 5 of the R rows.
+size_t smem_bytes(int64_t groups, int64_t rows, int64_t K) {
+  const int64_t KW = (K + 31) / 32;
+  return static_cast<size_t>(groups * 2 * K + groups * 8 + kMaxWarps * 4 + KW * 8 + rows * 8);
+}
+
+__device__ __forceinline__ void group_sync(int g, int nthreads) {
+  if (nthreads == 32) __syncwarp();
+  else asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "r"(nthreads) : "memory");
+}
+
+// The rows of a block are dealt to G row groups of GW warps (G = the number
+// of row slots that fit, GW so that each lane takes a few 8-column vectors
+// of a row).  Group g takes the rows g, g + G, ... and streams them through
+// its slot.
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) xact_rows_kernel(RowActArgs a) {
   extern __shared__ __align__(128) unsigned char sm[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int NT = blockDim.x;
-  const int CT = a.col_threads, RG = NT / CT;
-  const int g = tid / CT, t = tid - g * CT;
-  const int K = a.K, M = a.M, R = a.rows_per_block, H = a.chunk_rows, S = a.slots;
+  const int NT = blockDim.x, NW = NT >> 5;
+  const int G = a.groups, GW = NW / G;
+  const int K = a.K, M = a.M, R = a.rows_per_block;
   const int nvec = K / 8, KW = (K + 31) / 32;
   const int r0 = static_cast<int>(blockIdx.x) * R;
   const int nr = min(R, M - r0);
-  const int nch = (nr + H - 1) / H;  // chunks of this block's rows
-  const bool streaming = nch > 1;    // rows pass through the slots twice
   const uint32_t row_bytes = 2u * static_cast<uint32_t>(K);
 
-  uint4* xs = reinterpret_cast<uint4*>(sm);                                           // [S][nvec]
-  uint32_t* mask_s = reinterpret_cast<uint32_t*>(sm + static_cast<size_t>(S) * row_bytes);  // [KW]
-  int* pre_s = reinterpret_cast<int*>(mask_s + KW);                                   // [KW]
-  uint32_t* rowmax_s = reinterpret_cast<uint32_t*>(pre_s + KW);                       // [H]
-  float* c_s = reinterpret_cast<float*>(rowmax_s + H);                                // [H]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(rowmax_s + ((2 * H + 1) & ~1));          // [S], 8-byte aligned
+  uint4* slots = reinterpret_cast<uint4*>(sm);                                            // [G][nvec]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + static_cast<size_t>(G) * row_bytes);  // [G]
+  uint32_t* red_s = reinterpret_cast<uint32_t*>(bars + G);                               // [kMaxWarps]
+  uint32_t* mask_s = red_s + kMaxWarps;                                                  // [KW]
+  int* pre_s = reinterpret_cast<int*>(mask_s + KW);                                      // [KW]
+  uint32_t* smax_s = reinterpret_cast<uint32_t*>(pre_s + KW);                            // [R] S_i bits
+  uint32_t* redo_s = smax_s + R;                                                         // [R] step-5 marks
   __shared__ uint32_t s_gen;
-  __shared__ unsigned long long s_epoch;
-  __shared__ int s_ok;
-
-  // Chunk c (rows c H .. c H + H - 1 of the block) lives in half c % 2 of the
-  // slots when streaming, else in slots 0 .. nr - 1.  The mbarrier of a slot
-  // completes one phase per copy into it.  Only the last chunk can be short,
-  // so in pass 1 row i of chunk c is copy c / 2 into its slot, and in pass 2
-  // it follows the pass-1 copies into that slot (one fewer for the slots the
-  // short last chunk leaves out).
-  const int rc_last = nr - (nch - 1) * H;
-  auto slot_of = [&](int c, int i) { return streaming ? (c & 1) * H + i : i; };
-  auto parity = [&](int pass, int c, int i) -> uint32_t {
-    if (!streaming) return 0u;
-    if (pass == 1) return static_cast<uint32_t>((c >> 1) & 1);
-    const int h = c & 1;
-    const int n1 = (nch - h + 1) / 2 - ((((nch - 1) & 1) == h && i >= rc_last) ? 1 : 0);
-    return static_cast<uint32_t>((n1 + (c >> 1)) & 1);
-  };
-  int last_c[2] = {-1, -1}, last_pass[2] = {0, 0};  // thread 0: the latest copy into each half
-  auto issue = [&](int pass, int c) {  // thread 0: bulk copies of chunk c's rows
-    last_c[c & 1] = c;
-    last_pass[c & 1] = pass;
-    const int rb = c * H, rc = min(H, nr - rb);
-    const unsigned char* src =
-        reinterpret_cast<const unsigned char*>(a.X) + static_cast<size_t>(r0 + rb) * row_bytes;
-    for (int i = 0; i < rc; ++i) {
-      uint64_t* b = &bars[slot_of(c, i)];
-      mbar_arrive_expect_tx(b, row_bytes);
-      bulk_load_1d(xs + static_cast<size_t>(slot_of(c, i)) * nvec, src + static_cast<size_t>(i) * row_bytes,
-                   row_bytes, b);
-    }
-  };
-  // waits (bounded) for chunk c's rows of the given pass; any thread
-  auto wait_chunk = [&](int pass, int c) -> bool {
-    const int rc = min(H, nr - c * H);
-    for (int i = 0; i < rc; ++i)
-      if (!mbar_wait(&bars[slot_of(c, i)], parity(pass, c, i), a.timeout_ns, nullptr)) return false;
-    return true;
-  };
-  // thread 0, after a failed wait: let the copies still in flight land
-  auto drain = [&]() {
-    for (int h = 0; h < 2; ++h)
-      if (last_c[h] >= 0) wait_chunk(last_pass[h], last_c[h]);
-  };
+  __shared__ int s_ok, s_count;
 
   // The GEMM that follows may launch now; its blocks take the SMs this
   // kernel leaves.
   pdl_launch_dependents();
   if (tid == 0) {
     s_gen = *reinterpret_cast<volatile uint32_t*>(a.sync + 2);
-    s_epoch = *reinterpret_cast<volatile unsigned long long*>(a.epoch);
-    for (int j = 0; j < S; ++j) mbar_init(&bars[j], 1);
+    for (int g = 0; g < G; ++g) mbar_init(&bars[g], 1);
     fence_mbar_init();
   }
   for (int w = tid; w < KW; w += NT) mask_s[w] = 0u;
-  for (int j = tid; j < H; j += NT) rowmax_s[j] = 0u;
+  for (int i = tid; i < R; i += NT) redo_s[i] = 0u;
   __syncthreads();
-  if (tid == 0) {
-    issue(1, 0);
-    if (streaming) issue(1, 1);
-  }
 
   // ------------------------------------------------------------- phase 1
-  // max |x| of the owned vectors over the group's rows, as rows land; a
-  // streamed half is refilled once every thread is done with it
-  uint32_t mx[VPT][4];
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) mx[i][0] = mx[i][1] = mx[i][2] = mx[i][3] = 0u;
-  int ok = 1;
-  for (int c = 0; c < nch; ++c) {
-    const int rc = min(H, nr - c * H);
-    for (int i = g; i < rc && ok; i += RG) {
-      const int sl = slot_of(c, i);
-      if (!mbar_wait(&bars[sl], parity(1, c, i), a.timeout_ns, nullptr)) {
-        ok = 0;
-        break;
-      }
-      const uint4* row = xs + static_cast<size_t>(sl) * nvec;
-#pragma unroll
-      for (int i2 = 0; i2 < VPT; ++i2) {
-        const int v = t + i2 * CT;
-        if (v < nvec) {
-          const uint4 x = row[v];
-          mx[i2][0] = __vmaxu2(mx[i2][0], x.x & 0x7fff7fffu);
-          mx[i2][1] = __vmaxu2(mx[i2][1], x.y & 0x7fff7fffu);
-          mx[i2][2] = __vmaxu2(mx[i2][2], x.z & 0x7fff7fffu);
-          mx[i2][3] = __vmaxu2(mx[i2][3], x.w & 0x7fff7fffu);
-        }
-      }
-    }
-    if (streaming) {
-      ok = __syncthreads_and(ok);  // the half is free
-      if (tid == 0 && ok && c + 2 < nch) issue(1, c + 2);
-    }
-  }
-  // a column is an outlier when some entry exceeds alpha; row groups OR
-  // their flags into the block's bitmask
   const bool all_out = a.thr < 0;  // alpha < 0: every column is an outlier
-  const uint32_t thr2 = all_out ? 0u : (static_cast<uint32_t>(a.thr) * 0x00010001u);
-  const unsigned long long tag = s_epoch << 16;
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int v = t + i * CT;
-    if (v < nvec && ok) {
-      uint32_t fl = 0;
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const uint32_t gt = all_out ? 0xffffffffu : __vcmpgtu2(mx[i][p], thr2);
-        fl |= ((gt & 1u) << (2 * p)) | (((gt >> 16) & 1u) << (2 * p + 1));
-      }
-      if (fl) atomicOr(&mask_s[v >> 2], fl << ((v & 3) * 8));
-      if (a.colkey != nullptr) {  // column maxima for the debug dump
+  const uint32_t thr2 = all_out ? 0u : static_cast<uint32_t>(a.thr) * 0x00010001u;
+  const int g = warp / GW, wg = warp - g * GW;  // row group, warp within it
+  const int gthreads = GW * 32, gt = wg * 32 + lane;
+  const bool leader = gt == 0;
+  const int my_rows = nr > g ? (nr - g + G - 1) / G : 0;  // local rows g + j G
+  uint4* slot = slots + static_cast<size_t>(g) * nvec;
+  uint64_t* bar = &bars[g];
+  auto issue = [&](int j) {  // leader: the bulk copy of the group's j-th row into its slot
+    const int lr = g + j * G;
+    mbar_arrive_expect_tx(bar, row_bytes);
+    bulk_load_1d(slot, reinterpret_cast<const unsigned char*>(a.X) + static_cast<size_t>(r0 + lr) * row_bytes,
+                 row_bytes, bar);
+  };
+  // all lanes of the group agree on v (a wait that ran out in one of them)
+  auto group_all = [&](bool v) -> bool {
+    if (GW == 1) return __all_sync(0xffffffffu, v);
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n bar.red.and.pred p, %2, %3, q;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v)), "r"(1 + g), "r"(gthreads)
+        : "memory");
+    return r != 0;
+  };
+  // (1) waits for the group's j-th row, then flags the columns of its
+  //     entries above alpha in the block's bitmask (a branch per vector
+  //     that holds one)
+  auto land_and_flag = [&](int j) -> bool {
+    bool landed = mbar_wait(bar, static_cast<uint32_t>(j & 1), a.timeout_ns, nullptr);
+    if (!group_all(landed)) {
+      // leave no bulk copy in flight into the slot before the block can exit
+      mbar_wait(bar, static_cast<uint32_t>(j & 1), a.timeout_ns, nullptr);
+      return false;
+    }
+#pragma unroll 4
+    for (int v = gt; v < nvec; v += gthreads) {
+      const uint4 x = slot[v];
+      const uint32_t m0 = x.x & 0x7fff7fffu, m1 = x.y & 0x7fff7fffu;
+      const uint32_t m2 = x.z & 0x7fff7fffu, m3 = x.w & 0x7fff7fffu;
+      const uint32_t f = __vmaxu2(__vmaxu2(m0, m1), __vmaxu2(m2, m3));
+      if (all_out || __vcmpgtu2(f, thr2) != 0u) {
+        const uint32_t mw[4] = {m0, m1, m2, m3};
+        uint32_t fl = 0u;
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-          atomicMax(a.colkey + 8 * v + 2 * p, tag | (mx[i][p] & 0xffffu));
-          atomicMax(a.colkey + 8 * v + 2 * p + 1, tag | (mx[i][p] >> 16));
+          const uint32_t big = all_out ? 0xffffffffu : __vcmpgtu2(mw[p], thr2);
+          fl |= ((big & 1u) << (2 * p)) | (((big >> 16) & 1u) << (2 * p + 1));
         }
+        atomicOr(&mask_s[v >> 2], fl << ((v & 3) * 8));
       }
     }
-  }
+    return true;
+  };
+  if (leader && my_rows > 0) issue(0);
+  // The first row of every group is flagged before any row is quantised:
+  // the outlier columns then show in the block's bitmask (in the pages'
+  // activations an outlier column is large in most rows), so S_i below
+  // leaves them out and rarely needs the correction after the barrier.
+  int ok = my_rows > 0 ? land_and_flag(0) : 1;
   ok = __syncthreads_and(ok);
-  // streaming: the second pass's first two chunks load during the barrier
-  if (streaming && tid == 0 && ok) {
-    issue(2, 0);
-    issue(2, 1);
+  for (int j = 0; j < my_rows && ok; ++j) {
+    const int lr = g + j * G;
+    if (j > 0 && !land_and_flag(j)) {
+      ok = 0;
+      break;
+    }
+    // (2) S_i: max |x| over the columns not flagged so far (every entry
+    //     above alpha is flagged, by the lane that reads it again here)
+    uint32_t rm = 0u;
+#pragma unroll 4
+    for (int v = gt; v < nvec; v += gthreads) {
+      const uint32_t fl = (mask_s[v >> 2] >> ((v & 3) * 8)) & 0xffu;
+      rm = masked_absmax2(rm, slot[v], fl);
+    }
+    uint32_t S = __reduce_max_sync(0xffffffffu, max_pair(rm));
+    if (GW > 1) {
+      if (lane == 0) red_s[warp] = S;
+      group_sync(g, gthreads);
+      for (int u = 0; u < GW; ++u) S = max(S, red_s[g * GW + u]);
+    }
+    const float c = scale_from_absmax_bits(S);
+    // (3) the codes of every column with c = 127 / S_i; those of the
+    //     outlier columns are set to 0 after the barrier
+    int8_t* qrow = a.Xq + static_cast<size_t>(r0 + lr) * K;
+#pragma unroll 4
+    for (int v = gt; v < nvec; v += gthreads)
+      *reinterpret_cast<uint2*>(qrow + static_cast<size_t>(v) * 8) = quant8_fma(slot[v], c);
+    if (leader) {
+      smax_s[lr] = S;
+      a.c_x[r0 + lr] = c;
+    }
+    group_sync(g, gthreads);  // the group is done with the slot (and with red_s)
+    if (leader && j + 1 < my_rows) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(j + 1);
+    }
   }
+
+  // the block's outlier bits into the global bitmask of this generation
+  ok = __syncthreads_and(ok);
   const uint32_t gen = s_gen;
   uint32_t* gmask = a.omask + static_cast<size_t>(gen & 1u) * KW;
   for (int w = tid; w < KW; w += NT) {
@@ -223,16 +235,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1) xact_rows_kernel(RowActArgs a)
     s_ok = ok && bar_ok;
   }
   __syncthreads();
-  if (!s_ok) {
-    // leave no bulk copy in flight into this block's shared memory
-    if (tid == 0) drain();
-    return;
-  }
+  if (!s_ok) return;  // no copy is in flight: every group waited for its last one
   if (blockIdx.x == 0 && tid == 0) {
-    // every block has read the generation and the epoch (before arriving)
+    // every block has read the generation (before arriving)
     a.sync[(gen + 1u) & 1u] = 0u;
     a.sync[2] = gen + 1u;
-    *a.epoch = s_epoch + 1;
   }
 
   // ------------------------------------------------------------- phase 3
@@ -254,203 +261,108 @@ __global__ void __launch_bounds__(kMaxThreads, 1) xact_rows_kernel(RowActArgs a)
     int pos = incl - cnt;
     for (int w = w0; w < w1; ++w) {
       pre_s[w] = pos;
-      if (blockIdx.x == 0) {
-        uint32_t bits = mask_s[w];
-        int o = pos;
-        while (bits) {
-          a.idx[o++] = w * 32 + __ffs(bits) - 1;
-          bits &= bits - 1;
-        }
-      }
       pos += __popc(mask_s[w]);
     }
-    if (blockIdx.x == 0 && lane == 31) *a.count = incl;
+    if (lane == 31) {
+      s_count = incl;
+      if (blockIdx.x == 0) *a.count = incl;
+    }
   }
   if (blockIdx.x == 0) {
     uint32_t* next = a.omask + static_cast<size_t>((gen + 1u) & 1u) * KW;
     for (int w = tid; w < KW; w += NT) next[w] = 0u;
-    if (a.colkey != nullptr)
-      for (int c = tid; c < K; c += NT) {
-        const unsigned long long key = __ldcg(a.colkey + c);
-        a.colmax[c] = (key >> 16) == s_epoch
-                          ? __half2float(__ushort_as_half(static_cast<unsigned short>(key & 0xffffu)))
-                          : 0.0f;
-      }
   }
   __syncthreads();
-  // per owned vector: outlier flags, the masks that keep its non-outlier codes,
-  // and the X_OT slot of its first outlier column
-  uint32_t fl[VPT], keep[VPT][2];
-  int slot[VPT];
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int v = t + i * CT;
-    fl[i] = 0u;
-    keep[i][0] = keep[i][1] = 0u;
-    slot[i] = 0;
-    if (v < nvec) {
-      const int w = v >> 2, sh = (v & 3) * 8;
-      fl[i] = (mask_s[w] >> sh) & 0xffu;
-      keep[i][0] = ~expand_nibble(fl[i] & 0xfu);
-      keep[i][1] = ~expand_nibble(fl[i] >> 4);
-      slot[i] = pre_s[w] + __popc(mask_s[w] & ((1u << sh) - 1u));
+  // the ascending list of outlier columns, in the (now free) row slots: at
+  // most K entries of 2 bytes; block 0 also writes it out as idx
+  uint16_t* cols = reinterpret_cast<uint16_t*>(slots);
+  for (int w = tid; w < KW; w += NT) {
+    uint32_t bits = mask_s[w];
+    int o = pre_s[w];
+    while (bits) {
+      const int col = w * 32 + __ffs(bits) - 1;
+      bits &= bits - 1;
+      cols[o] = static_cast<uint16_t>(col);
+      if (blockIdx.x == 0) a.idx[o] = col;
+      ++o;
     }
   }
-  int ok3 = 1;
-  for (int c = 0; c < nch; ++c) {
-    const int rb = c * H, rc = min(H, nr - rb);
-    // streaming: the chunk's rows again (every thread reads all of them
-    // below: its group's rows, and group 0 every row for the outlier entries)
-    if (streaming && ok3 && !wait_chunk(2, c)) ok3 = 0;
-    ok3 = __syncthreads_and(ok3);
-    if (ok3) {
-      // row maxima over the non-outlier columns (vectors past K have keep = 0),
-      // four rows at a time so that their loads and reductions overlap
-      for (int k0 = 0; g + RG * k0 < rc; k0 += 4) {
-        uint32_t m[4] = {0u, 0u, 0u, 0u};
+  __syncthreads();
+  // (4) every (outlier, row) pair of the block, rows fastest: gather the
+  //     entry, zero its code, and mark the row when the entry is <= alpha
+  //     and equal to S_i; four pairs' loads in flight per thread
+  const int n_out = s_count;
+  const unsigned short* xb = reinterpret_cast<const unsigned short*>(a.X);
+  const int pairs = n_out * nr;
+  for (int p0 = tid; p0 < pairs; p0 += 4 * NT) {
+    unsigned short x[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = g + RG * (k0 + u);
-          if (i < rc) {
-            const uint4* row = xs + static_cast<size_t>(slot_of(c, i)) * nvec;
-#pragma unroll
-            for (int i2 = 0; i2 < VPT; ++i2) {
-              const uint4 x = row[min(t + i2 * CT, nvec - 1)];
-              // the byte masks widened to 16-bit lanes, with the sign bits cleared
-              m[u] = __vmaxu2(m[u], x.x & __byte_perm(keep[i2][0], 0u, 0x1100) & 0x7fff7fffu);
-              m[u] = __vmaxu2(m[u], x.y & __byte_perm(keep[i2][0], 0u, 0x3322) & 0x7fff7fffu);
-              m[u] = __vmaxu2(m[u], x.z & __byte_perm(keep[i2][1], 0u, 0x1100) & 0x7fff7fffu);
-              m[u] = __vmaxu2(m[u], x.w & __byte_perm(keep[i2][1], 0u, 0x3322) & 0x7fff7fffu);
-            }
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = g + RG * (k0 + u);  // the same for the whole warp
-          const uint32_t r = __reduce_max_sync(0xffffffffu, max_pair(m[u]));
-          if (lane == 0 && i < rc) atomicMax(&rowmax_s[i], r);
-        }
-      }
-      __syncthreads();
-      for (int i = tid; i < rc; i += NT) {
-        const float cx = scale_from_absmax_bits(rowmax_s[i]);
-        c_s[i] = cx;
-        a.c_x[r0 + rb + i] = cx;
-        rowmax_s[i] = 0u;  // for the next chunk
-      }
-      __syncthreads();
-      // codes (outlier columns 0)
-#pragma unroll 2
-      for (int i = g; i < rc; i += RG) {
-        const float cx = c_s[i];
-        const uint4* row = xs + static_cast<size_t>(slot_of(c, i)) * nvec;
-        int8_t* qrow = a.Xq + static_cast<size_t>(r0 + rb + i) * K;
-#pragma unroll
-        for (int i2 = 0; i2 < VPT; ++i2) {
-          const int v = t + i2 * CT;
-          if (v < nvec) {
-            const uint4 x = row[v];
-            uint2 q = quant8_fma(x, cx);
-            q.x &= keep[i2][0];
-            q.y &= keep[i2][1];
-            *reinterpret_cast<uint2*>(qrow + static_cast<size_t>(v) * 8) = q;
-          }
-        }
-      }
-      // the outlier entries, X_OT[o][r0 + rb + i]: the warps of row group 0
-      // take the outlier vectors their lanes own, one at a time, and write
-      // the chunk's rows of each outlier column with consecutive lanes on
-      // consecutive rows (one coalesced store per column and 32 rows, instead
-      // of a partial-sector store per entry)
-      if (g == 0) {
-        const __half* xh = reinterpret_cast<const __half*>(xs);
-#pragma unroll
-        for (int i2 = 0; i2 < VPT; ++i2) {
-          uint32_t owners = __ballot_sync(0xffffffffu, fl[i2] != 0u);
-          while (owners) {
-            const int src = __ffs(owners) - 1;
-            owners &= owners - 1;
-            const uint32_t f = __shfl_sync(0xffffffffu, fl[i2], src);
-            const int col0 = 8 * (__shfl_sync(0xffffffffu, t, src) + i2 * CT);
-            int o = __shfl_sync(0xffffffffu, slot[i2], src);
-            for (int e = 0; e < 8; ++e) {
-              if ((f >> e) & 1u) {
-                __half* dst = a.X_OT + static_cast<size_t>(o) * a.ld_xo + r0 + rb;
-                for (int i = lane; i < rc; i += 32)
-                  dst[i] = xh[static_cast<size_t>(slot_of(c, i)) * K + col0 + e];
-                ++o;
-              }
-            }
-          }
-        }
+    for (int u = 0; u < 4; ++u) {
+      const int p = p0 + u * NT;
+      x[u] = 0;
+      if (p < pairs) {
+        const int o = p / nr, r = p - o * nr;
+        x[u] = __ldg(xb + static_cast<size_t>(r0 + r) * K + cols[o]);
       }
     }
-    if (streaming) {
-      __syncthreads();  // the half is free
-      if (tid == 0 && ok3 && c + 2 < nch) issue(2, c + 2);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int p = p0 + u * NT;
+      if (p < pairs) {
+        const int o = p / nr, r = p - o * nr;
+        a.X_OT[static_cast<size_t>(o) * a.ld_xo + r0 + r] = __ushort_as_half(x[u]);
+        a.Xq[static_cast<size_t>(r0 + r) * K + cols[o]] = 0;
+        const uint32_t mag = x[u] & 0x7fffu;
+        if (!all_out && mag <= static_cast<uint32_t>(a.thr) && mag == smax_s[r]) redo_s[r] = 1u;
+      }
     }
   }
-  if (!ok3 && tid == 0) {
-    atomicOr(a.status, kStatusTimeout);
-    drain();  // leave no bulk copy in flight into this block's shared memory
+  __syncthreads();
+  // (5) marked rows: the exact absmax over the columns outside O, c_x and
+  //     the codes again (outlier columns 0)
+  for (int lr = warp; lr < nr; lr += NW) {
+    if (smax_s[lr] == 0u || redo_s[lr] == 0u) continue;  // warp-uniform
+    const uint4* xr = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(r0 + lr) * K);
+    uint32_t m = 0u;
+    for (int v = lane; v < nvec; v += 32) {
+      const uint32_t fl = (mask_s[v >> 2] >> ((v & 3) * 8)) & 0xffu;
+      m = masked_absmax2(m, __ldg(xr + v), fl);
+    }
+    const uint32_t S2 = __reduce_max_sync(0xffffffffu, max_pair(m));
+    const float c = scale_from_absmax_bits(S2);
+    int8_t* qrow = a.Xq + static_cast<size_t>(r0 + lr) * K;
+    for (int v = lane; v < nvec; v += 32) {
+      const uint32_t fl = (mask_s[v >> 2] >> ((v & 3) * 8)) & 0xffu;
+      uint2 q = quant8_fma(__ldg(xr + v), c);
+      q.x &= ~expand_nibble(fl & 0xfu);
+      q.y &= ~expand_nibble(fl >> 4);
+      *reinterpret_cast<uint2*>(qrow + static_cast<size_t>(v) * 8) = q;
+    }
+    if (lane == 0) a.c_x[r0 + lr] = c;
   }
 }
 
 struct Shape {
-  int vpt, col_threads, threads;
-  int64_t rows;   // per block
-  int64_t chunk;  // rows per chunk (= rows when they all fit at once)
-  int64_t slots;  // row slots in shared memory
+  int64_t rows;    // per block
+  int64_t groups;  // row groups per block: one row slot each
+  int64_t gw;      // warps per row group
 };
-
-size_t smem_bytes(int64_t slots, int64_t chunk, int64_t K) {
-  const int64_t KW = (K + 31) / 32;
-  return static_cast<size_t>(slots * 2 * K + KW * 8 + ((2 * chunk + 1) & ~int64_t(1)) * 4 + slots * 8);
-}
 
 Shape shape_for(int64_t M, int64_t K, int num_sms) {
   Shape s;
-  const int64_t nvec = K / 8;
-  s.vpt = nvec <= kMaxThreads ? 1 : nvec <= 2 * kMaxThreads ? 2 : 4;
-  s.col_threads = static_cast<int>(32 * ((nvec + 32 * s.vpt - 1) / (32 * s.vpt)));
   s.rows = (M + num_sms - 1) / num_sms;
-  if (s.rows <= kRowActMaxRows && smem_bytes(s.rows, s.rows, K) <= kRowActSmemMax) {
-    s.chunk = s.slots = s.rows;  // every row of the block stays in shared memory
-  } else {
-    // streamed in chunks through two halves of the slots
-    int64_t h = std::min<int64_t>(kRowActMaxRows, s.rows);
-    while (h > 0 && smem_bytes(2 * h, h, K) > kRowActSmemMax) --h;
-    s.chunk = h;
-    s.slots = 2 * h;
-  }
-  const int64_t groups = std::max<int64_t>(1, std::min<int64_t>(kMaxThreads / s.col_threads, std::max<int64_t>(1, s.chunk)));
-  s.threads = static_cast<int>(groups * s.col_threads);
+  const int64_t KW = (K + 31) / 32;
+  const int64_t fixed = KW * 8 + s.rows * 8 + kMaxWarps * 4;
+  const int64_t per_group = 2 * K + 8;
+  const int64_t fit = static_cast<int64_t>(kRowActSmemMax) > fixed
+                          ? (static_cast<int64_t>(kRowActSmemMax) - fixed) / per_group
+                          : 0;
+  s.groups = std::min<int64_t>({s.rows, static_cast<int64_t>(kMaxGroups), fit});
+  // warps per group: about four 8-column vectors per lane and row, within
+  // the block's 32 warps
+  const int64_t nvec = K / 8;
+  s.gw = s.groups > 0 ? std::max<int64_t>(1, std::min<int64_t>(kMaxWarps / s.groups, nvec / 128)) : 1;
   return s;
-}
-
-template <int VPT>
-cudaError_t launch_t(const RowActArgs& a, unsigned grid, unsigned threads, size_t smem, cudaStream_t stream) {
-  static unsigned long long attr_set = 0;  // one bit per device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(attr_set & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(xact_rows_kernel<VPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kRowActSmemMax));
-    if (e != cudaSuccess) return e;
-    attr_set |= bit;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeCooperative;  // all blocks resident at once (grid barrier)
-  attr.val.cooperative = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, xact_rows_kernel<VPT>, a);
 }
 
 }  // namespace
@@ -474,23 +386,37 @@ int half_magnitude_threshold(float alpha) {
 
 bool row_act_fits(int64_t M, int64_t K, int num_sms) {
   if (M <= 0 || K > kRowActMaxK || num_sms <= 0) return false;
-  return shape_for(M, K, num_sms).chunk >= 1;
+  const Shape s = shape_for(M, K, num_sms);
+  return s.rows <= kRowActMaxRows && s.groups >= 1;
 }
 
 cudaError_t launch_row_act(const RowActArgs& args, int num_sms, cudaStream_t stream) {
   RowActArgs a = args;
   const Shape s = shape_for(a.M, a.K, num_sms);
-  if (s.chunk < 1) return cudaErrorInvalidValue;
+  if (s.groups < 1 || s.rows > kRowActMaxRows) return cudaErrorInvalidValue;
   a.rows_per_block = static_cast<int>(s.rows);
-  a.chunk_rows = static_cast<int>(s.chunk);
-  a.slots = static_cast<int>(s.slots);
-  a.col_threads = s.col_threads;
-  const unsigned grid = static_cast<unsigned>((a.M + s.rows - 1) / s.rows);
-  const size_t smem = smem_bytes(s.slots, s.chunk, a.K);
-  const unsigned threads = static_cast<unsigned>(s.threads);
-  if (s.vpt == 1) return launch_t<1>(a, grid, threads, smem, stream);
-  if (s.vpt == 2) return launch_t<2>(a, grid, threads, smem, stream);
-  return launch_t<4>(a, grid, threads, smem, stream);
+  a.groups = static_cast<int>(s.groups);
+  static unsigned long long attr_set = 0;  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(xact_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kRowActSmemMax));
+    if (e != cudaSuccess) return e;
+    attr_set |= bit;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((a.M + s.rows - 1) / s.rows));
+  cfg.blockDim = dim3(static_cast<unsigned>(32 * s.groups * s.gw));
+  cfg.dynamicSmemBytes = smem_bytes(s.groups, s.rows, a.K);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeCooperative;  // all blocks resident at once (grid barrier)
+  attr.val.cooperative = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, xact_rows_kernel, a);
 }
 
 }  // namespace i8mm

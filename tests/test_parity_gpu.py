@@ -103,7 +103,9 @@ SHAPES = [
     (3000, 5120, 256, 7, 6.0),      # 21 rows (210 KB) of X per block
     (4000, 5120, 256, 5, 6.0),      # streamed: 28 rows per block in chunks of 10, a short last chunk
     (600, 20480, 256, 7, 6.0),      # streamed, two 40 KB rows per chunk
-    (130, 40960, 256, 3, 6.0),      # K > 32768: two-kernel activation path
+    (130, 40960, 256, 3, 6.0),      # 80 KB rows: one row slot per block
+    (3, 65536, 32, 2, 6.0),         # largest K: a 128 KB row slot
+    (38000, 32, 16, 2, 6.0),        # more than 256 rows per SM: two-kernel activation path
 ]
 
 
@@ -147,6 +149,26 @@ def test_threshold_ties_single_launch_pass():
     p.X[0, 63] = -100
     out = check(p)
     assert out["cnt"] == 2
+
+
+@pytest.mark.parametrize("M,K", [(300, 1040), (2048, 5120), (4000, 5120)])
+def test_row_absmax_reached_in_an_outlier_column(M, K):
+    # rows whose largest entry <= alpha lies in an outlier column that only
+    # another block of rows (or a later row) shows as an outlier: the row's
+    # scale must still come from the other columns (bit-exact c_x and codes)
+    p = workloads.small(M, K, 256, 0, seed=M + K + 17)
+    cols = [5, K // 2 + 3, K - 1]
+    p.X[0, cols[0]] = 100.0          # outlier columns, each from one far row
+    p.X[M - 1, cols[1]] = -90.0
+    p.X[M // 2, cols[2]] = 7.0
+    rng = np.random.default_rng(M)
+    for r in rng.choice(np.arange(1, M - 1), size=min(M - 2, 40), replace=False):
+        if r == M // 2:
+            continue
+        c = cols[int(r) % 3]
+        p.X[r, c] = np.float16(5.75 if r % 2 else -5.9)   # above every other entry of the row, <= alpha
+    out = check(p)
+    assert out["cnt"] == 3
 
 
 @pytest.mark.parametrize("K", [4096, 4112])
@@ -430,11 +452,12 @@ def test_launches_per_forward():
     W = torch.from_numpy(workloads.weight(5120, 256, 43)).to(dev())
     w = m.int8mm_prepare_weight(W)
     assert m.int8mm_launches_per_forward(w, 0) == 0
-    assert m.int8mm_launches_per_forward(w, 1) == 2       # single-cluster activation pass + decode GEMM
-    assert m.int8mm_launches_per_forward(w, 2048) == 2    # rows held in shared memory
-    assert m.int8mm_launches_per_forward(w, 4096) == 2    # rows streamed through it
+    assert m.int8mm_launches_per_forward(w, 1) == 2       # single-launch activation pass + decode GEMM
+    assert m.int8mm_launches_per_forward(w, 2048) == 2    # activation pass + CTA-pair GEMM
+    assert m.int8mm_launches_per_forward(w, 4096) == 2    # more rows per block than row slots
     w2 = m.int8mm_prepare_weight(torch.from_numpy(workloads.weight(40960, 256, 44)).to(dev()))
-    assert m.int8mm_launches_per_forward(w2, 2048) == 3   # K > 32768: two activation kernels
+    assert m.int8mm_launches_per_forward(w2, 2048) == 2   # 80 KB rows, one slot per block
+    assert m.int8mm_launches_per_forward(w, 40000) == 3   # > 256 rows per SM: two activation kernels
     with pytest.raises(m.Int8mmError):
         m.int8mm_launches_per_forward(w, -1)
 
