@@ -160,7 +160,10 @@ int8mm_status int8mm_forward_bias(int8mm_weight_t h, const void* X_fp16_dev, int
  * [M, K] into a handle-owned device buffer, runs the forward, and copies Y
  * back into Y_fp16_host [M, N], all enqueued on `stream`.  Y_fp16_host is
  * valid once `stream` has been synchronised.  Use page-locked host memory
- * for the copies to be asynchronous.
+ * for the copies to be asynchronous.  For prefills of at least 512 rows the
+ * GEMM runs in up to four row chunks and each chunk of Y is copied back on a
+ * handle-owned stream while the next chunk computes; `stream` waits for
+ * those copies.
  */
 int8mm_status int8mm_forward_host(int8mm_weight_t h, const void* X_fp16_host, int64_t M, float alpha,
                                   void* Y_fp16_host, void* stream);

@@ -13,6 +13,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdarg>
+#include <functional>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -21,6 +22,10 @@
 #include <vector>
 
 using namespace i8mm;
+
+// Row chunks of the host-buffer forward's prefill GEMM (Y of one chunk is
+// copied out while the next computes).
+constexpr int kHostChunks = 4;
 
 struct int8mm_weight {
   int device = 0;
@@ -66,10 +71,13 @@ struct int8mm_weight {
   const void* tmA_ptr = nullptr;
   int64_t tmA_rows = -1;
   int tmA_box = 0;
-  // device copies for host-buffer forwards
+  // device copies for host-buffer forwards, and the stream and events that
+  // copy Y out chunk by chunk while the next chunk computes
   int64_t io_rows = 0;
   __half* dX = nullptr;
   __half* dY = nullptr;
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t chunk_ev[kHostChunks + 1] = {};
   // memory-saving weight (int8mm_prepare_weight_static): the stored fp16
   // rows, the row map, and per forward the gathered outlier rows, which the
   // GEMMs read as W with idx = 0, 1, 2, ...
@@ -173,6 +181,15 @@ void free_all(int8mm_weight* h) {
   free_workspace(h);
   release(&h->dX);
   release(&h->dY);
+  for (cudaEvent_t& ev : h->chunk_ev)
+    if (ev) {
+      cudaEventDestroy(ev);
+      ev = nullptr;
+    }
+  if (h->copy_stream) {
+    cudaStreamDestroy(h->copy_stream);
+    h->copy_stream = nullptr;
+  }
   release(&h->part);
   release(&h->dticket);
   release(&h->sk_ws);
@@ -332,8 +349,16 @@ int8mm_status set_device(const int8mm_weight* h) {
   return INT8MM_OK;
 }
 
+// With chunk_rows > 0, the prefill GEMM runs on row chunks of that many
+// rows (a multiple of 256) and after_chunk(r0, rows) is called once each
+// chunk's GEMM is enqueued; *whole tells the caller whether that happened
+// (false for the decode GEMM, which runs once).
 int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alpha, void* Y, cudaStream_t s,
-                           void* const* events, const int8mm_debug_bufs* dbg, const void* bias = nullptr) {
+                           void* const* events, const int8mm_debug_bufs* dbg, const void* bias = nullptr,
+                           int64_t chunk_rows = 0,
+                           const std::function<int8mm_status(int64_t, int64_t)>& after_chunk = nullptr,
+                           bool* chunked = nullptr) {
+  bool whole_done = false;
   int8mm_status st = check_forward_args(h, X, M, alpha, Y);
   if (st != INT8MM_OK) return st;
   if (M == 0) return INT8MM_OK;
@@ -425,39 +450,50 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     if ((e = launch_gemm_decode(h->tmW128, h->tmA, d, h->num_sms, pdl, s)) != cudaSuccess)
       return cuda_fail(e, "int8 decode GEMM launch");
   } else {
-    // split K for the CTA-pair tiles; the scratch grows on demand
-    const int split = split_for(h, M);
-    if (split > 1) {
-      const size_t tiles = pair_tiles(h, M);
-      if ((st = ensure_split_scratch(h, static_cast<size_t>(split - 1) * tiles * 2 * kGemmBM * kGemmBN, tiles * 4,
-                                     s)) != INT8MM_OK)
-        return st;
+    // Rows [r0, r0 + rows) at a time (all of them unless the host-buffer
+    // forward asks for chunks, to copy each chunk of Y out while the next
+    // one computes); the first launch is the activation pass's dependent.
+    const int64_t step = (chunk_rows > 0 && chunk_rows < M) ? chunk_rows : M;
+    for (int64_t r0 = 0; r0 < M; r0 += step) {
+      const int64_t rows = std::min(step, M - r0);
+      // split K for the CTA-pair tiles; the scratch grows on demand
+      const int split = split_for(h, rows);
+      if (split > 1) {
+        const size_t tiles = pair_tiles(h, rows);
+        if ((st = ensure_split_scratch(h, static_cast<size_t>(split - 1) * tiles * 2 * kGemmBM * kGemmBN,
+                                       tiles * 4, s)) != INT8MM_OK)
+          return st;
+      }
+      GemmArgs a;
+      a.M = static_cast<int>(rows);
+      a.a_row0 = static_cast<int>(r0);
+      a.N = static_cast<int>(h->N);
+      a.K = static_cast<int>(h->K);
+      a.N_pad = static_cast<int>(h->N_pad);
+      a.c_x = h->c_x + r0;
+      a.inv_cw = h->inv_cw;
+      a.W = Wrows;
+      a.X_OT = h->X_OT + r0;
+      a.ld_xo = static_cast<int>(ld_xo);
+      a.idx = widx;
+      a.count = wcount;
+      a.Y = static_cast<__half*>(Y) + r0 * h->N;
+      a.bias = static_cast<const __half*>(bias);
+      a.acc_dump = dbg ? dbg->acc + r0 * h->N : nullptr;
+      a.split = split;
+      a.sk_ws = h->sk_ws;
+      a.sk_ticket = h->sk_ticket;
+      a.status = h->status;
+      a.timeout_ns = h->timeout_ns;
+      a.skip_arrival = (h->test_skip & INT8MM_TEST_SKIP_SPLITK_TICKET) != 0;
+      if ((e = launch_gemm_decomp(h->tmA, h->tmW128, a, h->num_sms, pdl && r0 == 0, s)) != cudaSuccess)
+        return cuda_fail(e, "int8 GEMM launch");
+      if (after_chunk && (st = after_chunk(r0, rows)) != INT8MM_OK) return st;
     }
-    GemmArgs a;
-    a.M = static_cast<int>(M);
-    a.N = static_cast<int>(h->N);
-    a.K = static_cast<int>(h->K);
-    a.N_pad = static_cast<int>(h->N_pad);
-    a.c_x = h->c_x;
-    a.inv_cw = h->inv_cw;
-    a.W = Wrows;
-    a.X_OT = h->X_OT;
-    a.ld_xo = static_cast<int>(ld_xo);
-    a.idx = widx;
-    a.count = wcount;
-    a.Y = static_cast<__half*>(Y);
-    a.bias = static_cast<const __half*>(bias);
-    a.acc_dump = dbg ? dbg->acc : nullptr;
-    a.split = split;
-    a.sk_ws = h->sk_ws;
-    a.sk_ticket = h->sk_ticket;
-    a.status = h->status;
-    a.timeout_ns = h->timeout_ns;
-    a.skip_arrival = (h->test_skip & INT8MM_TEST_SKIP_SPLITK_TICKET) != 0;
-    if ((e = launch_gemm_decomp(h->tmA, h->tmW128, a, h->num_sms, pdl, s)) != cudaSuccess)
-      return cuda_fail(e, "int8 GEMM launch");
+    whole_done = true;
   }
   rec(2);
+  if (chunked) *chunked = whole_done;
   if (dbg) {
     const size_t K = static_cast<size_t>(h->K), N = static_cast<size_t>(h->N), Mz = static_cast<size_t>(M);
     struct C {
@@ -701,8 +737,49 @@ int8mm_status int8mm_forward_host(int8mm_weight_t h, const void* X_fp16_host, in
   if ((e = cudaMemcpyAsync(h->dX, X_fp16_host, static_cast<size_t>(M) * h->K * 2, cudaMemcpyHostToDevice, s)) !=
       cudaSuccess)
     return cuda_fail(e, "copy of X to the device");
-  if ((st = forward_impl(h, h->dX, M, alpha, h->dY, s, nullptr, nullptr)) != INT8MM_OK) return st;
-  if ((e = cudaMemcpyAsync(Y_fp16_host, h->dY, static_cast<size_t>(M) * h->N * 2, cudaMemcpyDeviceToHost, s)) !=
+  const size_t row_bytes = static_cast<size_t>(h->N) * 2;
+  // Tall prefills: the GEMM runs in kHostChunks row chunks (multiples of its
+  // 256-row tiles) and each chunk of Y goes back on a second stream as soon
+  // as it is written, overlapping the read-back with the next chunks (the
+  // activation pass needs all of X, so the upload stays in front).
+  const int64_t chunk = (M + kHostChunks - 1) / kHostChunks;
+  const int64_t chunk_rows = (chunk + 2 * kGemmBM - 1) / (2 * kGemmBM) * (2 * kGemmBM);
+  if (M > kDecodeMaxM && M >= 2 * chunk_rows) {
+    if (h->copy_stream == nullptr) {
+      if ((e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking)) != cudaSuccess)
+        return cuda_fail(e, "copy stream");
+      for (cudaEvent_t& ev : h->chunk_ev)
+        if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess)
+          return cuda_fail(e, "copy events");
+    }
+    int n = 0;
+    auto copy_out = [&](int64_t r0, int64_t rows) -> int8mm_status {
+      cudaError_t ce;
+      if ((ce = cudaEventRecord(h->chunk_ev[n], s)) != cudaSuccess ||
+          (ce = cudaStreamWaitEvent(h->copy_stream, h->chunk_ev[n], 0)) != cudaSuccess ||
+          (ce = cudaMemcpyAsync(static_cast<char*>(Y_fp16_host) + static_cast<size_t>(r0) * row_bytes,
+                                reinterpret_cast<char*>(h->dY) + static_cast<size_t>(r0) * row_bytes,
+                                static_cast<size_t>(rows) * row_bytes, cudaMemcpyDeviceToHost, h->copy_stream)) !=
+              cudaSuccess)
+        return cuda_fail(ce, "copy of Y to the host");
+      ++n;
+      return INT8MM_OK;
+    };
+    bool chunked = false;
+    if ((st = forward_impl(h, h->dX, M, alpha, h->dY, s, nullptr, nullptr, nullptr, chunk_rows, copy_out,
+                           &chunked)) != INT8MM_OK)
+      return st;
+    if (chunked) {
+      // `stream` is done once every chunk has arrived
+      if ((e = cudaEventRecord(h->chunk_ev[kHostChunks], h->copy_stream)) != cudaSuccess ||
+          (e = cudaStreamWaitEvent(s, h->chunk_ev[kHostChunks], 0)) != cudaSuccess)
+        return cuda_fail(e, "copy of Y to the host");
+      return INT8MM_OK;
+    }
+  } else if ((st = forward_impl(h, h->dX, M, alpha, h->dY, s, nullptr, nullptr)) != INT8MM_OK) {
+    return st;
+  }
+  if ((e = cudaMemcpyAsync(Y_fp16_host, h->dY, static_cast<size_t>(M) * row_bytes, cudaMemcpyDeviceToHost, s)) !=
       cudaSuccess)
     return cuda_fail(e, "copy of Y to the host");
   return INT8MM_OK;

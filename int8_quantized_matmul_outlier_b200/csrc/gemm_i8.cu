@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (rank == 0) mbar_arrive_expect_tx(&full[st], 2 * STAGE_BYTES);
       };
       auto load_a = [&](int st, int kb, int m_blk) {
-        const int row = m_blk * TILE_M + static_cast<int>(rank) * BM;
+        const int row = a.a_row0 + m_blk * TILE_M + static_cast<int>(rank) * BM;
         tma_load_2d_pair(smem + st * STAGE_BYTES, &tmA, full_of(st), kb * BK, row);
       };
       auto load_b = [&](int st, int kb, int n_blk) {

@@ -62,6 +62,8 @@ cudaError_t launch_row_quant(const __half* X, int64_t M, int64_t K, const Outlie
 // ---- fused tcgen05 GEMM ---------------------------------------------------
 struct GemmArgs {
   int M, N, K;
+  int a_row0;              // first row of Xq that this launch computes (M rows from there); the
+                           // row pointers below (c_x, X_OT, Y, acc_dump) start at that row
   int N_pad;               // rows per k block in the weight layout
   const float* c_x;        // [M]
   const float* inv_cw;     // [N] 1/c_w (0 where c_w == 0)

@@ -566,6 +566,26 @@ def test_captured_forward_replays_like_the_eager_one():
     m.int8mm_free(w)
 
 
+@pytest.mark.parametrize("M", [600, 2048])
+def test_host_forward_in_row_chunks_equals_the_device_forward(M):
+    # the host-buffer forward copies Y back chunk by chunk while later
+    # chunks compute: the same Y, bit for bit, as the device forward
+    p = workloads.small(M, 1040, 784, 5, seed=M + 81)
+    X = torch.from_numpy(p.X).to(dev())
+    W = torch.from_numpy(p.W).to(dev())
+    w = m.int8mm_prepare_weight(W)
+    y_dev = m.int8mm_forward(w, X, p.alpha)
+    Xh = torch.from_numpy(p.X).pin_memory()
+    Yh = torch.empty((M, 784), dtype=torch.float16).pin_memory()
+    for _ in range(2):
+        Yh.fill_(0)
+        m.int8mm_forward_host(w, Xh, p.alpha, Yh)
+        torch.cuda.synchronize()
+        assert m.int8mm_get_status(w) == m.INT8MM_OK
+        assert torch.equal(Yh, y_dev.cpu())
+    m.int8mm_free(w)
+
+
 def test_events_time_each_kernel():
     p = workloads.small(256, 1024, 1024, 3, seed=31)
     X = torch.from_numpy(p.X).to(dev())
