@@ -13,7 +13,8 @@ on its own GPU (weak scaling: the path has no exchange step); the reported
 time is the maximum over ranks.  Rank 0 prints one JSON line.
 
 Metric: effective TOPS = 2*M*N*K / time per step (the int8 contraction over
-the full K), inputs resident in HBM, L2 scrubbed (256 MB write) between steps.
+the full K), inputs resident in HBM.  Every timed step is preceded by an L2
+flush outside the timed events: a 256 MB write, then a 256 MB read.
 The headline workload is the 175B-scale FFN expansion prefill (M=2048,
 K=12288, N=49152); the same JSON line carries further sections: the OPT-13B
 prefill, the OPT-13B FFN contraction, the memory-saving weight, decode (few
@@ -49,6 +50,7 @@ METRIC = "int8-decomp matmul effective TOPS & % INT8 tensor peak; decode-shape H
 INT8_PER_BF16 = 2.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_SCRUB_BYTES = 256 << 20
+L2_BYTES = 126 << 20  # B200
 GEMM_SOURCES = ["int8_quantized_matmul_outlier_b200/csrc/gemm_i8.cu",
                 "int8_quantized_matmul_outlier_b200/csrc/ptx.cuh",
                 "int8_quantized_matmul_outlier_b200/csrc/kernels.cuh"]
@@ -130,7 +132,35 @@ def workload_config(p: workloads.Problem) -> dict:
     return {"workload": p.name, "M": M, "K": K, "N": N, "alpha": p.alpha,
             "planted_outlier_columns": int(p.planted.size),
             "inputs": "seeded synthetic fp16 (FFN-input statistics of the pages' OPT-13B example)",
-            "l2": "scrubbed between steps (256 MB write), outside the timed events"}
+            "l2": L2Flush.describe(forward_bytes(M, K, N))}
+
+
+def forward_bytes(M: int, K: int, N: int) -> int:
+    """Bytes a forward streams: X in, the int8 weight, Y out."""
+    return 2 * M * K + N * K + 2 * M * N
+
+
+class L2Flush:
+    """Keeps every timed step cold in L2: before each step, a 256 MB write
+    replaces the L2's lines and a 256 MB read then pushes the written (dirty)
+    lines back to HBM, so the timed step neither finds its data in L2 nor
+    pays for the write-back of the flush's own lines."""
+
+    def __init__(self, torch, dev):
+        self.w = torch.empty(L2_SCRUB_BYTES // 4, dtype=torch.float32, device=dev)
+        self.r = torch.ones(L2_SCRUB_BYTES // 4, dtype=torch.float32, device=dev)
+
+    @staticmethod
+    def describe(nbytes: int) -> str:
+        return ("flushed between steps (256 MB write, then 256 MB read), outside the timed events; "
+                f"the step streams {nbytes / 1e6:.0f} MB (L2 126 MB)")
+
+    def for_bytes(self, nbytes: int):
+        """The flush to run between steps of a workload of nbytes."""
+        def flush():
+            self.w.zero_()
+            self.r.sum()
+        return flush
 
 
 def measured_peaks() -> dict:
@@ -350,7 +380,7 @@ def decode_algorithmic_bytes(M: int, K: int, N: int, n_out: int) -> int:
     return N * K + 4 * N + 2 * n_out * N + 2 * M * K + 2 * M * N
 
 
-def run_decode(m, torch, dev, stream, scrub, steps: int, peaks: dict, max_over, rank: int, w=None):
+def run_decode(m, torch, dev, stream, l2, steps: int, peaks: dict, max_over, rank: int, w=None):
     """Decode steps (few tokens against the 175B-scale weight, K=12288 x
     N=49152): each step one forward, timed with events around it only, so the
     GEMM stays a programmatic dependent launch of the activation pass.  `w`
@@ -367,10 +397,12 @@ def run_decode(m, torch, dev, stream, scrub, steps: int, peaks: dict, max_over, 
         p = workloads.decode(M, repeat=rank, with_weight=False)
         X = torch.from_numpy(p.X).to(dev)
         Y = torch.empty((M, DECODE_N), dtype=torch.float16, device=dev)
-        ms = max_over(time_forwards(m, torch, w, X, p.alpha, Y, stream, scrub, steps))
+        ms = max_over(time_forwards(m, torch, w, X, p.alpha, Y, stream,
+                                    l2.for_bytes(forward_bytes(M, DECODE_K, DECODE_N)), steps))
         nbytes = decode_algorithmic_bytes(M, DECODE_K, DECODE_N, int(p.planted.size))
         gbps = nbytes / (ms * 1e-3) / 1e9
         out.append({"M": M, "K": DECODE_K, "N": DECODE_N, "ms_per_step": ms, "GBps": gbps,
+                    "l2": L2Flush.describe(forward_bytes(M, DECODE_K, DECODE_N)),
                     "frac_hbm": gbps / peaks["hbm_gbs"], "algorithmic_bytes": nbytes,
                     "gpu_launches_per_step": m.int8mm_launches_per_forward(w, M)})
     if own:
@@ -406,53 +438,55 @@ def accuracy_report(torch, dev, X, W, Y, rows: int = 32, seed: int = 0):
     return rep, r, exact_np
 
 
-def time_forwards(m, torch, w, X, alpha, Y, stream, scrub, steps: int, warm: int = 5) -> float:
+def time_forwards(m, torch, w, X, alpha, Y, stream, flush, steps: int, warm: int = 5) -> float:
     """Mean device time (ms) of whole forwards, CUDA events around each one
     only (the GEMM stays a programmatic dependent of the activation pass),
-    L2 scrubbed between steps outside the events."""
+    `flush` run between steps outside the events."""
     for _ in range(warm):
         m.int8mm_forward(w, X, alpha, Y, stream=stream)
-        scrub.zero_()
+        flush()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     torch.cuda.synchronize()
     for e0, e1 in ev:
         e0.record(stream)
         m.int8mm_forward(w, X, alpha, Y, stream=stream)
         e1.record(stream)
-        scrub.zero_()
+        flush()
     torch.cuda.synchronize()
     if m.int8mm_get_status(w) != m.INT8MM_OK:
         raise RuntimeError("device wait timed out")
     return float(np.mean([e0.elapsed_time(e1) for e0, e1 in ev]))
 
 
-def time_kernels(m, torch, w, X, alpha, Y, stream, scrub, steps: int):
+def time_kernels(m, torch, w, X, alpha, Y, stream, flush, steps: int):
     """Mean device times (ms) of the activation pass and of the GEMM, from
     an event between them (the GEMM then an ordinary launch)."""
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     torch.cuda.synchronize()
     for e in kev:
         m.int8mm_forward_events(w, X, alpha, Y, e, stream=stream)
-        scrub.zero_()
+        flush()
     torch.cuda.synchronize()
     seg = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(2)] for e in kev])
     return float(seg[:, 0].mean()), float(seg[:, 1].mean())
 
 
-def run_prefill_section(m, torch, dev, stream, scrub, p, steps: int, peak_tops: float, max_over) -> dict:
+def run_prefill_section(m, torch, dev, stream, l2, p, steps: int, peak_tops: float, max_over) -> dict:
     """Another prefill workload: whole forwards, plus the GEMM alone."""
     M, K, N = p.shape
     X = torch.from_numpy(p.X).to(dev)
     W = torch.from_numpy(p.W).to(dev)
     w = m.int8mm_prepare_weight(W)
     Y = torch.empty((M, N), dtype=torch.float16, device=dev)
-    ms = max_over(time_forwards(m, torch, w, X, p.alpha, Y, stream, scrub, steps))
-    act_ms, gemm_ms = time_kernels(m, torch, w, X, p.alpha, Y, stream, scrub, steps)
+    flush = l2.for_bytes(forward_bytes(M, K, N))
+    ms = max_over(time_forwards(m, torch, w, X, p.alpha, Y, stream, flush, steps))
+    act_ms, gemm_ms = time_kernels(m, torch, w, X, p.alpha, Y, stream, flush, steps)
     act_ms, gemm_ms = max_over(act_ms), max_over(gemm_ms)
     flops = 2.0 * M * N * K
     tops = flops / (ms * 1e-3) / 1e12
     out = {"workload": p.name, "M": M, "K": K, "N": N, "ms_per_step": ms, "TOPS": tops,
            "frac_int8_peak": tops / peak_tops, "gpu_launches_per_step": m.int8mm_launches_per_forward(w, M),
+           "l2": L2Flush.describe(forward_bytes(M, K, N)),
            "kernels_ms": {"activation pass": act_ms, "gemm_i8_decomp": gemm_ms},
            "gemm_TOPS": flops / (gemm_ms * 1e-3) / 1e12,
            "gemm_frac_int8_peak": flops / (gemm_ms * 1e-3) / 1e12 / peak_tops,
@@ -466,12 +500,12 @@ SWEEP_MS = (16, 128, 1024, 8192)
 SWEEP_OUTLIERS = (0, 1, 7, 32, 128)
 
 
-def run_sweep(m, torch, dev, stream, scrub, steps: int, peaks: dict, peak_tops: float, max_over, rank: int) -> dict:
+def run_sweep(m, torch, dev, stream, l2, steps: int, peaks: dict, peak_tops: float, max_over, rank: int) -> dict:
     """K = N = 8192 sweep: M in (16, 128, 1024, 8192) x outlier count in
     (0, 1, 7, 32, 128) at alpha = 6, plus alpha = inf (pure vector-wise int8)
     on the 7-outlier activations; the 0-outlier points stand for a small model
     with no outliers (detection runs and finds none).  Whole forwards, L2
-    scrubbed between steps (the 64 MB weight would otherwise stay in L2).
+    flushed between steps (the 64 MB weight would otherwise stay in L2).
     M <= 128 is weight-bandwidth bound (GB/s vs measured HBM), M >= 1024 tensor
     bound (TOPS vs the int8 peak); both figures are given for every point."""
     W = torch.from_numpy(workloads.weight(SWEEP_K, SWEEP_N, 4 * 1000 + 500_000 + rank)).to(dev)
@@ -484,7 +518,8 @@ def run_sweep(m, torch, dev, stream, scrub, steps: int, peaks: dict, peak_tops: 
         for n_out, alpha in runs:
             p = workloads.sweep(M, n_out, repeat=rank, alpha=alpha, with_weight=False)
             X = torch.from_numpy(p.X).to(dev)
-            ms = max_over(time_forwards(m, torch, w, X, alpha, Y, stream, scrub, steps))
+            ms = max_over(time_forwards(m, torch, w, X, alpha, Y, stream,
+                                        l2.for_bytes(forward_bytes(M, SWEEP_K, SWEEP_N)), steps))
             flops = 2.0 * M * SWEEP_N * SWEEP_K
             n_used = 0 if math.isinf(alpha) else n_out
             nbytes = decode_algorithmic_bytes(M, SWEEP_K, SWEEP_N, n_used)
@@ -500,11 +535,12 @@ def run_sweep(m, torch, dev, stream, scrub, steps: int, peaks: dict, peak_tops: 
     m.int8mm_free(w)
     return {"workload": "sweep: K=N=8192, M in (16,128,1024,8192) x |O| in (0,1,7,32,128), alpha=6; "
                         "plus alpha=inf on the |O|=7 activations",
-            "timing": "CUDA events around each whole forward, L2 scrubbed between steps",
+            "timing": "CUDA events around each whole forward; L2 flushed between steps (256 MB write, then "
+                      "256 MB read), outside the events",
             "steps_per_point": steps, "points": points}
 
 
-def run_static_weight(m, torch, dev, stream, scrub, p, X, W, Y_ref, steps: int, peak_tops: float,
+def run_static_weight(m, torch, dev, stream, l2, p, X, W, Y_ref, steps: int, peak_tops: float,
                       max_over) -> dict:
     """The headline workload with the memory-saving weight: fp16 rows kept
     only for the planted outlier dimensions (standing in for a calibrated
@@ -512,7 +548,7 @@ def run_static_weight(m, torch, dev, stream, scrub, p, X, W, Y_ref, steps: int, 
     M, K, N = p.shape
     w = m.int8mm_prepare_weight_static(W, p.planted.tolist(), max_outliers=64)
     Y = torch.empty((M, N), dtype=torch.float16, device=dev)
-    ms = max_over(time_forwards(m, torch, w, X, p.alpha, Y, stream, scrub, steps))
+    ms = max_over(time_forwards(m, torch, w, X, p.alpha, Y, stream, l2.for_bytes(forward_bytes(M, K, N)), steps))
     tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
     out = {"workload": p.name, "stored_rows": int(p.planted.size), "max_outliers": 64,
            "ms_per_step": ms, "TOPS": tops, "frac_int8_peak": tops / peak_tops,
@@ -592,13 +628,14 @@ def run_ours(args):
     w = m.int8mm_prepare_weight(W)
     m.int8mm_reserve(w, M)
     Y = torch.empty((M, N), dtype=torch.float16, device=dev)
-    scrub = torch.empty(L2_SCRUB_BYTES // 4, dtype=torch.float32, device=dev)
+    l2 = L2Flush(torch, dev)
+    flush = l2.for_bytes(forward_bytes(M, K, N))
     stream = torch.cuda.current_stream()
 
     # warm-up (untimed)
     for _ in range(args.warmup):
         m.int8mm_forward(w, X, p.alpha, Y)
-        scrub.zero_()
+        flush()
     torch.cuda.synchronize()
     if m.int8mm_get_status(w) != m.INT8MM_OK:
         raise RuntimeError("device wait timed out during warm-up")
@@ -606,7 +643,7 @@ def run_ours(args):
         # plain forwards for an ncu capture: no timing, no output
         for _ in range(args.profile_forwards):
             m.int8mm_forward(w, X, p.alpha, Y)
-            scrub.zero_()
+            flush()
         torch.cuda.synchronize()
         ok = m.int8mm_get_status(w) == m.INT8MM_OK
         m.int8mm_free(w)
@@ -627,7 +664,7 @@ def run_ours(args):
             e0.record(stream)
             m.int8mm_forward(w, X, p.alpha, Y, stream=stream)
             e1.record(stream)
-            scrub.zero_()
+            flush()
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
     barrier()
@@ -644,7 +681,7 @@ def run_ours(args):
     # launch, so these steps are timed apart from the headline ones.
     ksteps = max(1, min(steps, 200))
     barrier()
-    xprep_ms, gemm_ms = time_kernels(m, torch, w, X, p.alpha, Y, stream, scrub, ksteps)
+    xprep_ms, gemm_ms = time_kernels(m, torch, w, X, p.alpha, Y, stream, flush, ksteps)
     xprep_ms, gemm_ms = max_over(xprep_ms), max_over(gemm_ms)
 
     # end to end through the host-buffer entry point: pinned X in, pinned Y out
@@ -699,27 +736,27 @@ def run_ours(args):
     sec = args.sections
     sec_steps = max(1, min(args.decode_steps, 100))
     if "opt13b" in sec and args.config != "opt13b":
-        line["opt13b_prefill"] = run_prefill_section(m, torch, dev, stream, scrub, workloads.opt13b_prefill(repeat=rank),
+        line["opt13b_prefill"] = run_prefill_section(m, torch, dev, stream, l2, workloads.opt13b_prefill(repeat=rank),
                                                      sec_steps, peak_tops, max_over)
     if "ffn_contraction" in sec:
-        line["ffn_contraction"] = run_prefill_section(m, torch, dev, stream, scrub,
+        line["ffn_contraction"] = run_prefill_section(m, torch, dev, stream, l2,
                                                       workloads.opt13b_contraction(repeat=rank), sec_steps, peak_tops,
                                                       max_over)
     if "static_weight" in sec:
-        line["static_weight"] = run_static_weight(m, torch, dev, stream, scrub, p, X, W, Y, sec_steps, peak_tops,
+        line["static_weight"] = run_static_weight(m, torch, dev, stream, l2, p, X, W, Y, sec_steps, peak_tops,
                                                   max_over)
     if "decode" in sec and args.decode_steps > 0:
         same = (K, N) == (DECODE_K, DECODE_N)
         line["decode"] = {
             "workload": "decode: M in (1, 8, 32) tokens x K=12288 x N=49152, 7 outlier columns in every row",
-            "timing": "CUDA events around each whole forward (no event between its kernels), L2 scrubbed "
-                      "between steps; GB/s = algorithmic bytes / step time, vs measured HBM copy bandwidth",
+            "timing": "CUDA events around each whole forward (no event between its kernels); GB/s = "
+                      "algorithmic bytes / step time, vs measured HBM copy bandwidth",
             "weight": "the headline's prepared 175B-scale weight" if same else "a seeded K=12288 x N=49152 weight",
             "hbm_peak_gbs": peaks["hbm_gbs"],
-            "shapes": run_decode(m, torch, dev, stream, scrub, args.decode_steps, peaks, max_over, rank,
+            "shapes": run_decode(m, torch, dev, stream, l2, args.decode_steps, peaks, max_over, rank,
                                  w=w if same else None)}
     if "sweep" in sec and args.sweep_steps > 0:
-        line["sweep"] = run_sweep(m, torch, dev, stream, scrub, args.sweep_steps, peaks, peak_tops, max_over, rank)
+        line["sweep"] = run_sweep(m, torch, dev, stream, l2, args.sweep_steps, peaks, peak_tops, max_over, rank)
     m.int8mm_free(w)
     del W
     torch.cuda.empty_cache()

@@ -26,9 +26,10 @@
 //      the columns outside O, and equal to it unless S_i is reached in an
 //      outlier column not flagged yet;
 //   3. writes c_x[i] = 127 / S_i and the codes of every column with it.
-// Every group flags its first row before any row is quantised, so in the
-// pages' activations (a few outlier columns, large in most rows) the block's
-// bitmask already holds the outlier columns when the rows are quantised.
+// A block quantises no row before four of its rows are flagged (all of
+// them, if it has fewer), so in the pages' activations (a few outlier
+// columns, large in most rows) the block's bitmask already holds the outlier
+// columns when the rows are quantised; rows are quantised as they land.
 // Then the block ORs its bitmask into a global one and meets the other
 // blocks at a grid barrier (a release add on an arrival counter, acquire
 // polling, bounded by %globaltimer).  After it, with the global bitmask:
@@ -55,6 +56,7 @@ namespace {
 
 constexpr int kMaxWarps = 32;
 constexpr int kMaxGroups = 15;  // named barriers 1..15, one per row group
+constexpr int kFirstRows = 4;   // rows flagged before the block quantises any
 
 // Shared memory of a block: one row slot of 2K bytes and one mbarrier per
 // row group, the per-warp partial maxima, the bitmask and its word prefix
@@ -93,6 +95,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) xact_rows_kernel(RowActArgs
   uint32_t* redo_s = smax_s + R;                                                         // [R] step-5 marks
   __shared__ uint32_t s_gen;
   __shared__ int s_ok, s_count;
+  __shared__ int s_flagged;  // rows of the block flagged so far
 
   // The GEMM that follows may launch now; its blocks take the SMs this
   // kernel leaves.
@@ -104,6 +107,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) xact_rows_kernel(RowActArgs
   }
   for (int w = tid; w < KW; w += NT) mask_s[w] = 0u;
   for (int i = tid; i < R; i += NT) redo_s[i] = 0u;
+  if (tid == 0) s_flagged = 0;
   __syncthreads();
 
   // ------------------------------------------------------------- phase 1
@@ -162,17 +166,37 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) xact_rows_kernel(RowActArgs
     return true;
   };
   if (leader && my_rows > 0) issue(0);
-  // The first row of every group is flagged before any row is quantised:
-  // the outlier columns then show in the block's bitmask (in the pages'
-  // activations an outlier column is large in most rows), so S_i below
-  // leaves them out and rarely needs the correction after the barrier.
-  int ok = my_rows > 0 ? land_and_flag(0) : 1;
-  ok = __syncthreads_and(ok);
+  // Rows are quantised as they land, but only once the block has flagged
+  // kFirstRows rows (or all of its rows, if fewer): the outlier columns then
+  // show in the block's bitmask (in the pages' activations an outlier column
+  // is large in most rows), so S_i below leaves them out and rarely needs
+  // the correction after the barrier.
+  const int need_flagged = min(nr, kFirstRows);
+  int ok = 1;
   for (int j = 0; j < my_rows && ok; ++j) {
     const int lr = g + j * G;
-    if (j > 0 && !land_and_flag(j)) {
+    if (!land_and_flag(j)) {
       ok = 0;
       break;
+    }
+    group_sync(g, gthreads);  // the group's flags are in the bitmask
+    if (leader) {
+      __threadfence_block();
+      atomicAdd(&s_flagged, 1);
+    }
+    if (j == 0) {  // later rows come after the first kFirstRows anyway
+      const uint64_t t0 = global_timer_ns();
+      for (uint32_t it = 0; *reinterpret_cast<volatile int*>(&s_flagged) < need_flagged; ++it) {
+        if ((it & 15u) == 15u && global_timer_ns() - t0 > a.timeout_ns) {
+          ok = 0;
+          break;
+        }
+      }
+      __threadfence_block();
+      if (!group_all(ok)) {
+        ok = 0;
+        break;
+      }
     }
     // (2) S_i: max |x| over the columns not flagged so far (every entry
     //     above alpha is flagged, by the lane that reads it again here)
