@@ -256,14 +256,16 @@ int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns);
 int8mm_status int8mm_set_test_skip(int8mm_weight_t h, int bits);
 
 /*
- * Split of the prefill GEMM along K (forwards with M > 128, whose 256 x 256
+ * Split of the prefill GEMM along K (forwards with M > 64, whose 256 x 256
  * output tiles are computed by pairs of SMs).  0 (the default) lets the
- * library choose: it cuts each tile's K range into the S in 1..4 pieces that
- * best fill the pairs' rounds of work (K-heavy shapes with few tiles, such
- * as an FFN contraction, get S > 1).  1..4 forces S (capped at the number of
- * 128-deep k-blocks).  Piece sums are exact int32, so every S gives the
- * same results.  With S > 1 the handle holds a workspace of (S-1) x 256 KB
- * per tile.  INT8MM_ERR_INVALID_ARG for a value outside 0..4.
+ * library choose the plan that best fills the pairs' rounds of work: no
+ * split; every tile cut into S in 2..4 pieces; or, when the tiles leave a
+ * last round part-filled (such as an FFN contraction's 160 tiles for 74
+ * pairs), only the tiles past the last full round cut into up to 8 pieces
+ * spread over all pairs.  1..4 forces every tile into S pieces (capped at
+ * the number of 128-deep k-blocks).  Piece sums are exact int32, so every
+ * plan gives the same results.  A split tile needs (S-1) x 256 KB of
+ * handle workspace.  INT8MM_ERR_INVALID_ARG for a value outside 0..4.
  */
 int8mm_status int8mm_set_split_k(int8mm_weight_t h, int split);
 

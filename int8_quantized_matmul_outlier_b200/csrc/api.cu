@@ -276,18 +276,16 @@ int8mm_status ensure_decode_scratch(int8mm_weight* h, cudaStream_t s) {
   return INT8MM_OK;
 }
 
-// Pieces along K of the prefill GEMM for M rows.
-int split_for(const int8mm_weight* h, int64_t M) {
-  const int64_t num_kb = (h->K + kGemmBK - 1) / kGemmBK;
-  return h->split_override > 0 ? static_cast<int>(std::min<int64_t>(h->split_override, num_kb))
-                               : gemm_split_for(M, h->N, h->K, h->num_sms);
+// Split K of the prefill GEMM for M rows (the handle's forced split, or
+// the library's choice), and the scratch it needs: (pieces - 1) partial
+// tiles per split tile and 4 tickets per split tile.
+GemmSplit split_for(const int8mm_weight* h, int64_t M) {
+  return gemm_split_for(M, h->N, h->K, h->num_sms, h->split_override);
 }
-
-// 256 x 256 tiles of the CTA-pair GEMM for M rows.
-size_t pair_tiles(const int8mm_weight* h, int64_t M) {
-  return static_cast<size_t>((M + 2 * kGemmBM - 1) / (2 * kGemmBM)) *
-         static_cast<size_t>((h->N + kGemmBN - 1) / kGemmBN);
+size_t split_ws_elems(const GemmSplit& sp) {
+  return sp.pieces > 1 ? static_cast<size_t>(sp.pieces - 1) * sp.tail * 2 * kGemmBM * kGemmBN : 0;
 }
+size_t split_tickets(const GemmSplit& sp) { return sp.pieces > 1 ? static_cast<size_t>(sp.tail) * 4 : 0; }
 
 // Grows the split-K partial-tile workspace to ws_elems int32 and the tickets
 // to n_tickets zeroed counters, in stream order (old buffers freed on s).
@@ -457,13 +455,9 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     for (int64_t r0 = 0; r0 < M; r0 += step) {
       const int64_t rows = std::min(step, M - r0);
       // split K for the CTA-pair tiles; the scratch grows on demand
-      const int split = split_for(h, rows);
-      if (split > 1) {
-        const size_t tiles = pair_tiles(h, rows);
-        if ((st = ensure_split_scratch(h, static_cast<size_t>(split - 1) * tiles * 2 * kGemmBM * kGemmBN,
-                                       tiles * 4, s)) != INT8MM_OK)
-          return st;
-      }
+      const GemmSplit sp = split_for(h, rows);
+      if (sp.pieces > 1 && (st = ensure_split_scratch(h, split_ws_elems(sp), split_tickets(sp), s)) != INT8MM_OK)
+        return st;
       GemmArgs a;
       a.M = static_cast<int>(rows);
       a.a_row0 = static_cast<int>(r0);
@@ -480,7 +474,8 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
       a.Y = static_cast<__half*>(Y) + r0 * h->N;
       a.bias = static_cast<const __half*>(bias);
       a.acc_dump = dbg ? dbg->acc + r0 * h->N : nullptr;
-      a.split = split;
+      a.split = sp.pieces;
+      a.tail_tiles = sp.pieces > 1 ? sp.tail : 0;
       a.sk_ws = h->sk_ws;
       a.sk_ticket = h->sk_ticket;
       a.status = h->status;
@@ -672,12 +667,9 @@ int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream) {
   for (int64_t mt = 1; (mt - 1) * 2 * kGemmBM < M_max; ++mt) {
     const int64_t M = std::min<int64_t>(M_max, mt * 2 * kGemmBM);
     if (M <= kDecodeMaxM) continue;  // the decode GEMM: no split
-    const int split = split_for(h, M);
-    if (split > 1) {
-      const size_t tiles = pair_tiles(h, M);
-      ws_max = std::max(ws_max, static_cast<size_t>(split - 1) * tiles * 2 * kGemmBM * kGemmBN);
-      tickets_max = std::max(tickets_max, tiles * 4);
-    }
+    const GemmSplit sp = split_for(h, M);
+    ws_max = std::max(ws_max, split_ws_elems(sp));
+    tickets_max = std::max(tickets_max, split_tickets(sp));
   }
   if (ws_max > 0) return ensure_split_scratch(h, ws_max, tickets_max, s);
   return INT8MM_OK;

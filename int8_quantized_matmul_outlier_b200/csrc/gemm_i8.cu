@@ -173,17 +173,23 @@ __device__ __forceinline__ void transpose8x8_b16(const uint4 (&v)[8], uint4 (&t)
   }
 }
 
-// One work unit: k-blocks [kb0, kb1) of a tile; piece S-1 finishes the tile.
+// One work unit: k-blocks [kb0, kb1) of a tile cut into S pieces; piece S-1
+// finishes the tile.  With split K the last `tail` tiles are the split ones
+// (ti: a split tile's index among them); the others are whole units.
 struct Unit {
-  int tile, piece, kb0, kb1;
+  int tile, piece, S, ti, kb0, kb1;
 };
 
 template <bool SPLIT>
-__device__ __forceinline__ Unit unit_at(int u, int num_tiles, int num_kb, int split) {
-  if (!SPLIT) return Unit{u, 0, 0, num_kb};
+__device__ __forceinline__ Unit unit_at(int u, int num_tiles, int num_kb, int tail, int split) {
+  const int n_whole = num_tiles - tail;
+  if (!SPLIT || u < n_whole) return Unit{u, 0, 1, 0, 0, num_kb};
   Unit w;
-  w.piece = u / num_tiles;
-  w.tile = u - w.piece * num_tiles;
+  const int t = u - n_whole;
+  w.piece = t / tail;
+  w.ti = t - w.piece * tail;
+  w.tile = n_whole + w.ti;
+  w.S = split;
   w.kb0 = w.piece * num_kb / split;
   w.kb1 = (w.piece + 1) * num_kb / split;
   return w;
@@ -218,8 +224,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int num_n = (N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kb = (K + BK - 1) / BK;
-  const int S = SPLIT ? a.split : 1;  // pieces per tile
-  const int num_units = num_tiles * S;
+  const int S = SPLIT ? a.split : 1;        // pieces per split tile
+  const int tail = SPLIT ? a.tail_tiles : 0;  // the last `tail` tiles are split
+  const int num_units = num_tiles - tail + tail * S;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -278,7 +285,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // The weight tiles of the first k-blocks do not depend on the
       // activation pass: issue them before waiting for it, then the
       // matching activation tiles (all stages start empty).
-      const Unit first = unit_at<SPLIT>(tile0, num_tiles, num_kb, S);
+      const Unit first = unit_at<SPLIT>(tile0, num_tiles, num_kb, tail, S);
       const int pre = tile0 < num_units ? min(STAGES, first.kb1 - first.kb0) : 0;
       for (int i = 0; i < pre; ++i) {
         expect(i);
@@ -292,7 +299,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       stage = pre % STAGES;
       phase = pre == STAGES ? 1u : 0u;
       for (int u = tile0; u < num_units && ok; u += tstride) {
-        const Unit w = unit_at<SPLIT>(u, num_tiles, num_kb, S);
+        const Unit w = unit_at<SPLIT>(u, num_tiles, num_kb, tail, S);
         const int m_blk = w.tile % num_m, n_blk = w.tile / num_m;
         for (int kb = w.kb0 + (u == tile0 ? pre : 0); kb < w.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, tmo, abort_flag)) {
@@ -368,7 +375,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         return 1;
       };
       for (int u = tile0; u < num_units && ok; u += tstride, ++lt) {
-        const Unit w = unit_at<SPLIT>(u, num_tiles, num_kb, S);
+        const Unit w = unit_at<SPLIT>(u, num_tiles, num_kb, tail, S);
         const int buf = lt & 1;
         const uint32_t use = static_cast<uint32_t>(lt >> 1);
         if (!mbar_wait(&tempty[buf], (use & 1u) ^ 1u, tmo, abort_flag)) {
@@ -408,7 +415,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (ok) mma_commit_pair(&tfull[buf], 0x3);
         // the previous tile's product is complete before this one's is due
         while (ok && pend >= 0) ok = issue_chunk(true) > 0;
-        if (nchunks > 0 && w.piece == S - 1) {  // the tile is complete: its outlier product is due
+        if (nchunks > 0 && w.piece == w.S - 1) {  // the tile is complete: its outlier product is due
           pend = buf;
           pend_chunk = 0;
           pend_base = chunk_ph[buf];
@@ -494,12 +501,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tdeq[buf]), 0));
     };
     for (int u = tile0; u < num_units; u += tstride, ++lt) {
-      const Unit w = unit_at<SPLIT>(u, num_tiles, num_kb, S);
+      const Unit w = unit_at<SPLIT>(u, num_tiles, num_kb, tail, S);
       const int tile = w.tile;
       const int m_blk = tile % num_m, n_blk = tile / num_m;
       // a unit that finishes its tile (always, without split K); the others
       // only hand their partial sums on
-      const bool fin = !SPLIT || w.piece == S - 1;
+      const bool fin = w.piece == w.S - 1;
       const bool outl_u = cnt > 0 && fin;
       const int buf = lt & 1;
       const uint32_t use = static_cast<uint32_t>(lt >> 1);
@@ -528,8 +535,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (SPLIT && fin && h == 0 && tl == 0) {
         // the other pieces' partial tiles (normally stored long before): pull
         // them into L2 while the tensor cores finish this piece
-        for (int p = 0; p < S - 1; ++p)
-          bulk_prefetch_l2(a.sk_ws + ((static_cast<size_t>(p) * num_tiles + tile) * 2 + rank) * (BM * BN),
+        for (int p = 0; p < w.S - 1; ++p)
+          bulk_prefetch_l2(a.sk_ws + ((static_cast<size_t>(p) * tail + w.ti) * 2 + rank) * (BM * BN),
                            BM * BN * 4);
       }
       named_bar_sync(bar_id, 128);  // staging visible to the half's 4 warps
@@ -551,10 +558,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // int4: the workspace holds [piece][tile][CTA rank][half][chunk][int4
       // t4][row] so that a warp's access is 512 contiguous bytes
       auto part_at = [&](int p, int ch) {
-        return reinterpret_cast<int4*>(a.sk_ws + ((static_cast<size_t>(p) * num_tiles + tile) * 2 + rank) * (BM * BN)) +
+        return reinterpret_cast<int4*>(a.sk_ws + ((static_cast<size_t>(p) * tail + w.ti) * 2 + rank) * (BM * BN)) +
                (h * (HALF_N / 32) + ch) * 8 * BM + row_t;
       };
-      uint32_t* ticket = SPLIT ? a.sk_ticket + (static_cast<size_t>(tile) * 2 + rank) * 2 + h : nullptr;
+      uint32_t* ticket = SPLIT ? a.sk_ticket + (static_cast<size_t>(w.ti) * 2 + rank) * 2 + h : nullptr;
       if (SPLIT && !fin) {
         // a piece that does not finish the tile: store the partial sums,
         // then count this half on the owner's ticket
@@ -580,10 +587,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (tl == 0 && !a.skip_arrival) red_release_add_gpu(ticket, 1u);
         continue;
       }
-      if (SPLIT) {
+      if (SPLIT && w.S > 1) {
         // the owner: wait until the other S-1 pieces of this half are stored
         if (tl == 0) {
-          const uint32_t need = static_cast<uint32_t>(S - 1);
+          const uint32_t need = static_cast<uint32_t>(w.S - 1);
           int got = 1;
           if (ld_acquire_gpu_u32(ticket) != need) {
             const uint64_t t0 = global_timer_ns();
@@ -606,7 +613,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // adds the other pieces' partial sums to the 32 accumulator columns of chunk ch
       auto add_parts = [&](uint32_t(&r)[32], int ch) {
-        for (int p = 0; p < S - 1; ++p) {
+        for (int p = 0; p < w.S - 1; ++p) {
           const int4* pp = part_at(p, ch);
           int4 v[8];
 #pragma unroll
@@ -783,7 +790,7 @@ cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmA
     ++n;
   }
   const int num_tiles = ((a.M + TILE_M - 1) / TILE_M) * ((a.N + BN - 1) / BN);
-  const int units_of_work = num_tiles * (SPLIT ? a.split : 1);
+  const int units_of_work = SPLIT ? num_tiles - a.tail_tiles + a.tail_tiles * a.split : num_tiles;
   // one CTA pair per pair of SMs, all resident at once: owners of split
   // tiles wait on other pairs' pieces
   const int slots = num_sms / 2;
@@ -798,21 +805,45 @@ cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmA
 
 }  // namespace
 
-int gemm_split_for(int64_t M, int64_t N, int64_t K, int num_sms) {
+GemmSplit gemm_split_for(int64_t M, int64_t N, int64_t K, int num_sms, int force) {
   const int64_t tiles = ((M + TILE_M - 1) / TILE_M) * ((N + BN - 1) / BN);
   const int64_t pairs = std::max(1, num_sms / 2);
   const int64_t num_kb = (K + BK - 1) / BK;
-  // time of the slowest pair, in k-blocks: rounds of units x (k-blocks per
+  if (force > 0) {  // every tile in `force` pieces
+    const int s = static_cast<int>(std::min<int64_t>(force, num_kb));
+    return GemmSplit{s, s > 1 ? static_cast<int>(tiles) : 0};
+  }
+  // Time of the slowest pair, in k-blocks: rounds of units x (k-blocks per
   // unit + a fixed cost per unit of about 16 k-blocks, as measured on a
   // 2048 x 20480 x 5120 contraction: the pipeline turn-around and the
-  // owner's pass over the partial tiles)
-  auto cost = [&](int64_t s) {
-    const int64_t rounds = (tiles * s + pairs - 1) / pairs;
-    return rounds * ((num_kb + s - 1) / s + 16);
+  // owner's pass over the partial tiles).  Candidates: every tile cut into
+  // s pieces, or only the tiles past the last full round of pairs (the
+  // whole rounds then run unsplit and the leftover tiles are spread over
+  // all pairs).
+  auto cost = [&](int64_t whole, int64_t split_tiles, int64_t s) {
+    const int64_t whole_rounds = (whole + pairs - 1) / pairs;
+    const int64_t split_rounds = (split_tiles * s + pairs - 1) / pairs;
+    return whole_rounds * (num_kb + 16) + split_rounds * ((num_kb + s - 1) / s + 16);
   };
-  int best = 1;
-  for (int s = 2; s <= kGemmMaxSplit && num_kb / s >= 8; ++s)
-    if (cost(s) < cost(best)) best = s;
+  GemmSplit best{1, 0};
+  int64_t best_cost = cost(tiles, 0, 1);
+  const int64_t leftover = tiles % pairs;
+  for (int s = 2; s <= kGemmMaxTailSplit && num_kb / s >= 8; ++s) {
+    if (s <= kGemmMaxSplit) {
+      const int64_t c = cost(0, tiles, s);
+      if (c < best_cost) {
+        best_cost = c;
+        best = GemmSplit{s, static_cast<int>(tiles)};
+      }
+    }
+    if (leftover > 0 && leftover < tiles) {
+      const int64_t c = cost(tiles - leftover, leftover, s);
+      if (c < best_cost) {
+        best_cost = c;
+        best = GemmSplit{s, static_cast<int>(leftover)};
+      }
+    }
+  }
   return best;
 }
 

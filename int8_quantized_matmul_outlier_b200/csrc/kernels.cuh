@@ -75,9 +75,10 @@ struct GemmArgs {
   __half* Y;               // [M,N] fp16 output
   const __half* bias;      // [N] fp16 layer bias added before the rounding, or nullptr
   int32_t* acc_dump;       // [M,N] int32 accumulators, or nullptr
-  int split;               // pieces per tile along K (CTA pairs): 1, or 2 .. kGemmMaxSplit
-  int32_t* sk_ws;          // split > 1: [split-1][tiles][2][128][256] int32 partial tiles
-  uint32_t* sk_ticket;     // split > 1: [tiles][2][2] counters, zero between launches
+  int split;               // pieces per split tile along K: 1, or 2 .. kGemmMaxTailSplit
+  int tail_tiles;          // split > 1: the last tail_tiles tiles are split (the others whole)
+  int32_t* sk_ws;          // split > 1: [split-1][tail_tiles][2][128][256] int32 partial tiles
+  uint32_t* sk_ticket;     // split > 1: [tail_tiles][2][2] counters, zero between launches
   int* status;             // device status word
   unsigned long long timeout_ns;
   int skip_arrival;        // failure-detection test only: split-K pieces do not count
@@ -92,10 +93,16 @@ struct GemmArgs {
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 128;
-constexpr int kGemmMaxSplit = 4;
-// Pieces along K per 256x256 tile of the CTA-pair GEMM for an M x N x K
-// problem: the split that best fills the pairs' rounds of work.
-int gemm_split_for(int64_t M, int64_t N, int64_t K, int num_sms);
+constexpr int kGemmMaxSplit = 4;      // pieces when every tile is split (also the forced range)
+constexpr int kGemmMaxTailSplit = 8;  // pieces when only the leftover tiles are split
+// Split K of the CTA-pair GEMM for an M x N x K problem: the last `tail`
+// tiles (of the n-major order) are cut into `pieces` along K, the others
+// are whole; pieces == 1 is no split.  `force` > 0 cuts every tile into
+// that many pieces; 0 picks the plan that best fills the pairs' rounds.
+struct GemmSplit {
+  int pieces, tail;
+};
+GemmSplit gemm_split_for(int64_t M, int64_t N, int64_t K, int num_sms, int force);
 // With `pdl`, launched as a programmatic dependent of the activation pass:
 // its prologue and the first weight-tile loads overlap that pass.
 cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,

@@ -248,6 +248,22 @@ def test_split_k(M, K, N, n_out, alpha, split):
     m.int8mm_free(w)
 
 
+def test_split_of_the_leftover_tiles_only():
+    # 8 x 10 = 80 tiles for 74 pairs: the library runs 74 tiles whole and
+    # cuts the 6 left over into pieces spread over all pairs
+    p = workloads.small(2048, 4096, 2560, 5, seed=91)
+    out = check(p, rows=sample_rows(2048, 64, seed=91))
+    assert out["cnt"] == 5
+    w = out["w"]
+    X = torch.from_numpy(p.X).to(dev())
+    y_auto = m.int8mm_forward(w, X, p.alpha)
+    m.int8mm_set_split_k(w, 1)
+    y_one = m.int8mm_forward(w, X, p.alpha)
+    torch.cuda.synchronize()
+    assert torch.equal(y_auto, y_one)
+    m.int8mm_free(w)
+
+
 def test_split_k_with_bias():
     M, K, N = 300, 2064, 784
     p = workloads.small(M, K, N, 5, seed=17)
