@@ -129,13 +129,17 @@ int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream);
  * alpha: outlier threshold (6.0 in the pages); INFINITY disables the fp16
  *   path (pure vector-wise int8); any value below every |x| makes every
  *   column an outlier.  NaN is an argument error.
- * M == 0 is a no-op.  Two or three kernels run on `stream`: the activation
- * pass (outlier detection, row quantisation and the outlier gather) and the
- * fused int8 GEMM, a programmatic dependent launch that starts while the
- * activation pass finishes.  The activation pass is one kernel for up to
- * 256 rows per SM (37888 on a 148-SM B200), else two (detection, then
- * quantisation); a static weight adds the gather of the outlier rows; see
- * int8mm_launches_per_forward.  The outlier count never leaves the device,
+ * M == 0 is a no-op.  Decode shapes (M <= 64, K <= 16384) run as ONE
+ * kernel on `stream`: the decode GEMM (a cooperative launch) does the
+ * activation pass itself, each CTA on a slice of X's columns, with two grid
+ * barriers, while its first weight tiles already stream.  Otherwise two or
+ * three kernels run: the activation pass (outlier detection, row
+ * quantisation and the outlier gather) and the fused int8 GEMM, a
+ * programmatic dependent launch that starts while the activation pass
+ * finishes.  That activation pass is one kernel for up to 256 rows per SM
+ * (37888 on a 148-SM B200), else two (detection, then quantisation); a
+ * static weight adds the gather of the outlier rows (and always takes the
+ * separate activation pass); see int8mm_launches_per_forward.  The outlier count never leaves the device,
  * so the call does not synchronise.  Grows the workspace when M exceeds every
  * earlier M (stream-ordered allocation).
  */
@@ -174,7 +178,9 @@ int8mm_status int8mm_forward_host(int8mm_weight_t h, const void* X_fp16_host, in
  * before the activation pass, between it and the GEMM, and after the
  * GEMM, so that the GEMM can be timed on the stream it runs on.  A middle
  * event makes the GEMM an ordinary launch instead of a programmatic
- * dependent of the activation pass (its prologue then no longer overlaps it).
+ * dependent of the activation pass (its prologue then no longer overlaps it),
+ * and makes decode shapes take the separate activation pass too (the same
+ * results as the single decode kernel, which has no point between the two).
  */
 int8mm_status int8mm_forward_events(int8mm_weight_t h, const void* X_fp16_dev, int64_t M, float alpha,
                                     void* Y_fp16_dev, void* stream, void* const events[3]);
@@ -207,7 +213,7 @@ int8mm_status int8mm_forward_debug(int8mm_weight_t h, const void* X_fp16_dev, in
  * After a timeout, the forward that timed out AND every later forward on the
  * handle are invalid until this call has returned INT8MM_ERR_TIMEOUT: an
  * aborted kernel can leave counters (split-K and decode tickets, the
- * activation pass's grid barrier) that a later forward would misread, and
+ * activation pass's grid barriers and row maxima) that a later forward would misread, and
  * this call is what resets them.
  */
 int8mm_status int8mm_get_status(int8mm_weight_t h);
@@ -247,7 +253,9 @@ int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns);
  *   INT8MM_TEST_SKIP_DECODE_TICKET    split n blocks of the decode GEMM (M <=
  *                                     64) likewise;
  *   INT8MM_TEST_SKIP_BARRIER_ARRIVAL  block 0 of the single-launch activation
- *                                     pass does not arrive at its grid barrier.
+ *                                     pass does not arrive at its grid barrier,
+ *                                     nor CTA 0 of the decode GEMM at the first
+ *                                     barrier of its own activation pass.
  * INT8MM_ERR_INVALID_ARG for other bits.
  */
 #define INT8MM_TEST_SKIP_SPLITK_TICKET 1
@@ -273,8 +281,8 @@ int8mm_status int8mm_set_split_k(int8mm_weight_t h, int split);
 int8mm_status int8mm_weight_bytes(int8mm_weight_t h, size_t* bytes);
 
 /* Number of kernels a forward of M rows launches with this handle (0 for
- * M == 0, else 2 or 3, one more for a static weight).  Host-side only;
- * nothing is enqueued. */
+ * M == 0; 1 for decode shapes that run as one kernel; else 2 or 3, one more
+ * for a static weight).  Host-side only; nothing is enqueued. */
 int8mm_status int8mm_launches_per_forward(int8mm_weight_t h, int64_t M, int* count);
 
 /*

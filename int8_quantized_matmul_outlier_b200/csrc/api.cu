@@ -57,6 +57,7 @@ struct int8mm_weight {
   // the grid barrier's arrival counter and generation
   uint32_t* omask = nullptr;  // [2][ceil(K/32)]
   uint32_t* xsync = nullptr;  // [4]: arrivals by generation parity, generation
+  uint32_t* rowmax = nullptr;  // [kDecodeMaxM][kRowMaxStride] row maxima of the decode kernel's own activation pass
   int32_t* idx = nullptr;
   int32_t* count = nullptr;
   float* colmax = nullptr;
@@ -205,6 +206,7 @@ void free_all(int8mm_weight* h) {
   release(&h->pre);
   release(&h->omask);
   release(&h->xsync);
+  release(&h->rowmax);
   release(&h->idx);
   release(&h->count);
   release(&h->colmax);
@@ -379,7 +381,16 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     if (events && events[i]) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
   };
   rec(0);
-  if (row_act_fits(M, h->K, h->num_sms)) {
+  // Decode shapes run the activation pass inside the decode GEMM's launch
+  // (not with a static weight, whose outlier rows are gathered in between,
+  // nor when events should time the two passes apart).
+  const bool fused = decode && !h->wstatic && !(events && events[1]) &&
+                     decode_fused_fits(M, h->K, h->N, h->num_sms);
+  if (fused) {
+    // the debug dump's column maxima come from the detection kernel
+    if (dbg && (e = launch_outlier_detect(Xh, M, h->K, alpha, sc, s)) != cudaSuccess)
+      return cuda_fail(e, "outlier detection launch");
+  } else if (row_act_fits(M, h->K, h->num_sms)) {
     RowActArgs ra;
     ra.X = Xh;
     ra.M = static_cast<int>(M);
@@ -445,6 +456,17 @@ int8mm_status forward_impl(int8mm_weight* h, const void* X, int64_t M, float alp
     d.status = h->status;
     d.timeout_ns = h->timeout_ns;
     d.skip_arrival = (h->test_skip & INT8MM_TEST_SKIP_DECODE_TICKET) != 0;
+    d.X = fused ? Xh : nullptr;
+    d.thr = half_magnitude_threshold(alpha);
+    d.Xq_out = h->Xq;
+    d.c_x_out = h->c_x;
+    d.X_OT_out = h->X_OT;
+    d.idx_out = h->idx;
+    d.count_out = h->count;
+    d.omask = h->omask;
+    d.sync = h->xsync;
+    d.rowmax = h->rowmax;
+    d.skip_barrier = (h->test_skip & INT8MM_TEST_SKIP_BARRIER_ARRIVAL) != 0;
     if ((e = launch_gemm_decode(h->tmW128, h->tmA, d, h->num_sms, pdl, s)) != cudaSuccess)
       return cuda_fail(e, "int8 decode GEMM launch");
   } else {
@@ -559,7 +581,8 @@ int8mm_status prepare_impl(const void* W_fp16_dev, int64_t K, int64_t N, void* s
       (e = alloc(&h->colkey, Kz, s, tot)) != cudaSuccess || (e = alloc(&h->epoch, 1, s, tot)) != cudaSuccess ||
       (e = alloc(&h->ticket, 1, s, tot)) != cudaSuccess || (e = alloc(&h->mask, words, s, tot)) != cudaSuccess ||
       (e = alloc(&h->pre, words, s, tot)) != cudaSuccess || (e = alloc(&h->omask, 2 * words, s, tot)) != cudaSuccess ||
-      (e = alloc(&h->xsync, 4, s, tot)) != cudaSuccess || (e = alloc(&h->idx, Kz, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->xsync, 4, s, tot)) != cudaSuccess || (e = alloc(&h->rowmax, kDecodeMaxM * kRowMaxStride, s, tot)) != cudaSuccess ||
+      (e = alloc(&h->idx, Kz, s, tot)) != cudaSuccess ||
       (e = alloc(&h->count, 1, s, tot)) != cudaSuccess || (e = alloc(&h->colmax, Kz, s, tot)) != cudaSuccess ||
       (e = alloc(&h->status, 1, s, tot)) != cudaSuccess) {
     cudaStreamSynchronize(s);
@@ -574,6 +597,7 @@ int8mm_status prepare_impl(const void* W_fp16_dev, int64_t K, int64_t N, void* s
       (e = cudaMemsetAsync(h->mask, 0, words * 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->omask, 0, 2 * words * 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->xsync, 0, 16, s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(h->rowmax, 0, kDecodeMaxM * kRowMaxStride * 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->count, 0, 4, s)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->status, 0, 4, s)) != cudaSuccess ||
       (e = launch_weight_prep(h->W, K, N, h->colmax_bits, h->Wb, h->N_pad, h->c_w, h->inv_cw, h->num_sms, s)) !=
@@ -794,8 +818,10 @@ int8mm_status int8mm_get_status(int8mm_weight_t h) {
     if (h->dticket) cudaMemset(h->dticket, 0, static_cast<size_t>((h->N + 127) / 128) * 4);
     // an aborted split-K GEMM its tile tickets,
     if (h->sk_ticket) cudaMemset(h->sk_ticket, 0, h->sk_ticket_n * 4);
-    // and an aborted single-launch activation pass its barrier counts and bitmasks
+    // and an aborted single-launch activation pass (separate or inside the
+    // decode GEMM) its barrier counts, bitmasks and row maxima
     cudaMemset(h->xsync, 0, 16);
+    cudaMemset(h->rowmax, 0, kDecodeMaxM * kRowMaxStride * 4);
     cudaMemset(h->omask, 0, static_cast<size_t>((h->K + 31) / 32) * 8);
     cudaDeviceSynchronize();
     return fail(INT8MM_ERR_TIMEOUT, "a device wait ran out of time");
@@ -861,6 +887,7 @@ int8mm_status int8mm_launches_per_forward(int8mm_weight_t h, int64_t M, int* cou
   if (!live(h) || count == nullptr) return fail(INT8MM_ERR_INVALID_ARG, "invalid handle or NULL output");
   if (M < 0) return fail(INT8MM_ERR_INVALID_ARG, "M=%lld is negative", (long long)M);
   if (M == 0) *count = 0;
+  else if (M <= kDecodeMaxM && !h->wstatic && decode_fused_fits(M, h->K, h->N, h->num_sms)) *count = 1;
   else *count = row_act_fits(M, h->K, h->num_sms) ? 2 : 3;
   if (M > 0 && h->wstatic) *count += 1;  // the outlier row gather
   return INT8MM_OK;

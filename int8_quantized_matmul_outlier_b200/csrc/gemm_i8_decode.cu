@@ -23,12 +23,35 @@
 // wait only on pieces that wait on nothing.  Integer sums make the result
 // independent of order.
 //
+// Activation pass in the same launch (for K up to 16384): the CTAs are
+// co-resident (a cooperative launch), and CTA c of G takes the columns
+// [8 v0, 8 v1) of X, v0 = c nvec / G (nvec = K/8).  Its epilogue warps, idle
+// until the first accumulator is ready, load X[0..M, slice] once and
+//   1. flag the slice's outlier columns, exactly: all M rows are at hand;
+//   2. take each row's absmax over the slice's columns outside O, fold it
+//      into a global per-row maximum (atomicMax on the magnitude bits) and
+//      OR the flags into a global bitmask;
+//   3. meet the other CTAs at a grid barrier; then c_x = 127/absmax of every
+//      row, the codes of the slice (outlier columns 0), and, from the
+//      bitmask's bits before the slice, the positions in O of the slice's
+//      outlier columns: idx and X_OT for them;
+//   4. meet at a second grid barrier, after which the producer loads the
+//      token tiles of Xq with TMA.
+// Meanwhile the producer has issued the first ring of weight tiles and
+// prefetched the next ones into L2, so the weight streams from the first
+// instruction on.  The barrier state (bitmasks, arrival counters and the
+// generation word) is the one the separate activation pass keeps, with the
+// same rule: the launch of generation g uses the parity-g buffers, finds
+// them zero, and clears the parity-(g+1) ones for the next launch.
+//
 // Warps: 0 TMA producer (weight tile + token tile per stage, 6-deep ring,
-// weight loads marked evict-first in L2; the first weight tiles are issued
-// before waiting on the activation pass), 1 MMA issuer and TMEM owner (double-buffered 128 x MP int32
+// weight loads marked evict-first in L2; the first ring of weight tiles is
+// loaded, and the next D_PF_TILES prefetched into L2, before waiting on the
+// activation pass), 1 MMA issuer and TMEM owner (double-buffered 128 x MP int32
 // accumulator), 2-9 epilogue (one output column n per thread, half of the
 // tokens: two warps share each TMEM lane quarter).
 // Every wait is bounded; a timeout sets the status word and the CTA exits.
+#include "actq.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -42,6 +65,9 @@ constexpr int DBK = 128;  // K bytes per stage
 // Six stages of weight tiles in flight per SM measured faster than deeper
 // rings (4: slower, 11: 12% slower): more outstanding reads only congest HBM.
 constexpr int D_STAGES = 6;
+// Weight tiles past the ring that the producer prefetches into L2 before it
+// waits for the activation pass (at most this many per CTA, 16 KB each).
+constexpr int D_PF_TILES = 24;
 constexpr int D_OUT_STAGE = 128;  // outliers whose activations (and indices) are staged in smem
 constexpr int D_EPI = 256;  // epilogue threads: eight warps
 constexpr int D_THREADS = 64 + D_EPI;
@@ -53,12 +79,18 @@ struct DCfg {
   static constexpr int STAGE = W_BYTES + X_BYTES;
   static constexpr int STAGES = D_STAGES;
   static constexpr int BAR_OFF = STAGES * STAGE;
-  static constexpr int NBARS = 2 * STAGES + 5;
+  static constexpr int NBARS = 2 * STAGES + 6;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-  static constexpr int XO_OFF = (MISC_OFF + 32 + 15) & ~15;        // half [D_OUT_STAGE][64]
+  // half [D_OUT_STAGE][64]; before the outliers are staged, the fused
+  // activation pass's slice of X, uint4 [64 rows][16 vectors] (16 KB too)
+  static constexpr int XO_OFF = (MISC_OFF + 32 + 15) & ~15;
   static constexpr int RX_OFF = XO_OFF + D_OUT_STAGE * 64 * 2;     // float [64]
   static constexpr int IDX_OFF = RX_OFF + 64 * 4;                  // int [D_OUT_STAGE]
-  static constexpr int SMEM = IDX_OFF + D_OUT_STAGE * 4 + 1024;
+  static constexpr int CX_OFF = IDX_OFF + D_OUT_STAGE * 4;         // float [64]: c_x (fused)
+  static constexpr int FL_OFF = CX_OFF + 64 * 4;                   // u32 [16]: flags per vector (fused)
+  static constexpr int OL_OFF = FL_OFF + 16 * 4;                   // u32 [128]: the slice's outliers (fused)
+  static constexpr int RED_OFF = OL_OFF + 128 * 4;                 // u32 [16]: reductions (fused)
+  static constexpr int SMEM = RED_OFF + 16 * 4 + 1024;
   // outlier weight values prefetched into registers per segment
   static constexpr int WCAP = 16;
   static constexpr int TMEM_COLS = 2 * MP < 32 ? 32 : 2 * MP;
@@ -78,6 +110,26 @@ __device__ __forceinline__ void dfail(const DecodeArgs& a, volatile int* abort_f
   atomicOr(a.status, kStatusTimeout);
 }
 
+// Persistent CTAs of the decode GEMM: one per SM, at most one per
+// (n block, k block) step.
+int64_t decode_grid(int64_t N, int64_t K, int num_sms) {
+  const int64_t total = ((N + DBM - 1) / DBM) * ((K + DBK - 1) / DBK);
+  return std::max<int64_t>(1, std::min<int64_t>(total, num_sms));
+}
+
+// Grid barrier of the fused activation pass (one thread per CTA): optionally
+// counts this CTA with a release add, then waits (acquire) until the counter
+// reaches `target`; false once timeout_ns have passed.
+__device__ __forceinline__ bool grid_wait(uint32_t* ctr, uint32_t target, bool arrive, uint64_t timeout_ns) {
+  if (arrive) red_release_add_gpu(ctr, 1u);
+  if (ld_acquire_gpu_u32(ctr) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire_gpu_u32(ctr) >= target) return true;
+    if ((it & 15u) == 0 && global_timer_ns() - t0 > timeout_ns) return false;
+  }
+}
+
 // One segment of a CTA's range: n block `nb`, k blocks [kb0, kb1).
 struct Seg {
   int nb, kb0, kb1;
@@ -92,7 +144,7 @@ __device__ __forceinline__ Seg segment_at(long long u, long long u_end, int num_
   return s;
 }
 
-template <int MP>
+template <int MP, bool FUSED>
 __global__ void __launch_bounds__(D_THREADS, 1)
     gemm_i8_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                           const DecodeArgs a) {
@@ -105,12 +157,14 @@ __global__ void __launch_bounds__(D_THREADS, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
+  uint64_t* act_ready = drain + 1;  // fused: the token tiles of Xq may be loaded
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
   volatile int* s_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 8);
   __half* xo_s = reinterpret_cast<__half*>(smem + C::XO_OFF);
   float* rx_s = reinterpret_cast<float*>(smem + C::RX_OFF);
   int* idx_s = reinterpret_cast<int*>(smem + C::IDX_OFF);
+  float* cx_s = reinterpret_cast<float*>(smem + C::CX_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = a.M, N = a.N, K = a.K;
@@ -130,6 +184,7 @@ __global__ void __launch_bounds__(D_THREADS, 1)
       mbar_init(&tempty[b], D_EPI / 32);
     }
     mbar_init(drain, 1);
+    mbar_init(act_ready, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmW);
@@ -138,6 +193,24 @@ __global__ void __launch_bounds__(D_THREADS, 1)
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
+  }
+  // fused: the epilogue warps start loading their slice of X right away
+  // (vectors e = et + j D_EPI of the [M][16] slice; see the activation pass)
+  constexpr int XR = 64 * 16 / D_EPI;
+  uint4 xr[XR];
+  int xv0 = 0, xnv = 0;
+  if constexpr (FUSED) {
+    const int nvec = K >> 3;
+    xv0 = static_cast<int>(static_cast<long long>(nvec) * blockIdx.x / gridDim.x);
+    xnv = static_cast<int>(static_cast<long long>(nvec) * (blockIdx.x + 1) / gridDim.x) - xv0;  // <= 16
+    if (warp >= 2) {
+      const uint4* X4 = reinterpret_cast<const uint4*>(a.X);
+#pragma unroll
+      for (int j = 0; j < XR; ++j) {
+        const int e = static_cast<int>(threadIdx.x) - 64 + j * D_EPI, m = e >> 4, v = e & 15;
+        xr[j] = (m < M && v < xnv) ? __ldg(X4 + static_cast<size_t>(m) * nvec + xv0 + v) : make_uint4(0, 0, 0, 0);
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -161,7 +234,23 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         mbar_arrive_expect_tx(&full[i], C::STAGE);
         tma_load_2d_hint(smem + i * C::STAGE, &tmW, &full[i], 0, kb * a.N_pad + nb * DBM, wpol);
       }
-      dpdl_wait();
+      // and the next tiles of the range into L2, so that the weight streams
+      // from HBM while the activation pass runs
+      const long long pf_end = min(u_end, u_begin + pre + D_PF_TILES);
+      for (long long uu = u_begin + pre; uu < pf_end; ++uu) {
+        const int nb = static_cast<int>(uu / num_kb), kb = static_cast<int>(uu % num_kb);
+        tma_prefetch_2d(&tmW, 0, kb * a.N_pad + nb * DBM);
+      }
+      if constexpr (FUSED) {
+        // Xq is written by the CTAs' activation pass; the epilogue warps
+        // signal after its second grid barrier (also when a barrier ran
+        // out, with the abort flag set: the token tiles are loaded all the
+        // same, so that every issued stage completes)
+        if (!mbar_wait(act_ready, 0, 3 * tmo, nullptr)) dfail(a, abort_flag);
+        fence_proxy_async_global();
+      } else {
+        dpdl_wait();
+      }
       for (int i = 0; i < pre; ++i) {
         const int kb = static_cast<int>((u_begin + i) % num_kb);
         tma_load_2d(smem + i * C::STAGE + C::W_BYTES, &tmX, &full[i], kb * DBK, 0);
@@ -242,20 +331,172 @@ __global__ void __launch_bounds__(D_THREADS, 1)
     // Two warps per TMEM lane quarter (warp w may read lanes 32 (w % 4) ..):
     // warps 2-5 take tokens [0, HM), warps 6-9 tokens [HM, MP).
     constexpr int HM = MP / 2;
+    constexpr int HC = HM > 16 ? 16 : HM;  // tokens per chunk of the epilogue
     const int q = warp & 3;
     const int m0 = ((warp - 2) >> 2) * HM;
     const int n_local = q * 32 + lane;
     const int et = threadIdx.x - 64;  // 0 .. D_EPI-1
-    dpdl_wait();  // count, idx, X_OT and c_x come from the activation pass
-    const int cnt = *a.count;
+    if constexpr (FUSED) {
+      // ------------------------------------------ activation pass of the slice
+      uint4* xs = reinterpret_cast<uint4*>(smem + C::XO_OFF);  // [64][16] (aliases xo_s)
+      uint32_t* fl_s = reinterpret_cast<uint32_t*>(smem + C::FL_OFF);
+      uint32_t* ol_s = reinterpret_cast<uint32_t*>(smem + C::OL_OFF);
+      uint32_t* red_s = reinterpret_cast<uint32_t*>(smem + C::RED_OFF);
+      volatile uint32_t* s_gen = reinterpret_cast<volatile uint32_t*>(smem + C::MISC_OFF + 12);
+      volatile int* s_nloc = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 16);
+      const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
+      const int KW = (K + 31) >> 5;
+      const int v0 = xv0, nv = xnv;
+      if (et == 0) *s_gen = *reinterpret_cast<volatile uint32_t*>(a.sync + 2);
+      // (0) X[0..M, 8 v0 .. 8 (v0 + nv)): 16 vectors of 8 columns per row,
+      //     loaded before the setup barrier
+#pragma unroll
+      for (int j = 0; j < XR; ++j) {
+        const int e = et + j * D_EPI;
+        if (e < M * 16) xs[e] = xr[j];
+      }
+      dbar_sync(1, D_EPI);
+      // (1) outlier flags of the slice's columns (one thread per column, one
+      //     flag byte per vector)
+      {
+        bool out = false;
+        if (et < nv * 8) {
+          const unsigned short* hs = reinterpret_cast<const unsigned short*>(xs) + et;
+          uint32_t mx = 0u;
+          for (int m = 0; m < M; ++m) mx = max(mx, static_cast<uint32_t>(hs[m * 128] & 0x7fffu));
+          out = a.thr < 0 || mx > static_cast<uint32_t>(a.thr);
+        }
+        if (et < 128) {  // whole warps: columns et of vectors et / 8
+          const uint32_t b = __ballot_sync(0xffffffffu, out);
+          if (lane < 4) fl_s[(et >> 5) * 4 + lane] = (b >> (8 * lane)) & 0xffu;
+        }
+      }
+      dbar_sync(1, D_EPI);
+      // (2) the flags into this generation's bitmask; per row, the absmax over
+      //     the slice's columns outside O into the global maximum (16 lanes
+      //     per row, reduced by shuffles)
+      const uint32_t gen = *s_gen;
+      uint32_t* gmask = a.omask + static_cast<size_t>(gen & 1u) * KW;
+      if (et < nv && fl_s[et] != 0u) atomicOr(gmask + ((v0 + et) >> 2), fl_s[et] << (((v0 + et) & 3) * 8));
+      for (int base = 0; base < M * 16; base += D_EPI) {
+        const int e = base + et, m = e >> 4, v = e & 15;
+        uint32_t r = 0u;
+        if (e < M * 16 && v < nv) r = max_pair(masked_absmax2(0u, xs[e], fl_s[v]));
+        r = max(r, __shfl_xor_sync(0xffffffffu, r, 8));
+        r = max(r, __shfl_xor_sync(0xffffffffu, r, 4));
+        r = max(r, __shfl_xor_sync(0xffffffffu, r, 2));
+        r = max(r, __shfl_xor_sync(0xffffffffu, r, 1));
+        if (e < M * 16 && v == 0 && r != 0u) atomicMax(a.rowmax + m * kRowMaxStride, r);
+      }
+      // (3) grid barrier: every CTA's flags and row maxima are in
+      dbar_sync(1, D_EPI);
+      if (et == 0) {
+        const bool arrive = !(a.skip_barrier && cta == 0);
+        const bool ok1 = grid_wait(a.sync + (gen & 1u), static_cast<uint32_t>(G), arrive, tmo);
+        if (!ok1) dfail(a, abort_flag);
+        *s_flag = ok1 ? 1 : 0;
+      }
+      dbar_sync(1, D_EPI);
+      if (*s_flag) {
+        // (4) the row maxima and the bitmask, read together: the scales of
+        //     all rows (CTA 0 writes them out), and the position in O of the
+        //     slice's first column, i.e. the bits of the bitmask before it
+        //     (for CTA 0 also |O|: all of them)
+        const uint32_t rmax = et < M ? __ldcg(a.rowmax + et * kRowMaxStride) : 0u;
+        const int wf = v0 >> 2;
+        const uint32_t below = (1u << ((v0 & 3) * 8)) - 1u;
+        uint32_t before = 0u, total = 0u;
+        for (int w = et; w < KW; w += D_EPI) {
+          const uint32_t bits = __ldcg(gmask + w);
+          total += __popc(bits);
+          before += w < wf ? __popc(bits) : (w == wf ? __popc(bits & below) : 0);
+        }
+        if (et < M) {
+          const float c = scale_from_absmax_bits(rmax);
+          cx_s[et] = c;
+          if (cta == 0) a.c_x_out[et] = c;
+        }
+        before = __reduce_add_sync(0xffffffffu, before);
+        total = __reduce_add_sync(0xffffffffu, total);
+        if (lane == 0) {
+          red_s[2 * (warp - 2)] = before;
+          red_s[2 * (warp - 2) + 1] = total;
+        }
+        dbar_sync(1, D_EPI);
+        // the codes of the slice, outlier columns 0
+        for (int e = et; e < M * 16; e += D_EPI) {
+          const int m = e >> 4, v = e & 15;
+          if (v < nv) {
+            const uint32_t fl = fl_s[v];
+            uint2 q = quant8_fma(xs[e], cx_s[m]);
+            q.x &= ~expand_nibble(fl & 0xfu);
+            q.y &= ~expand_nibble(fl >> 4);
+            *reinterpret_cast<uint2*>(a.Xq_out + static_cast<size_t>(m) * K + static_cast<size_t>(v0 + v) * 8) = q;
+          }
+        }
+        // (5) the slice's outlier columns: idx and their local list
+        if (et == 0) {
+          uint32_t o = 0u, n_all = 0u;
+          for (int u = 0; u < D_EPI / 32; ++u) {
+            o += red_s[2 * u];
+            n_all += red_s[2 * u + 1];
+          }
+          int n = 0;
+          for (int v = 0; v < nv; ++v) {
+            uint32_t b = fl_s[v];
+            while (b != 0u) {
+              const int q = __ffs(static_cast<int>(b)) - 1;
+              b &= b - 1u;
+              a.idx_out[o] = (v0 + v) * 8 + q;
+              ol_s[n++] = (o << 8) | static_cast<uint32_t>(v * 8 + q);
+              ++o;
+            }
+          }
+          *s_nloc = n;
+          if (cta == 0) *a.count_out = static_cast<int32_t>(n_all);
+        }
+        dbar_sync(1, D_EPI);
+        // (6) X_OT for the slice's outlier columns
+        const int n_loc = *s_nloc;
+        for (int e = et; e < n_loc * M; e += D_EPI) {
+          const int j = e / M, m = e - j * M;
+          const uint32_t oc = ol_s[j];
+          a.X_OT_out[static_cast<size_t>(oc >> 8) * a.ld_xo + m] =
+              reinterpret_cast<const __half*>(xs)[m * 128 + static_cast<int>(oc & 255u)];
+        }
+        // the next launch's bitmask and arrival counter start at zero
+        if (cta == 0) {
+          uint32_t* next = a.omask + static_cast<size_t>((gen + 1u) & 1u) * KW;
+          for (int w = et; w < KW; w += D_EPI) next[w] = 0u;
+          if (et == 0) a.sync[(gen + 1u) & 1u] = 0u;
+        }
+        fence_proxy_async_global();  // other CTAs read these codes with TMA
+        // (7) second grid barrier: Xq, c_x, idx, count and X_OT are out
+        dbar_sync(1, D_EPI);
+        if (et == 0) {
+          const bool ok2 = grid_wait(a.sync + (gen & 1u), 2u * static_cast<uint32_t>(G), true, tmo);
+          if (!ok2) dfail(a, abort_flag);
+          else if (cta == 0) a.sync[2] = gen + 1u;
+          *s_flag = ok2 ? 1 : 0;
+        }
+        dbar_sync(1, D_EPI);
+        // every CTA read the row maxima before it arrived
+        if (*s_flag && cta == 0 && et < kDecodeMaxM) a.rowmax[et * kRowMaxStride] = 0u;
+      }
+      if (et == 0) mbar_arrive(act_ready);
+    } else {
+      dpdl_wait();  // count, idx, X_OT and c_x come from the activation pass
+    }
+    const int cnt = __ldcg(a.count);
     const int cs = min(cnt, D_OUT_STAGE);
+    dbar_sync(1, D_EPI);  // the slice of X (fused) is no longer read: xo_s reuses it
     for (int e = et; e < cs * M; e += D_EPI) {
       const int o = e / M, m = e % M;
-      xo_s[o * 64 + m] = a.X_OT[static_cast<size_t>(o) * a.ld_xo + m];
+      xo_s[o * 64 + m] = __ldcg(a.X_OT + static_cast<size_t>(o) * a.ld_xo + m);
     }
-    for (int o = et; o < cs; o += D_EPI) idx_s[o] = a.idx[o];
+    for (int o = et; o < cs; o += D_EPI) idx_s[o] = __ldcg(a.idx + o);
     if (et < M) {
-      const float c = a.c_x[et];
+      const float c = FUSED ? cx_s[et] : __ldcg(a.c_x + et);
       rx_s[et] = c == 0.0f ? 0.0f : __frcp_rn(c);
     }
     dbar_sync(1, D_EPI);
@@ -280,37 +521,10 @@ __global__ void __launch_bounds__(D_THREADS, 1)
       if (et == 0) *s_flag = *abort_flag ? 0 : 1;
       dbar_sync(1, D_EPI);
       if (!*s_flag) continue;
-      tc_fence_after();
-      uint32_t r[HM];
-      const uint32_t t =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * MP + m0);
-      if constexpr (HM >= 16) {
-#pragma unroll
-        for (int j = 0; j < HM / 16; ++j) tmem_ld_32x32b_x16(t + 16 * j, r + 16 * j);
-      } else {
-        tmem_ld_32x32b_x8(t, r);
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
-
-      if (sg.kb0 != 0) {
-        // a later piece of a split n block: add into the global sums and
-        // count the k steps for the block's owner
-        if (n_ok) {
-#pragma unroll
-          for (int j = 0; j < HM; ++j)
-            if (m0 + j < M) atomicAdd(a.part + static_cast<size_t>(m0 + j) * N + n, static_cast<int>(r[j]));
-        }
-        __threadfence();
-        dbar_sync(1, D_EPI);
-        if (et == 0 && !a.skip_arrival) atomicAdd(a.ticket + sg.nb, static_cast<unsigned>(sg.kb1 - sg.kb0));
-        continue;
-      }
-      if (sg.kb1 != num_kb) {
-        // the owner of a split n block: wait for the other pieces' k steps,
-        // then add their sums
+      const bool piece = sg.kb0 != 0;                     // a later piece of a split n block
+      const bool split_owner = !piece && sg.kb1 != num_kb;  // the owner of a split n block
+      if (split_owner) {
+        // wait until the other pieces' k steps are on the block's ticket
         if (et == 0) {
           const unsigned need = static_cast<unsigned>(num_kb - sg.kb1);
           int got = 1;
@@ -329,72 +543,112 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         dbar_sync(1, D_EPI);
         const int got = *s_flag;
         dbar_sync(1, D_EPI);  // s_flag is reused by the next segment
-        if (!got) continue;
-        if (n_ok) {
-          // all loads first: a store between them would serialise the round
-          // trips (the compiler cannot tell the addresses apart)
-          int32_t v[HM];
-#pragma unroll
-          for (int j = 0; j < HM; ++j)
-            v[j] = m0 + j < M ? __ldcg(a.part + static_cast<size_t>(m0 + j) * N + n) : 0;
-#pragma unroll
-          for (int j = 0; j < HM; ++j)
-            if (m0 + j < M) a.part[static_cast<size_t>(m0 + j) * N + n] = 0;
-#pragma unroll
-          for (int j = 0; j < HM; ++j) r[j] = static_cast<uint32_t>(static_cast<int>(r[j]) + v[j]);
+        if (!got) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+          continue;
         }
-        if (et == 0) a.ticket[sg.nb] = 0u;
       }
-      if (!n_ok) continue;
-      // dequantise, add the fp16 outlier product, write fp16 (coalesced over n)
-      const float rw = __ldg(a.inv_cw + n);
-      const float bn = a.bias != nullptr ? __half2float(a.bias[n]) : 0.0f;
-      float y[HM];
+      tc_fence_after();
+      const uint32_t t =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * MP + m0);
+      const float rw = n_ok ? __ldg(a.inv_cw + n) : 0.0f;
+      const float bn = (n_ok && a.bias != nullptr) ? __half2float(a.bias[n]) : 0.0f;
+      // the thread's HM tokens in chunks of HC (fewer live registers)
+#pragma unroll 1
+      for (int c = 0; c < HM / HC; ++c) {
+        const int mc = m0 + c * HC;  // first token of the chunk
+        uint32_t r[HC];
+        if constexpr (HC >= 16) {
 #pragma unroll
-      for (int j = 0; j < HM; ++j)
-        y[j] = m0 + j < M
-                   ? __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), rx_s[m0 + j]), rw), bn)
-                   : 0.0f;
-#pragma unroll
-      for (int o = 0; o < C::WCAP; ++o)
-        if (o < cs) {
-#pragma unroll
-          for (int j = 0; j < HM; ++j)
-            if (m0 + j < M) y[j] = __fmaf_rn(__half2float(xo_s[o * 64 + m0 + j]), wo[o], y[j]);
+          for (int j = 0; j < HC / 16; ++j) tmem_ld_32x32b_x16(t + c * HC + 16 * j, r + 16 * j);
+        } else {
+          tmem_ld_32x32b_x8(t + c * HC, r);
         }
-      // outliers past WCAP: their weight values in batches (eight, four
-      // with 64 tokens, where registers are scarcer), the loads of a batch
-      // all in flight before its FMAs (still in ascending o)
-      constexpr int OB = MP >= 64 ? 4 : 8;
-      for (int o0 = C::WCAP; o0 < cnt; o0 += OB) {
-        float w8[OB];
-#pragma unroll
-        for (int u = 0; u < OB; ++u) {
-          const int o = o0 + u;
-          w8[u] = o < cnt ? __half2float(a.W[static_cast<size_t>(o < cs ? idx_s[o] : __ldg(a.idx + o)) * N + n])
-                          : 0.0f;
+        tmem_wait_ld();
+        if (c == HM / HC - 1) {  // the accumulator buffer is free for the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
         }
+        if (!n_ok) continue;
+        if (piece) {
+          // add into the global sums
 #pragma unroll
-        for (int u = 0; u < OB; ++u) {
-          const int o = o0 + u;
-          if (o < cnt) {
+          for (int j = 0; j < HC; ++j)
+            if (mc + j < M) atomicAdd(a.part + static_cast<size_t>(mc + j) * N + n, static_cast<int>(r[j]));
+          continue;
+        }
+        if (split_owner) {
+          // the other pieces' sums; all loads first: a store between them
+          // would serialise the round trips (the compiler cannot tell the
+          // addresses apart)
+          int32_t v[HC];
 #pragma unroll
-            for (int j = 0; j < HM; ++j)
-              if (m0 + j < M) {
-                const float xo = o < cs ? __half2float(xo_s[o * 64 + m0 + j])
-                                        : __half2float(a.X_OT[static_cast<size_t>(o) * a.ld_xo + m0 + j]);
-                y[j] = __fmaf_rn(xo, w8[u], y[j]);
-              }
+          for (int j = 0; j < HC; ++j)
+            v[j] = mc + j < M ? __ldcg(a.part + static_cast<size_t>(mc + j) * N + n) : 0;
+#pragma unroll
+          for (int j = 0; j < HC; ++j)
+            if (mc + j < M) a.part[static_cast<size_t>(mc + j) * N + n] = 0;
+#pragma unroll
+          for (int j = 0; j < HC; ++j) r[j] = static_cast<uint32_t>(static_cast<int>(r[j]) + v[j]);
+        }
+        // dequantise, add the fp16 outlier product, write fp16 (coalesced over n)
+        float y[HC];
+#pragma unroll
+        for (int j = 0; j < HC; ++j)
+          y[j] = mc + j < M
+                     ? __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), rx_s[mc + j]), rw), bn)
+                     : 0.0f;
+#pragma unroll
+        for (int o = 0; o < C::WCAP; ++o)
+          if (o < cs) {
+#pragma unroll
+            for (int j = 0; j < HC; ++j)
+              if (mc + j < M) y[j] = __fmaf_rn(__half2float(xo_s[o * 64 + mc + j]), wo[o], y[j]);
+          }
+        // outliers past WCAP: their weight values in batches of OB, the
+        // loads of a batch all in flight before its FMAs (still in
+        // ascending o)
+        constexpr int OB = 8;
+        for (int o0 = C::WCAP; o0 < cnt; o0 += OB) {
+          float w8[OB];
+#pragma unroll
+          for (int u = 0; u < OB; ++u) {
+            const int o = o0 + u;
+            w8[u] = o < cnt ? __half2float(a.W[static_cast<size_t>(o < cs ? idx_s[o] : __ldcg(a.idx + o)) * N + n])
+                            : 0.0f;
+          }
+#pragma unroll
+          for (int u = 0; u < OB; ++u) {
+            const int o = o0 + u;
+            if (o < cnt) {
+#pragma unroll
+              for (int j = 0; j < HC; ++j)
+                if (mc + j < M) {
+                  const float xo = o < cs ? __half2float(xo_s[o * 64 + mc + j])
+                                          : __half2float(__ldcg(a.X_OT + static_cast<size_t>(o) * a.ld_xo + mc + j));
+                  y[j] = __fmaf_rn(xo, w8[u], y[j]);
+                }
+            }
           }
         }
+#pragma unroll
+        for (int j = 0; j < HC; ++j)
+          if (mc + j < M) a.Y[static_cast<size_t>(mc + j) * N + n] = __float2half_rn(y[j]);
+        if (a.acc_dump != nullptr) {
+#pragma unroll
+          for (int j = 0; j < HC; ++j)
+            if (mc + j < M) a.acc_dump[static_cast<size_t>(mc + j) * N + n] = static_cast<int32_t>(r[j]);
+        }
       }
-#pragma unroll
-      for (int j = 0; j < HM; ++j)
-        if (m0 + j < M) a.Y[static_cast<size_t>(m0 + j) * N + n] = __float2half_rn(y[j]);
-      if (a.acc_dump != nullptr) {
-#pragma unroll
-        for (int j = 0; j < HM; ++j)
-          if (m0 + j < M) a.acc_dump[static_cast<size_t>(m0 + j) * N + n] = static_cast<int32_t>(r[j]);
+      if (piece) {
+        // count the k steps for the block's owner
+        __threadfence();
+        dbar_sync(1, D_EPI);
+        if (et == 0 && !a.skip_arrival) atomicAdd(a.ticket + sg.nb, static_cast<unsigned>(sg.kb1 - sg.kb0));
+      } else if (split_owner && et == 0) {
+        a.ticket[sg.nb] = 0u;
       }
     }
   }
@@ -407,7 +661,7 @@ __global__ void __launch_bounds__(D_THREADS, 1)
   }
 }
 
-template <int MP>
+template <int MP, bool FUSED>
 cudaError_t launch_decode_t(const CUtensorMap& tmW, const CUtensorMap& tmX, const DecodeArgs& a, int num_sms,
                             bool pdl, cudaStream_t stream) {
   using C = DCfg<MP>;
@@ -416,37 +670,57 @@ cudaError_t launch_decode_t(const CUtensorMap& tmW, const CUtensorMap& tmX, cons
   cudaGetDevice(&dev);
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_i8_decode_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(gemm_i8_decode_kernel<MP, FUSED>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set |= bit;
   }
-  const long long total = static_cast<long long>((a.N + DBM - 1) / DBM) * ((a.K + DBK - 1) / DBK);
-  const int grid = static_cast<int>(std::max(1LL, std::min<long long>(total, num_sms)));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  cfg.gridDim = dim3(static_cast<unsigned>(decode_grid(a.N, a.K, num_sms)));
   cfg.blockDim = dim3(D_THREADS);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr.val.programmaticStreamSerializationAllowed = 1;
+  if (FUSED) {
+    attr.id = cudaLaunchAttributeCooperative;  // all CTAs resident at once (grid barriers)
+    attr.val.cooperative = 1;
+  } else {
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+  }
   cfg.attrs = &attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemm_i8_decode_kernel<MP>, tmW, tmX, a);
+  cfg.numAttrs = (FUSED || pdl) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemm_i8_decode_kernel<MP, FUSED>, tmW, tmX, a);
+}
+
+template <bool FUSED>
+cudaError_t launch_decode_f(const CUtensorMap& tmW, const CUtensorMap& tmX, const DecodeArgs& a, int num_sms,
+                            bool pdl, cudaStream_t stream) {
+  switch (decode_padded_tokens(a.M)) {
+    case 16: return launch_decode_t<16, FUSED>(tmW, tmX, a, num_sms, pdl, stream);
+    case 32: return launch_decode_t<32, FUSED>(tmW, tmX, a, num_sms, pdl, stream);
+    default: return launch_decode_t<64, FUSED>(tmW, tmX, a, num_sms, pdl, stream);
+  }
 }
 
 }  // namespace
 
 int decode_padded_tokens(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
+bool decode_fused_fits(int64_t M, int64_t K, int64_t N, int num_sms) {
+  if (M < 1 || M > kDecodeMaxM || K < 16 || K % 16 != 0 || N < 1 || num_sms < 1) return false;
+  const int64_t nvec = K / 8;
+  const int64_t G = decode_grid(N, K, num_sms);
+  return nvec <= 16 * G;  // every CTA's slice has at most ceil(nvec / G) <= 16 vectors
+}
+
 cudaError_t launch_gemm_decode(const CUtensorMap& tmW, const CUtensorMap& tmX, const DecodeArgs& a, int num_sms,
                                bool pdl, cudaStream_t stream) {
-  switch (decode_padded_tokens(a.M)) {
-    case 16: return launch_decode_t<16>(tmW, tmX, a, num_sms, pdl, stream);
-    case 32: return launch_decode_t<32>(tmW, tmX, a, num_sms, pdl, stream);
-    default: return launch_decode_t<64>(tmW, tmX, a, num_sms, pdl, stream);
+  if (a.X != nullptr) {
+    if (!decode_fused_fits(a.M, a.K, a.N, num_sms)) return cudaErrorInvalidValue;
+    return launch_decode_f<true>(tmW, tmX, a, num_sms, false, stream);
   }
+  return launch_decode_f<false>(tmW, tmX, a, num_sms, pdl, stream);
 }
 
 }  // namespace i8mm

@@ -168,12 +168,36 @@ struct DecodeArgs {
   unsigned long long timeout_ns;
   int skip_arrival;        // failure-detection test only: split pieces do not count their
                            // k steps on the owner's ticket, so its wait runs out
+  // The activation pass inside the same launch (X != nullptr): the kernel
+  // computes O, c_x, Xq, X_OT, idx and count itself and writes them to the
+  // buffers below, which c_x, X_OT, idx and count above must name as well.
+  const __half* X;         // [M, K] fp16 activations, or nullptr (a separate activation pass ran)
+  int thr;                 // half_magnitude_threshold(alpha)
+  int8_t* Xq_out;          // [M, K] codes, read back through tmX
+  float* c_x_out;          // [M]
+  __half* X_OT_out;        // [|O|][ld_xo]
+  int32_t* idx_out;        // [K]
+  int32_t* count_out;      // [1]
+  uint32_t* omask;         // [2][ceil(K/32)] bitmasks by generation parity (as RowActArgs::omask)
+  uint32_t* sync;          // [3] arrivals by generation parity, generation (as RowActArgs::sync)
+  uint32_t* rowmax;        // [kDecodeMaxM][kRowMaxStride] row absmax bits (first word of
+                           // each row), zero between launches
+  int skip_barrier;        // failure-detection test only: CTA 0 does not arrive at the first
+                           // grid barrier, so every CTA's wait there runs out
 };
+// Words between the rows of DecodeArgs::rowmax: one 128-byte line per row,
+// so that the CTAs' atomics on different rows do not queue on one line.
+constexpr int kRowMaxStride = 32;
 // Tokens padded to the MMA N of the decode kernel: 16, 32 or 64.
 int decode_padded_tokens(int64_t M);
+// Whether the decode kernel can run the activation pass itself for M x K
+// against N columns: every CTA's slice of X must hold at most 16 vectors of
+// 8 columns per row (K <= 16384 on 128 or more SMs).
+bool decode_fused_fits(int64_t M, int64_t K, int64_t N, int num_sms);
 // tmW maps the K-blocked weight (rows of 128 bytes) with 128-row boxes; tmX
-// maps Xq [M,K] with 128 x decode_padded_tokens(M) boxes.  With `pdl`, the first weight tiles
-// stream while the activation pass finishes.
+// maps Xq [M,K] with 128 x decode_padded_tokens(M) boxes.  With a.X set, a
+// cooperative launch that runs the activation pass too; otherwise, with
+// `pdl`, the first weight tiles stream while the activation pass finishes.
 cudaError_t launch_gemm_decode(const CUtensorMap& tmW, const CUtensorMap& tmX, const DecodeArgs& a,
                                int num_sms, bool pdl, cudaStream_t stream);
 

@@ -77,6 +77,12 @@ __device__ __forceinline__ void red_release_add_gpu(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Orders this thread's generic-proxy global accesses with later (or, after
+// an acquire, other threads' earlier) async-proxy ones such as TMA loads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Prefetch `bytes` (a multiple of 16) of global memory from 16-byte-aligned
 // `p` into L2.
 __device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
@@ -98,6 +104,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
+}
+
+// Prefetch the box of a 2-D tiled tensor map at (c0, c1) into L2 (no shared
+// memory, no completion); the innermost coordinate obeys the 16-byte rule as
+// for the loads.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
 }
 
 // L2 policy for data read once (a weight streamed by the decode GEMM).

@@ -468,11 +468,14 @@ def test_launches_per_forward():
     W = torch.from_numpy(workloads.weight(5120, 256, 43)).to(dev())
     w = m.int8mm_prepare_weight(W)
     assert m.int8mm_launches_per_forward(w, 0) == 0
-    assert m.int8mm_launches_per_forward(w, 1) == 2       # single-launch activation pass + decode GEMM
+    assert m.int8mm_launches_per_forward(w, 1) == 1       # decode GEMM with its own activation pass
+    assert m.int8mm_launches_per_forward(w, 64) == 1
+    assert m.int8mm_launches_per_forward(w, 65) == 2      # activation pass + CTA-pair GEMM
     assert m.int8mm_launches_per_forward(w, 2048) == 2    # activation pass + CTA-pair GEMM
     assert m.int8mm_launches_per_forward(w, 4096) == 2    # more rows per block than row slots
     w2 = m.int8mm_prepare_weight(torch.from_numpy(workloads.weight(40960, 256, 44)).to(dev()))
     assert m.int8mm_launches_per_forward(w2, 2048) == 2   # 80 KB rows, one slot per block
+    assert m.int8mm_launches_per_forward(w2, 8) == 2      # K > 16384: decode GEMM after the activation pass
     assert m.int8mm_launches_per_forward(w, 40000) == 3   # > 256 rows per SM: two activation kernels
     with pytest.raises(m.Int8mmError):
         m.int8mm_launches_per_forward(w, -1)
@@ -492,6 +495,69 @@ def test_single_launch_pass_many_generations():
         torch.cuda.synchronize()
         assert int(d["outlier_count"].item()) == i % 4
         assert torch.equal(y, d["Y"])
+    assert m.int8mm_get_status(w) == m.INT8MM_OK
+
+
+FUSED_SHAPES = [
+    # M, K, N, planted outliers, alpha: decode shapes (M <= 64, K <= 16384)
+    (1, 4096, 1024, 3, 6.0),
+    (16, 8192, 2048, 7, 6.0),
+    (33, 12288, 1040, 7, 6.0),       # ragged 128-column block
+    (64, 16384, 512, 5, 6.0),        # largest K of the fused pass: 16-vector slices
+    (40, 2048, 4112, 0, 6.0),        # no outliers, stream-K splits across blocks
+    (8, 512, 256, 6, 0.0),           # alpha = 0: every non-zero column is an outlier
+    (5, 384, 128, 2, -1.0),          # alpha < 0: every column is an outlier
+    (9, 1040, 784, 4, math.inf),     # pure vector-wise
+    (2, 16, 16, 1, 6.0),             # one CTA, a 2-vector slice
+]
+
+
+@pytest.mark.parametrize("M,K,N,n_out,alpha", FUSED_SHAPES)
+def test_decode_activation_pass_in_the_gemm_launch_equals_the_separate_pass(M, K, N, n_out, alpha):
+    # forward runs the activation pass inside the decode GEMM's launch;
+    # forward_events (which times the passes apart) runs it as its own kernel
+    p = workloads.small(M, K, N, n_out, seed=M * 7 + K + N)
+    p.alpha = alpha
+    out = check(p)
+    w = out["w"]
+    X = torch.from_numpy(p.X).to(dev())
+    assert m.int8mm_launches_per_forward(w, M) == 1
+    y1 = m.int8mm_forward(w, X, alpha)
+    y2 = torch.empty_like(y1)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    m.int8mm_forward_events(w, X, alpha, y2, ev)
+    torch.cuda.synchronize()
+    assert m.int8mm_get_status(w) == m.INT8MM_OK
+    assert torch.equal(y1, y2)
+    assert torch.equal(y1, out["d"]["Y"])
+
+
+def test_decode_and_prefill_forwards_share_the_barrier_state():
+    # the decode GEMM's own activation pass and the separate single-launch
+    # pass keep one generation word, bitmask pair and arrival counters:
+    # alternate them (and the two-kernel decode path) on one handle
+    K, N = 2048, 1168
+    W = workloads.weight(K, N, 91)
+    w = m.int8mm_prepare_weight(torch.from_numpy(W).to(dev()))
+    wq = oracle.quantize_cols(W)
+    runs = [(40, 5), (300, 2), (8, 0), (8, 3), (2048, 7), (1, 1), (64, 4), (200, 0), (16, 6), (16, 6)]
+    counts = []
+    for i, (M, n_out) in enumerate(runs):
+        p = workloads.small(M, K, N, n_out, seed=700 + i)
+        p.W = W
+        out = check(p, w=w, wq=wq, rows=sample_rows(M, 16, seed=i), check_w_codes=False)
+        counts.append(out["cnt"])
+        X = torch.from_numpy(p.X).to(dev())
+        y = m.int8mm_forward(w, X, p.alpha)
+        if i % 3 == 0:  # the separate pass in between
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            y2 = torch.empty_like(y)
+            m.int8mm_forward_events(w, X, p.alpha, y2, ev)
+            torch.cuda.synchronize()
+            assert torch.equal(y, y2)
+        torch.cuda.synchronize()
+        assert torch.equal(y, out["d"]["Y"])
+    assert counts == [n for _, n in runs]
     assert m.int8mm_get_status(w) == m.INT8MM_OK
 
 

@@ -41,6 +41,7 @@ FORWARD_WAITS = [
     ("splitk_ticket", 300, 1040, 784, 5, 2),   # prefill GEMM: a tile owner's ticket
     ("decode_ticket", 40, 2048, 4112, 5, 0),   # decode GEMM: a split n block's ticket
     ("barrier_arrival", 300, 1040, 784, 5, 0),  # single-launch activation pass: grid barrier
+    ("barrier_arrival", 40, 2048, 4112, 5, 0),  # decode GEMM's own activation pass: first grid barrier
 ]
 
 
