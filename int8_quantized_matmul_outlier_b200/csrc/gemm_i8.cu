@@ -156,23 +156,6 @@ __device__ __forceinline__ void load_bias32(const __half* bias, int n, bool full
   }
 }
 
-// 8 x 8 transpose of 16-bit values: v[r] holds row r (8 values, two per
-// word); on return t[c] holds column c, i.e. element r of row c is value c of
-// v[r].
-__device__ __forceinline__ void transpose8x8_b16(const uint4 (&v)[8], uint4 (&t)[8]) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint32_t sel = (c & 1) ? 0x7632u : 0x5410u;  // high or low halves of the two words
-    uint32_t w[4];
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const uint32_t a = (&v[2 * p].x)[c >> 1], b = (&v[2 * p + 1].x)[c >> 1];
-      w[p] = __byte_perm(a, b, sel);
-    }
-    t[c] = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
-
 // One work unit: k-blocks [kb0, kb1) of a tile cut into S pieces; piece S-1
 // finishes the tile.  With split K the last `tail` tiles are the split ones
 // (ti: a split tile's index among them); the others are whole units.

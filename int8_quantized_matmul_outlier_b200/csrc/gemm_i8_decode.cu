@@ -44,12 +44,21 @@
 // same rule: the launch of generation g uses the parity-g buffers, finds
 // them zero, and clears the parity-(g+1) ones for the next launch.
 //
+// Outlier product on the tensor cores: for every segment that writes Y, the
+// epilogue warps stage W[O, n block] and X[:, O] as fp16 K-major operands, a
+// chunk of kOutMma outliers at a time (transposed in registers from
+// coalesced 16-byte loads), while the int8 part runs; after it, the MMA warp
+// adds D_O^T[n, m] = sum_{o} W[O_o, n] X[m, O_o] into a third, fp32 TMEM
+// accumulator (kind::f16, 128 x MP x 16 per instruction), which the
+// epilogue adds to the dequantised int8 part.
+//
 // Warps: 0 TMA producer (weight tile + token tile per stage, 6-deep ring,
 // weight loads marked evict-first in L2; the first ring of weight tiles is
 // loaded, and the next D_PF_TILES prefetched into L2, before waiting on the
 // activation pass), 1 MMA issuer and TMEM owner (double-buffered 128 x MP int32
-// accumulator), 2-9 epilogue (one output column n per thread, half of the
-// tokens: two warps share each TMEM lane quarter).
+// accumulator, 128 x MP fp32 outlier product), 2-9 epilogue (one output
+// column n per thread, half of the tokens: two warps share each TMEM lane
+// quarter) and outlier staging.
 // Every wait is bounded; a timeout sets the status word and the CTA exits.
 #include "actq.cuh"
 #include "kernels.cuh"
@@ -68,7 +77,7 @@ constexpr int D_STAGES = 6;
 // Weight tiles past the ring that the producer prefetches into L2 before it
 // waits for the activation pass (at most this many per CTA, 16 KB each).
 constexpr int D_PF_TILES = 24;
-constexpr int D_OUT_STAGE = 128;  // outliers whose activations (and indices) are staged in smem
+constexpr int D_OUT_STAGE = 128;  // outliers whose indices are staged in smem
 constexpr int D_EPI = 256;  // epilogue threads: eight warps
 constexpr int D_THREADS = 64 + D_EPI;
 
@@ -78,23 +87,29 @@ struct DCfg {
   static constexpr int X_BYTES = MP * DBK;
   static constexpr int STAGE = W_BYTES + X_BYTES;
   static constexpr int STAGES = D_STAGES;
-  static constexpr int BAR_OFF = STAGES * STAGE;
-  static constexpr int NBARS = 2 * STAGES + 6;
+  // operands of the outlier product, one chunk of kOutMma outliers, fp16,
+  // K-major rows of 128 bytes with the 128-byte swizzle: A = W[O, n block]
+  // (128 columns n), B = X[:, O] (MP tokens)
+  static constexpr int OA_OFF = STAGES * STAGE;
+  static constexpr int OB_OFF = OA_OFF + DBM * 128;
+  static constexpr int BAR_OFF = OB_OFF + MP * 128;
+  static constexpr int NBARS = 2 * STAGES + 8;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-  // half [D_OUT_STAGE][64]; before the outliers are staged, the fused
-  // activation pass's slice of X, uint4 [64 rows][16 vectors] (16 KB too)
+  // the fused activation pass's slice of X, uint4 [64 rows][16 vectors]
   static constexpr int XO_OFF = (MISC_OFF + 32 + 15) & ~15;
-  static constexpr int RX_OFF = XO_OFF + D_OUT_STAGE * 64 * 2;     // float [64]
+  static constexpr int RX_OFF = XO_OFF + 64 * 16 * 16;             // float [64]
   static constexpr int IDX_OFF = RX_OFF + 64 * 4;                  // int [D_OUT_STAGE]
   static constexpr int CX_OFF = IDX_OFF + D_OUT_STAGE * 4;         // float [64]: c_x (fused)
   static constexpr int FL_OFF = CX_OFF + 64 * 4;                   // u32 [16]: flags per vector (fused)
   static constexpr int OL_OFF = FL_OFF + 16 * 4;                   // u32 [128]: the slice's outliers (fused)
   static constexpr int RED_OFF = OL_OFF + 128 * 4;                 // u32 [16]: reductions (fused)
   static constexpr int SMEM = RED_OFF + 16 * 4 + 1024;
-  // outlier weight values prefetched into registers per segment
-  static constexpr int WCAP = 16;
-  static constexpr int TMEM_COLS = 2 * MP < 32 ? 32 : 2 * MP;
+  // TMEM: two int32 accumulators (double buffer) and the fp32 outlier
+  // product, MP columns each, in a power-of-two allocation
+  static constexpr int TMEM_COLS = 3 * MP <= 32 ? 32 : (3 * MP <= 64 ? 64 : (3 * MP <= 128 ? 128 : 256));
   static constexpr uint32_t IDESC = idesc_i8(DBM, MP);
+  static constexpr uint32_t IDESC_F16 = idesc_f16_f32(DBM, MP);
+  static_assert(OA_OFF % 1024 == 0 && OB_OFF % 1024 == 0, "outlier operands 1024-byte aligned");
   static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned for the 128B swizzle");
   static_assert(SMEM <= 232448, "fits the 227 KB of shared memory per block");
 };
@@ -158,10 +173,11 @@ __global__ void __launch_bounds__(D_THREADS, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* act_ready = drain + 1;  // fused: the token tiles of Xq may be loaded
+  uint64_t* ofull = act_ready + 1;   // an outlier chunk is staged (one arrival per epilogue warp)
+  uint64_t* oempty = ofull + 1;      // the tensor cores are done with the staged chunk
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
   volatile int* s_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 8);
-  __half* xo_s = reinterpret_cast<__half*>(smem + C::XO_OFF);
   float* rx_s = reinterpret_cast<float*>(smem + C::RX_OFF);
   int* idx_s = reinterpret_cast<int*>(smem + C::IDX_OFF);
   float* cx_s = reinterpret_cast<float*>(smem + C::CX_OFF);
@@ -185,6 +201,8 @@ __global__ void __launch_bounds__(D_THREADS, 1)
     }
     mbar_init(drain, 1);
     mbar_init(act_ready, 1);
+    mbar_init(ofull, D_EPI / 32);
+    mbar_init(oempty, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmW);
@@ -288,6 +306,9 @@ __global__ void __launch_bounds__(D_THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       int lt = 0;
+      int cnt = -1;             // |O|, read at the first segment that writes Y
+      uint32_t orounds = 0;     // outlier chunks issued so far
+      const uint32_t d2_tmem = tmem_base + static_cast<uint32_t>(2 * MP);
       for (long long u = u_begin; u < u_end && ok; ++lt) {
         const Seg sg = segment_at(u, u_end, num_kb);
         u += sg.kb1 - sg.kb0;
@@ -316,6 +337,33 @@ __global__ void __launch_bounds__(D_THREADS, 1)
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
+          }
+        }
+        if (ok && sg.kb0 == 0) {
+          // this segment writes Y: the fp16 outlier product into its own
+          // accumulator, one staged chunk of kOutMma outliers at a time
+          if (cnt < 0) {
+            if constexpr (FUSED) {
+              if (!mbar_wait(act_ready, 0, 3 * tmo, abort_flag)) ok = false;
+            } else {
+              dpdl_wait();
+            }
+            cnt = ok ? __ldcg(a.count) : 0;
+          }
+          const uint64_t oad = smem_desc_k_sw128(smem_u32(smem + C::OA_OFF));
+          const uint64_t obd = smem_desc_k_sw128(smem_u32(smem + C::OB_OFF));
+          for (int o0 = 0; o0 < cnt && ok; o0 += kOutMma) {
+            if (!mbar_wait(ofull, orounds & 1u, tmo, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const int ks = (min(cnt - o0, kOutMma) + 15) / 16;
+            for (int kk = 0; kk < ks; ++kk)
+              mma_f16(d2_tmem, oad + static_cast<uint64_t>(kk * 2), obd + static_cast<uint64_t>(kk * 2),
+                      C::IDESC_F16, (o0 > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(oempty);
+            ++orounds;
           }
         }
         if (ok) mma_commit(&tfull[buf]);
@@ -489,17 +537,63 @@ __global__ void __launch_bounds__(D_THREADS, 1)
     }
     const int cnt = __ldcg(a.count);
     const int cs = min(cnt, D_OUT_STAGE);
-    dbar_sync(1, D_EPI);  // the slice of X (fused) is no longer read: xo_s reuses it
-    for (int e = et; e < cs * M; e += D_EPI) {
-      const int o = e / M, m = e % M;
-      xo_s[o * 64 + m] = __ldcg(a.X_OT + static_cast<size_t>(o) * a.ld_xo + m);
-    }
     for (int o = et; o < cs; o += D_EPI) idx_s[o] = __ldcg(a.idx + o);
     if (et < M) {
       const float c = FUSED ? cx_s[et] : __ldcg(a.c_x + et);
       rx_s[et] = c == 0.0f ? 0.0f : __frcp_rn(c);
     }
     dbar_sync(1, D_EPI);
+    // Stages outliers [o0, o0 + kOutMma) of the product's operands for n
+    // block nb: A = W[O, n block] (128 rows n), B = X_OT^T (MP rows m).
+    // Thread et takes the 8 x 8 block of rows 8 (b >> 3) .. +7 and outliers
+    // 8 (b & 7) .. +7 (b = et: A, b = et - 128: B): eight 16-byte loads along
+    // the rows, transposed in registers into eight 16-byte pieces of the
+    // K-major 128-byte-swizzled layout (piece j of row r at j ^ (r % 8),
+    // groups of 8 rows 1024 bytes apart).  Only the 16-outlier steps the
+    // product reads are written; zero past |O| and past M or N.
+    auto stage_outliers = [&](int o0, int nb) {
+      const int no = min(cnt - o0, kOutMma);
+      const int n_og = 2 * ((no + 15) / 16);
+      const bool isA = et < DBM;
+      const int b = isA ? et : et - DBM;
+      if (b >= (isA ? DBM : MP)) return;
+      const int og = b & 7, rg = b >> 3;
+      if (og >= n_og) return;
+      const int r0 = isA ? nb * DBM + 8 * rg : 8 * rg;  // first column n (A) or token m (B)
+      const int lim = isA ? N : M;
+      uint4 v[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int o = o0 + 8 * og + r;
+        v[r] = make_uint4(0u, 0u, 0u, 0u);
+        if (o < cnt && r0 < lim) {
+          if (isA) {
+            const int row = o < cs ? idx_s[o] : __ldcg(a.idx + o);
+            v[r] = __ldg(reinterpret_cast<const uint4*>(a.W + static_cast<size_t>(row) * N + r0));
+          } else {
+            v[r] = __ldcg(reinterpret_cast<const uint4*>(a.X_OT + static_cast<size_t>(o) * a.ld_xo + r0));
+          }
+        }
+      }
+      if (r0 + 8 > lim) {  // columns past N or tokens past M: zero
+        const int keep = max(0, lim - r0);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          uint32_t* wv = &v[r].x;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (2 * e >= keep) wv[e] = 0u;
+            else if (2 * e + 1 >= keep) wv[e] &= 0xffffu;
+          }
+        }
+      }
+      uint4 tv[8];
+      transpose8x8_b16(v, tv);
+      uint8_t* blk = smem + (isA ? C::OA_OFF : C::OB_OFF) + rg * 1024;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4*>(blk + i * 128 + ((og ^ i) << 4)) = tv[i];
+    };
+    uint32_t orounds = 0;  // outlier chunks staged so far
     int lt = 0;
     for (long long u = u_begin; u < u_end; ++lt) {
       const Seg sg = segment_at(u, u_end, num_kb);
@@ -508,12 +602,27 @@ __global__ void __launch_bounds__(D_THREADS, 1)
       const uint32_t use = static_cast<uint32_t>(lt >> 1);
       const int n = sg.nb * DBM + n_local;
       const bool n_ok = n < N;
-      // outlier weight values of this column: they do not depend on the
-      // accumulator, so load them while the tensor cores still work
-      float wo[C::WCAP];
-#pragma unroll
-      for (int o = 0; o < C::WCAP; ++o)
-        wo[o] = (o < cs && n_ok) ? __half2float(a.W[static_cast<size_t>(idx_s[o]) * N + n]) : 0.0f;
+      const bool writer = sg.kb0 == 0;  // this segment writes Y
+      // the outlier product's operands, while the tensor cores work on the
+      // int8 part: chunk by chunk, each once the previous one is consumed
+      // (the previous segment's product was read from TMEM before this)
+      if (writer && cnt > 0) {
+        for (int o0 = 0; o0 < cnt; o0 += kOutMma) {
+          if (orounds > 0) {
+            const bool okw = __all_sync(0xffffffffu, mbar_wait(oempty, (orounds - 1) & 1u, tmo, abort_flag));
+            if (!okw) {
+              if (lane == 0) dfail(a, abort_flag);
+              break;
+            }
+          }
+          stage_outliers(o0, sg.nb);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(ofull);
+          ++orounds;
+        }
+      }
       // all lanes wait; the decision to go on is then made once for all warps
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], use & 1u, tmo, abort_flag));
       if (!ok && lane == 0) dfail(a, abort_flag);
@@ -552,18 +661,29 @@ __global__ void __launch_bounds__(D_THREADS, 1)
       tc_fence_after();
       const uint32_t t =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * MP + m0);
+      // the outlier product's accumulator (single-buffered, after the two int32 ones)
+      const uint32_t t2 = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(2 * MP + m0);
       const float rw = n_ok ? __ldg(a.inv_cw + n) : 0.0f;
+      const bool with_o = writer && cnt > 0;  // the segment has an outlier product
       const float bn = (n_ok && a.bias != nullptr) ? __half2float(a.bias[n]) : 0.0f;
       // the thread's HM tokens in chunks of HC (fewer live registers)
 #pragma unroll 1
       for (int c = 0; c < HM / HC; ++c) {
         const int mc = m0 + c * HC;  // first token of the chunk
-        uint32_t r[HC];
+        uint32_t r[HC], d2[HC];
         if constexpr (HC >= 16) {
 #pragma unroll
           for (int j = 0; j < HC / 16; ++j) tmem_ld_32x32b_x16(t + c * HC + 16 * j, r + 16 * j);
         } else {
           tmem_ld_32x32b_x8(t + c * HC, r);
+        }
+        if (with_o) {  // warp-uniform, like every tcgen05.ld
+          if constexpr (HC >= 16) {
+#pragma unroll
+            for (int j = 0; j < HC / 16; ++j) tmem_ld_32x32b_x16(t2 + c * HC + 16 * j, d2 + 16 * j);
+          } else {
+            tmem_ld_32x32b_x8(t2 + c * HC, d2);
+          }
         }
         tmem_wait_ld();
         if (c == HM / HC - 1) {  // the accumulator buffer is free for the MMA warp
@@ -593,45 +713,17 @@ __global__ void __launch_bounds__(D_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < HC; ++j) r[j] = static_cast<uint32_t>(static_cast<int>(r[j]) + v[j]);
         }
-        // dequantise, add the fp16 outlier product, write fp16 (coalesced over n)
+        // dequantise, add the layer bias and the fp16 outlier product (fp32
+        // from TMEM), write fp16 (coalesced over n)
         float y[HC];
 #pragma unroll
         for (int j = 0; j < HC; ++j)
           y[j] = mc + j < M
                      ? __fadd_rn(__fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[j])), rx_s[mc + j]), rw), bn)
                      : 0.0f;
+        if (with_o) {
 #pragma unroll
-        for (int o = 0; o < C::WCAP; ++o)
-          if (o < cs) {
-#pragma unroll
-            for (int j = 0; j < HC; ++j)
-              if (mc + j < M) y[j] = __fmaf_rn(__half2float(xo_s[o * 64 + mc + j]), wo[o], y[j]);
-          }
-        // outliers past WCAP: their weight values in batches of OB, the
-        // loads of a batch all in flight before its FMAs (still in
-        // ascending o)
-        constexpr int OB = 8;
-        for (int o0 = C::WCAP; o0 < cnt; o0 += OB) {
-          float w8[OB];
-#pragma unroll
-          for (int u = 0; u < OB; ++u) {
-            const int o = o0 + u;
-            w8[u] = o < cnt ? __half2float(a.W[static_cast<size_t>(o < cs ? idx_s[o] : __ldcg(a.idx + o)) * N + n])
-                            : 0.0f;
-          }
-#pragma unroll
-          for (int u = 0; u < OB; ++u) {
-            const int o = o0 + u;
-            if (o < cnt) {
-#pragma unroll
-              for (int j = 0; j < HC; ++j)
-                if (mc + j < M) {
-                  const float xo = o < cs ? __half2float(xo_s[o * 64 + mc + j])
-                                          : __half2float(__ldcg(a.X_OT + static_cast<size_t>(o) * a.ld_xo + mc + j));
-                  y[j] = __fmaf_rn(xo, w8[u], y[j]);
-                }
-            }
-          }
+          for (int j = 0; j < HC; ++j) y[j] = __fadd_rn(y[j], __uint_as_float(d2[j]));
         }
 #pragma unroll
         for (int j = 0; j < HC; ++j)

@@ -176,6 +176,35 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, fp16 x fp16 -> fp32 (kind::f16, K = 16
+// per instruction), one CTA.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 8 x 8 transpose of 16-bit values: v[r] holds row r (8 values, two per
+// word); on return t[c] holds column c, i.e. element r of row c is value c of
+// v[r].
+__device__ __forceinline__ void transpose8x8_b16(const uint4 (&v)[8], uint4 (&t)[8]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t sel = (c & 1) ? 0x7632u : 0x5410u;  // high or low halves of the two words
+    uint32_t w[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const uint32_t a = (&v[2 * p].x)[c >> 1], b = (&v[2 * p + 1].x)[c >> 1];
+      w[p] = __byte_perm(a, b, sel);
+    }
+    t[c] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
