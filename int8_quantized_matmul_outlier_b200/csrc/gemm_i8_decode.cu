@@ -37,9 +37,10 @@
 //      outlier columns: idx and X_OT for them;
 //   4. meet at a second grid barrier, after which the producer loads the
 //      token tiles of Xq with TMA.
-// Meanwhile the producer has issued the first ring of weight tiles and
-// prefetched the next ones into L2, so the weight streams from the first
-// instruction on.  The barrier state (bitmasks, arrival counters and the
+// Meanwhile the producer has issued the first ring of weight tiles.
+// Prefetching the next ones into L2 as well (24 tiles per CTA) measured
+// slower: it delayed the first grid barrier by about 2 us (the release of
+// the arrival waits for the CTA's outstanding memory operations).  The barrier state (bitmasks, arrival counters and the
 // generation word) is the one the separate activation pass keeps, with the
 // same rule: the launch of generation g uses the parity-g buffers, finds
 // them zero, and clears the parity-(g+1) ones for the next launch.
@@ -54,8 +55,7 @@
 //
 // Warps: 0 TMA producer (weight tile + token tile per stage, 6-deep ring,
 // weight loads marked evict-first in L2; the first ring of weight tiles is
-// loaded, and the next D_PF_TILES prefetched into L2, before waiting on the
-// activation pass), 1 MMA issuer and TMEM owner (double-buffered 128 x MP int32
+// loaded before waiting on the activation pass), 1 MMA issuer and TMEM owner (double-buffered 128 x MP int32
 // accumulator, 128 x MP fp32 outlier product), 2-9 epilogue (one output
 // column n per thread, half of the tokens: two warps share each TMEM lane
 // quarter) and outlier staging.
@@ -74,9 +74,6 @@ constexpr int DBK = 128;  // K bytes per stage
 // Six stages of weight tiles in flight per SM measured faster than deeper
 // rings (4: slower, 11: 12% slower): more outstanding reads only congest HBM.
 constexpr int D_STAGES = 6;
-// Weight tiles past the ring that the producer prefetches into L2 before it
-// waits for the activation pass (at most this many per CTA, 16 KB each).
-constexpr int D_PF_TILES = 24;
 constexpr int D_OUT_STAGE = 128;  // outliers whose indices are staged in smem
 constexpr int D_EPI = 256;  // epilogue threads: eight warps
 constexpr int D_THREADS = 64 + D_EPI;
@@ -251,13 +248,6 @@ __global__ void __launch_bounds__(D_THREADS, 1)
         const int nb = static_cast<int>(uu / num_kb), kb = static_cast<int>(uu % num_kb);
         mbar_arrive_expect_tx(&full[i], C::STAGE);
         tma_load_2d_hint(smem + i * C::STAGE, &tmW, &full[i], 0, kb * a.N_pad + nb * DBM, wpol);
-      }
-      // and the next tiles of the range into L2, so that the weight streams
-      // from HBM while the activation pass runs
-      const long long pf_end = min(u_end, u_begin + pre + D_PF_TILES);
-      for (long long uu = u_begin + pre; uu < pf_end; ++uu) {
-        const int nb = static_cast<int>(uu / num_kb), kb = static_cast<int>(uu % num_kb);
-        tma_prefetch_2d(&tmW, 0, kb * a.N_pad + nb * DBM);
       }
       if constexpr (FUSED) {
         // Xq is written by the CTAs' activation pass; the epilogue warps

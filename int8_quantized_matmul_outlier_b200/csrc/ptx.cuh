@@ -106,15 +106,6 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-// Prefetch the box of a 2-D tiled tensor map at (c0, c1) into L2 (no shared
-// memory, no completion); the innermost coordinate obeys the 16-byte rule as
-// for the loads.
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int32_t c0, int32_t c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1)
-               : "memory");
-}
-
 // L2 policy for data read once (a weight streamed by the decode GEMM).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t pol;
