@@ -129,7 +129,7 @@ int8mm_status int8mm_reserve(int8mm_weight_t h, int64_t M_max, void* stream);
  * alpha: outlier threshold (6.0 in the pages); INFINITY disables the fp16
  *   path (pure vector-wise int8); any value below every |x| makes every
  *   column an outlier.  NaN is an argument error.
- * M == 0 is a no-op.  Decode shapes (M <= 64, K <= 16384) run as ONE
+ * M == 0 is a no-op.  Decode shapes (M <= 128, K <= 16384) run as ONE
  * kernel on `stream`: the decode GEMM (a cooperative launch) does the
  * activation pass itself, each CTA on a slice of X's columns, with two grid
  * barriers, while its first weight tiles already stream.  Otherwise two or
@@ -264,7 +264,7 @@ int8mm_status int8mm_set_wait_limit(int8mm_weight_t h, uint64_t timeout_ns);
 int8mm_status int8mm_set_test_skip(int8mm_weight_t h, int bits);
 
 /*
- * Split of the prefill GEMM along K (forwards with M > 64, whose 256 x 256
+ * Split of the prefill GEMM along K (forwards with M > 128, whose 256 x 256
  * output tiles are computed by pairs of SMs).  0 (the default) lets the
  * library choose the plan that best fills the pairs' rounds of work: no
  * split; every tile cut into S in 2..4 pieces; or, when the tiles leave a

@@ -38,7 +38,7 @@ struct int8mm_weight {
   float* inv_cw = nullptr;    // [N]
   uint32_t* colmax_bits = nullptr;  // [N] prep scratch
   CUtensorMap tmW128;  // Wb, 128-row boxes (operand B of the prefill GEMM, A of the decode GEMM)
-  // decode (M <= 64) scratch: int32 partial sums and per-n-block tickets
+  // decode (M <= kDecodeMaxM) scratch: int32 partial sums and per-n-block tickets
   int32_t* part = nullptr;
   unsigned* dticket = nullptr;
   // prefill split-K scratch: partial tiles and per-(tile, CTA, half) tickets

@@ -1,4 +1,4 @@
-// Decode-shape variant of the fused int8 GEMM (few tokens, M <= 64) for sm_100a.
+// Decode-shape variant of the fused int8 GEMM (few tokens, M <= 128) for sm_100a.
 //
 //   Y[m,n] = fp16( Acc[m,n] / (c_x[m] c_w[n]) + sum_{k in O} X[m,k] W[k,n] [+ b[n]] ),  Acc = Xq Wq^T
 //
@@ -7,7 +7,8 @@
 //
 // With a handful of tokens the contraction is bound by streaming the int8
 // weight from HBM, so the operands are swapped: a 128-row tile of Wq (128
-// output columns n) takes the MMA's M slot and the MP padded tokens its N slot,
+// output columns n) takes the MMA's M slot and the MP padded tokens (16, 32,
+// 64 or 128) its N slot,
 // D^T[n, m] = sum_k Wq[n, k] Xq[m, k]  (tcgen05.mma kind::i8, 128 x MP x 32).
 //
 // Work split (stream-K): the N/128 x K/128 sequence of (n block, k block)
@@ -73,7 +74,9 @@ constexpr int DBM = 128;  // weight rows (output columns) per tile: the MMA M
 constexpr int DBK = 128;  // K bytes per stage
 // Six stages of weight tiles in flight per SM measured faster than deeper
 // rings (4: slower, 11: 12% slower): more outstanding reads only congest HBM.
+// With 128 tokens a stage holds 32 KB, and five fit.
 constexpr int D_STAGES = 6;
+constexpr int D_STAGES_128 = 5;
 constexpr int D_OUT_STAGE = 128;  // outliers whose indices are staged in smem
 constexpr int D_EPI = 256;  // epilogue threads: eight warps
 constexpr int D_THREADS = 64 + D_EPI;
@@ -83,7 +86,7 @@ struct DCfg {
   static constexpr int W_BYTES = DBM * DBK;
   static constexpr int X_BYTES = MP * DBK;
   static constexpr int STAGE = W_BYTES + X_BYTES;
-  static constexpr int STAGES = D_STAGES;
+  static constexpr int STAGES = MP > 64 ? D_STAGES_128 : D_STAGES;
   // operands of the outlier product, one chunk of kOutMma outliers, fp16,
   // K-major rows of 128 bytes with the 128-byte swizzle: A = W[O, n block]
   // (128 columns n), B = X[:, O] (MP tokens)
@@ -92,18 +95,22 @@ struct DCfg {
   static constexpr int BAR_OFF = OB_OFF + MP * 128;
   static constexpr int NBARS = 2 * STAGES + 8;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-  // the fused activation pass's slice of X, uint4 [64 rows][16 vectors]
-  static constexpr int XO_OFF = (MISC_OFF + 32 + 15) & ~15;
-  static constexpr int RX_OFF = XO_OFF + 64 * 16 * 16;             // float [64]
-  static constexpr int IDX_OFF = RX_OFF + 64 * 4;                  // int [D_OUT_STAGE]
-  static constexpr int CX_OFF = IDX_OFF + D_OUT_STAGE * 4;         // float [64]: c_x (fused)
-  static constexpr int FL_OFF = CX_OFF + 64 * 4;                   // u32 [16]: flags per vector (fused)
+  // The fused activation pass's slice of X, uint4 [MP rows][16 vectors],
+  // lives in the outlier operand blocks (16 KB + MP 128 bytes >= MP 256
+  // bytes): it is dead before the first outlier chunk is staged.
+  static constexpr int XS_OFF = OA_OFF;
+  static_assert(DBM * 128 + MP * 128 >= MP * 16 * 16, "the X slice fits the outlier operand blocks");
+  static constexpr int RX_OFF = (MISC_OFF + 32 + 15) & ~15;        // float [MP]
+  static constexpr int IDX_OFF = RX_OFF + MP * 4;                  // int [D_OUT_STAGE]
+  static constexpr int CX_OFF = IDX_OFF + D_OUT_STAGE * 4;         // float [MP]: c_x (fused)
+  static constexpr int FL_OFF = CX_OFF + MP * 4;                   // u32 [16]: flags per vector (fused)
   static constexpr int OL_OFF = FL_OFF + 16 * 4;                   // u32 [128]: the slice's outliers (fused)
   static constexpr int RED_OFF = OL_OFF + 128 * 4;                 // u32 [16]: reductions (fused)
   static constexpr int SMEM = RED_OFF + 16 * 4 + 1024;
   // TMEM: two int32 accumulators (double buffer) and the fp32 outlier
   // product, MP columns each, in a power-of-two allocation
-  static constexpr int TMEM_COLS = 3 * MP <= 32 ? 32 : (3 * MP <= 64 ? 64 : (3 * MP <= 128 ? 128 : 256));
+  static constexpr int TMEM_COLS =
+      3 * MP <= 32 ? 32 : (3 * MP <= 64 ? 64 : (3 * MP <= 128 ? 128 : (3 * MP <= 256 ? 256 : 512)));
   static constexpr uint32_t IDESC = idesc_i8(DBM, MP);
   static constexpr uint32_t IDESC_F16 = idesc_f16_f32(DBM, MP);
   static_assert(OA_OFF % 1024 == 0 && OB_OFF % 1024 == 0, "outlier operands 1024-byte aligned");
@@ -211,7 +218,7 @@ __global__ void __launch_bounds__(D_THREADS, 1)
   }
   // fused: the epilogue warps start loading their slice of X right away
   // (vectors e = et + j D_EPI of the [M][16] slice; see the activation pass)
-  constexpr int XR = 64 * 16 / D_EPI;
+  constexpr int XR = MP * 16 / D_EPI > 0 ? MP * 16 / D_EPI : 1;
   uint4 xr[XR];
   int xv0 = 0, xnv = 0;
   if constexpr (FUSED) {
@@ -376,7 +383,7 @@ __global__ void __launch_bounds__(D_THREADS, 1)
     const int et = threadIdx.x - 64;  // 0 .. D_EPI-1
     if constexpr (FUSED) {
       // ------------------------------------------ activation pass of the slice
-      uint4* xs = reinterpret_cast<uint4*>(smem + C::XO_OFF);  // [64][16] (aliases xo_s)
+      uint4* xs = reinterpret_cast<uint4*>(smem + C::XS_OFF);  // [MP][16] (in the outlier operand blocks)
       uint32_t* fl_s = reinterpret_cast<uint32_t*>(smem + C::FL_OFF);
       uint32_t* ol_s = reinterpret_cast<uint32_t*>(smem + C::OL_OFF);
       uint32_t* red_s = reinterpret_cast<uint32_t*>(smem + C::RED_OFF);
@@ -781,13 +788,14 @@ cudaError_t launch_decode_f(const CUtensorMap& tmW, const CUtensorMap& tmX, cons
   switch (decode_padded_tokens(a.M)) {
     case 16: return launch_decode_t<16, FUSED>(tmW, tmX, a, num_sms, pdl, stream);
     case 32: return launch_decode_t<32, FUSED>(tmW, tmX, a, num_sms, pdl, stream);
-    default: return launch_decode_t<64, FUSED>(tmW, tmX, a, num_sms, pdl, stream);
+    case 64: return launch_decode_t<64, FUSED>(tmW, tmX, a, num_sms, pdl, stream);
+    default: return launch_decode_t<128, FUSED>(tmW, tmX, a, num_sms, pdl, stream);
   }
 }
 
 }  // namespace
 
-int decode_padded_tokens(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
+int decode_padded_tokens(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
 
 bool decode_fused_fits(int64_t M, int64_t K, int64_t N, int num_sms) {
   if (M < 1 || M > kDecodeMaxM || K < 16 || K % 16 != 0 || N < 1 || num_sms < 1) return false;

@@ -111,7 +111,7 @@ cudaError_t launch_gemm_decomp(const CUtensorMap& tmA, const CUtensorMap& tmB, c
 // Largest K any kernel here accepts (the row kernels keep a row in registers).
 constexpr int64_t kMaxK = 65536;
 // Forwards with at most this many rows take the decode GEMM.
-constexpr int kDecodeMaxM = 64;
+constexpr int kDecodeMaxM = 128;
 
 // ---- activation pass in one launch --------------------------------------
 // Detection, quantisation and the outlier gather (csrc/xact_rows.cu) for K <=
@@ -148,7 +148,7 @@ int half_magnitude_threshold(float alpha);
 bool row_act_fits(int64_t M, int64_t K, int num_sms);
 cudaError_t launch_row_act(const RowActArgs& a, int num_sms, cudaStream_t stream);
 
-// ---- decode-shape GEMM (M <= 64 tokens) -----------------------------------
+// ---- decode-shape GEMM (M <= 128 tokens) ----------------------------------
 struct DecodeArgs {
   int M, N, K;
   int N_pad;               // rows per k block in the weight layout
@@ -162,7 +162,7 @@ struct DecodeArgs {
   __half* Y;               // [M,N]
   const __half* bias;      // [N] or nullptr
   int32_t* acc_dump;       // [M,N] or nullptr
-  int32_t* part;           // [64][N] int32 partial sums, zero between launches
+  int32_t* part;           // [kDecodeMaxM][N] int32 partial sums, zero between launches
   unsigned* ticket;        // [ceil(N/128)] k-steps done per n block, zero between launches
   int* status;
   unsigned long long timeout_ns;
@@ -188,7 +188,7 @@ struct DecodeArgs {
 // Words between the rows of DecodeArgs::rowmax: one 128-byte line per row,
 // so that the CTAs' atomics on different rows do not queue on one line.
 constexpr int kRowMaxStride = 32;
-// Tokens padded to the MMA N of the decode kernel: 16, 32 or 64.
+// Tokens padded to the MMA N of the decode kernel: 16, 32, 64 or 128.
 int decode_padded_tokens(int64_t M);
 // Whether the decode kernel can run the activation pass itself for M x K
 // against N columns: every CTA's slice of X must hold at most 16 vectors of

@@ -84,20 +84,22 @@ SHAPES = [
     (1, 16, 16, 0, 6.0),
     (3, 48, 48, 1, 6.0),
     (17, 256, 272, 2, 6.0),
-    (128, 128, 256, 3, 6.0),
-    (129, 272, 528, 4, 6.0),
+    (128, 128, 256, 3, 6.0),        # decode kernel, 128 tokens
+    (129, 272, 528, 4, 6.0),        # smallest prefill-kernel M
     (300, 1040, 784, 5, 6.0),
     (257, 384, 512, 7, math.inf),   # pure vector-wise int8
     (64, 512, 256, 6, 0.0),         # every non-zero column is an outlier
     (33, 4096, 1024, 7, 6.0),
     (130, 2064, 2320, 9, 6.0),
     (513, 640, 4112, 3, 6.0),       # many N tiles, ragged N tail
-    (64, 1040, 784, 3, 6.0),        # largest decode-kernel M, ragged 128-column blocks
-    (65, 1040, 784, 3, 6.0),        # smallest prefill-kernel M
+    (64, 1040, 784, 3, 6.0),        # 64 tokens, ragged 128-column blocks
+    (65, 1040, 784, 3, 6.0),        # 65 tokens: padded to 128
+    (128, 1040, 784, 70, 6.0),      # largest decode-kernel M, two outlier chunks
     (40, 2048, 4112, 5, 6.0),       # decode kernel, stream-K splits across blocks
     (8, 12288, 1024, 7, 6.0),       # decode, long K: whole and split blocks
-    (96, 512, 256, 6, 0.0),         # alpha = 0 on the single-launch activation pass
-    (100, 256, 128, 0, -1.0),       # alpha < 0: every column is an outlier
+    (196, 512, 256, 6, 0.0),        # alpha = 0 on the single-launch activation pass
+    (100, 256, 128, 0, -1.0),       # alpha < 0: every column is an outlier (decode kernel)
+    (300, 256, 128, 0, -1.0),       # alpha < 0 on the single-launch activation pass
     (300, 16, 32, 1, 6.0),          # smallest K, three rows per block
     (149, 32768, 256, 3, 6.0),      # largest K of the single-launch pass, one row per block
     (3000, 5120, 256, 7, 6.0),      # 21 rows (210 KB) of X per block
@@ -194,7 +196,7 @@ BIAS_SHAPES = [
     # M, K, N, planted outliers, alpha
     (300, 1040, 784, 5, 6.0),      # CTA pairs: bias joins the tensor-core outlier product
     (257, 384, 512, 3, math.inf),  # CTA pairs, no outliers: direct epilogue
-    (100, 512, 272, 4, 6.0),       # single CTAs: FMA epilogue, ragged N tail
+    (100, 512, 272, 4, 6.0),       # decode kernel, 128 tokens, ragged N tail
     (8, 2048, 1168, 4, 6.0),       # decode kernel with split n blocks
     (40, 1040, 784, 0, 6.0),       # decode kernel, no outliers
 ]
@@ -223,7 +225,7 @@ SPLIT_SHAPES = [
     (257, 2048, 512, 3, math.inf, 3),   # no outliers: the partials join the direct epilogue
     (513, 4096, 1040, 7, 6.0, 4),       # several tiles per pair, owners waiting on other pairs
     (130, 384, 256, 2, 6.0, 4),         # three k-blocks: the split is capped at 3
-    (513, 2048, 512, 80, 6.0, 2),       # more than 64 outliers: FMA tail on the owner
+    (513, 2048, 512, 80, 6.0, 2),       # more than 64 outliers: two chunks of the product on the owner
     (1000, 2048, 256, 4, 0.0, 3),       # alpha = 0: the int8 partials are all zero
 ]
 
@@ -469,8 +471,8 @@ def test_launches_per_forward():
     w = m.int8mm_prepare_weight(W)
     assert m.int8mm_launches_per_forward(w, 0) == 0
     assert m.int8mm_launches_per_forward(w, 1) == 1       # decode GEMM with its own activation pass
-    assert m.int8mm_launches_per_forward(w, 64) == 1
-    assert m.int8mm_launches_per_forward(w, 65) == 2      # activation pass + CTA-pair GEMM
+    assert m.int8mm_launches_per_forward(w, 128) == 1
+    assert m.int8mm_launches_per_forward(w, 129) == 2     # activation pass + CTA-pair GEMM
     assert m.int8mm_launches_per_forward(w, 2048) == 2    # activation pass + CTA-pair GEMM
     assert m.int8mm_launches_per_forward(w, 4096) == 2    # more rows per block than row slots
     w2 = m.int8mm_prepare_weight(torch.from_numpy(workloads.weight(40960, 256, 44)).to(dev()))
@@ -499,7 +501,7 @@ def test_single_launch_pass_many_generations():
 
 
 FUSED_SHAPES = [
-    # M, K, N, planted outliers, alpha: decode shapes (M <= 64, K <= 16384)
+    # M, K, N, planted outliers, alpha: decode shapes (M <= 128, K <= 16384)
     (1, 4096, 1024, 3, 6.0),
     (16, 8192, 2048, 7, 6.0),
     (33, 12288, 1040, 7, 6.0),       # ragged 128-column block
@@ -509,6 +511,8 @@ FUSED_SHAPES = [
     (5, 384, 128, 2, -1.0),          # alpha < 0: every column is an outlier
     (9, 1040, 784, 4, math.inf),     # pure vector-wise
     (2, 16, 16, 1, 6.0),             # one CTA, a 2-vector slice
+    (128, 8192, 1024, 7, 6.0),       # 128 tokens
+    (97, 16384, 512, 130, 6.0),      # 128 padded tokens, 16-vector slices, three outlier chunks
 ]
 
 
@@ -540,7 +544,7 @@ def test_decode_and_prefill_forwards_share_the_barrier_state():
     W = workloads.weight(K, N, 91)
     w = m.int8mm_prepare_weight(torch.from_numpy(W).to(dev()))
     wq = oracle.quantize_cols(W)
-    runs = [(40, 5), (300, 2), (8, 0), (8, 3), (2048, 7), (1, 1), (64, 4), (200, 0), (16, 6), (16, 6)]
+    runs = [(40, 5), (300, 2), (8, 0), (8, 3), (2048, 7), (1, 1), (128, 4), (200, 0), (16, 6), (100, 6)]
     counts = []
     for i, (M, n_out) in enumerate(runs):
         p = workloads.small(M, K, N, n_out, seed=700 + i)
@@ -561,7 +565,7 @@ def test_decode_and_prefill_forwards_share_the_barrier_state():
     assert m.int8mm_get_status(w) == m.INT8MM_OK
 
 
-@pytest.mark.parametrize("M", [1, 16, 40])
+@pytest.mark.parametrize("M", [1, 16, 40, 128])
 def test_decode_repeat_and_stale_partials(M):
     # split n blocks leave int32 partial sums and tickets behind for the next call
     K, N = 2048, 1168
