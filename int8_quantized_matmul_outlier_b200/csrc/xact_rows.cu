@@ -26,8 +26,8 @@
 //      the columns outside O, and equal to it unless S_i is reached in an
 //      outlier column not flagged yet;
 //   3. writes c_x[i] = 127 / S_i and the codes of every column with it.
-// A block quantises no row before four of its rows are flagged (all of
-// them, if it has fewer), so in the pages' activations (a few outlier
+// A block quantises no row before four of its rows are flagged (fewer if it
+// has fewer rows or row groups), so in the pages' activations (a few outlier
 // columns, large in most rows) the block's bitmask already holds the outlier
 // columns when the rows are quantised; rows are quantised as they land.
 // Then the block ORs its bitmask into a global one and meets the other
@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) xact_rows_kernel(RowActArgs
   __shared__ uint32_t s_gen;
   __shared__ int s_ok, s_count;
   __shared__ int s_flagged;  // rows of the block flagged so far
+  __shared__ int s_marked;   // a row is marked for step 5
 
   // The GEMM that follows may launch now; its blocks take the SMs this
   // kernel leaves.
@@ -107,7 +108,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) xact_rows_kernel(RowActArgs
   }
   for (int w = tid; w < KW; w += NT) mask_s[w] = 0u;
   for (int i = tid; i < R; i += NT) redo_s[i] = 0u;
-  if (tid == 0) s_flagged = 0;
+  if (tid == 0) {
+    s_flagged = 0;
+    s_marked = 0;
+  }
   __syncthreads();
 
   // ------------------------------------------------------------- phase 1
@@ -167,11 +171,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) xact_rows_kernel(RowActArgs
   };
   if (leader && my_rows > 0) issue(0);
   // Rows are quantised as they land, but only once the block has flagged
-  // kFirstRows rows (or all of its rows, if fewer): the outlier columns then
-  // show in the block's bitmask (in the pages' activations an outlier column
-  // is large in most rows), so S_i below leaves them out and rarely needs
-  // the correction after the barrier.
-  const int need_flagged = min(nr, kFirstRows);
+  // kFirstRows rows (fewer if it has fewer rows or row groups: before the
+  // wait ends, only each group's first row can be flagged): the outlier
+  // columns then show in the block's bitmask (in the pages' activations an
+  // outlier column is large in most rows), so S_i below leaves them out and
+  // rarely needs the correction after the barrier.
+  const int need_flagged = min(min(nr, G), kFirstRows);
   int ok = 1;
   for (int j = 0; j < my_rows && ok; ++j) {
     const int lr = g + j * G;
@@ -337,32 +342,42 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) xact_rows_kernel(RowActArgs
         a.X_OT[static_cast<size_t>(o) * a.ld_xo + r0 + r] = __ushort_as_half(x[u]);
         a.Xq[static_cast<size_t>(r0 + r) * K + cols[o]] = 0;
         const uint32_t mag = x[u] & 0x7fffu;
-        if (!all_out && mag <= static_cast<uint32_t>(a.thr) && mag == smax_s[r]) redo_s[r] = 1u;
+        if (!all_out && mag <= static_cast<uint32_t>(a.thr) && mag == smax_s[r]) {
+          redo_s[r] = 1u;
+          s_marked = 1;
+        }
       }
     }
   }
   __syncthreads();
-  // (5) marked rows: the exact absmax over the columns outside O, c_x and
-  //     the codes again (outlier columns 0)
-  for (int lr = warp; lr < nr; lr += NW) {
-    if (smax_s[lr] == 0u || redo_s[lr] == 0u) continue;  // warp-uniform
+  // (5) marked rows, one at a time with the whole block (a row's vectors
+  //     spread over all threads, so that its loads are in flight together;
+  //     one warp per row took ~16 us for a row): the exact absmax over the
+  //     columns outside O, c_x and the codes again (outlier columns 0)
+  for (int lr = 0; s_marked && lr < nr; ++lr) {
+    if (smax_s[lr] == 0u || redo_s[lr] == 0u) continue;  // block-uniform
     const uint4* xr = reinterpret_cast<const uint4*>(a.X + static_cast<size_t>(r0 + lr) * K);
     uint32_t m = 0u;
-    for (int v = lane; v < nvec; v += 32) {
+    for (int v = tid; v < nvec; v += NT) {
       const uint32_t fl = (mask_s[v >> 2] >> ((v & 3) * 8)) & 0xffu;
       m = masked_absmax2(m, __ldg(xr + v), fl);
     }
-    const uint32_t S2 = __reduce_max_sync(0xffffffffu, max_pair(m));
+    m = __reduce_max_sync(0xffffffffu, max_pair(m));
+    if (lane == 0) red_s[warp] = m;
+    __syncthreads();
+    uint32_t S2 = 0u;
+    for (int u = 0; u < NW; ++u) S2 = max(S2, red_s[u]);
     const float c = scale_from_absmax_bits(S2);
     int8_t* qrow = a.Xq + static_cast<size_t>(r0 + lr) * K;
-    for (int v = lane; v < nvec; v += 32) {
+    for (int v = tid; v < nvec; v += NT) {
       const uint32_t fl = (mask_s[v >> 2] >> ((v & 3) * 8)) & 0xffu;
       uint2 q = quant8_fma(__ldg(xr + v), c);
       q.x &= ~expand_nibble(fl & 0xfu);
       q.y &= ~expand_nibble(fl >> 4);
       *reinterpret_cast<uint2*>(qrow + static_cast<size_t>(v) * 8) = q;
     }
-    if (lane == 0) a.c_x[r0 + lr] = c;
+    if (tid == 0) a.c_x[r0 + lr] = c;
+    __syncthreads();  // red_s is reused by the next marked row
   }
 }
 

@@ -106,6 +106,8 @@ SHAPES = [
     (4000, 5120, 256, 5, 6.0),      # streamed: 28 rows per block in chunks of 10, a short last chunk
     (600, 20480, 256, 7, 6.0),      # streamed, two 40 KB rows per chunk
     (130, 40960, 256, 3, 6.0),      # 80 KB rows: one row slot per block
+    (300, 40960, 256, 5, 6.0),      # three rows per block, two row slots: the first-rows count stops at two
+    (600, 4096, 256, 160, 6.0),     # 160 outlier columns: three chunks of the product
     (3, 65536, 32, 2, 6.0),         # largest K: a 128 KB row slot
     (38000, 32, 16, 2, 6.0),        # more than 256 rows per SM: two-kernel activation path
 ]
@@ -151,6 +153,17 @@ def test_threshold_ties_single_launch_pass():
     p.X[0, 63] = -100
     out = check(p)
     assert out["cnt"] == 2
+
+
+@pytest.mark.parametrize("M,K,frac", [(2000, 1024, 0.002), (4000, 2048, 0.01), (300, 1040, 0.05)])
+def test_outlier_columns_the_first_rows_miss(M, K, frac):
+    # outlier columns large in few rows: most blocks flag them only after
+    # they start quantising, so rows are quantised with them unflagged and
+    # the pass after the barrier zeroes their codes and requantises the
+    # rows whose absmax they held
+    p = workloads.small(M, K, 256, 6, seed=M + K, row_fraction=frac)
+    out = check(p, rows=sample_rows(M, 64, seed=3))
+    assert out["cnt"] == 6
 
 
 @pytest.mark.parametrize("M,K", [(300, 1040), (2048, 5120), (4000, 5120)])
