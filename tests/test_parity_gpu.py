@@ -634,17 +634,20 @@ def test_reserve_then_forwards_allocate_nothing(split):
     m.int8mm_free(w)
 
 
-def test_captured_forward_replays_like_the_eager_one():
-    # a CTA-pair forward (single-launch activation pass + GEMM as its
-    # programmatic dependent) captured in a CUDA graph after int8mm_reserve;
-    # each replay on new activations equals the eager forward
-    p = workloads.small(300, 1040, 784, 5, seed=71)
+@pytest.mark.parametrize("M", [300, 16, 128])
+def test_captured_forward_replays_like_the_eager_one(M):
+    # a forward captured in a CUDA graph after int8mm_reserve: CTA pairs
+    # (single-launch activation pass + GEMM as its programmatic dependent,
+    # M = 300) or the decode kernel with its own activation pass (one
+    # cooperative launch, M = 16 and 128); each replay on new activations
+    # equals the eager forward
+    p = workloads.small(M, 1040, 784, 5, seed=71)
     X = torch.from_numpy(p.X).to(dev())
     W = torch.from_numpy(p.W).to(dev())
     w = m.int8mm_prepare_weight(W)
-    m.int8mm_reserve(w, 300)
+    m.int8mm_reserve(w, M)
     Xs = X.clone()
-    Ys = torch.empty((300, 784), dtype=torch.float16, device=dev())
+    Ys = torch.empty((M, 784), dtype=torch.float16, device=dev())
     m.int8mm_forward(w, Xs, p.alpha, Ys)  # warm-up outside the capture
     torch.cuda.synchronize()
     held = m.int8mm_weight_bytes(w)
@@ -653,7 +656,7 @@ def test_captured_forward_replays_like_the_eager_one():
         m.int8mm_forward(w, Xs, p.alpha, Ys)
     assert m.int8mm_weight_bytes(w) == held
     for seed in (72, 73):
-        q = workloads.small(300, 1040, 784, 5, seed=seed)
+        q = workloads.small(M, 1040, 784, 5, seed=seed)
         Xn = torch.from_numpy(q.X).to(dev())
         Xs.copy_(Xn)
         g.replay()
