@@ -265,8 +265,8 @@ def test_split_k(M, K, N, n_out, alpha, split):
 
 def test_split_of_the_leftover_tiles_only():
     # 8 x 10 = 80 tiles for 74 pairs: the library runs 74 tiles whole and
-    # cuts the 6 left over into pieces spread over all pairs
-    p = workloads.small(2048, 4096, 2560, 5, seed=91)
+    # cuts the 6 left over into pieces (of 24 k-blocks) spread over all pairs
+    p = workloads.small(2048, 6144, 2560, 5, seed=91)
     out = check(p, rows=sample_rows(2048, 64, seed=91))
     assert out["cnt"] == 5
     w = out["w"]
